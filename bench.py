@@ -1,0 +1,352 @@
+"""Benchmark of the MLA absorb decode step on B200.
+
+One step = the whole hot path on one batch: mla_absorb_q -> mla_attn_decode
+(split-t + combine) -> mla_out_proj, for the DeepSeek-V3 decode workload
+(batch 8, 128 heads, kv_lora_rank 512, rope 64, one query per sequence,
+4096 cached tokens each), seeded synthetic inputs resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line.  `value` is microseconds per step (lower is better),
+the max over ranks; with N > 1 every rank runs an independent replica (the
+path has no cross-GPU exchange).  L2 is flushed (a 256 MiB write) before every
+timed step, outside the timed events.  `--impl reference` times the fp64 CPU
+oracle on the host cores instead, one (sequence, head) pair per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA absorb decode µs/step & cache GB/s, TFLOP/s as % of roofline (1×B200)"
+UNIT = "us/step"
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+KV_BYTES_PER_TOKEN = (512 + 64) * 2            # latent + rotary key, bf16
+FLOP_PER_TOKEN_PER_HEAD = 2 * (576 + 512)      # score and value products
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", type=int, default=1, help="workload index (1 = DeepSeek-V3 decode b8 t4096)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0)
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "deepseek_mla_latent_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload_name: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary,
+    if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", f"attn_decode_{workload_name}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        self.gpu_id = gpu_id
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline_oracle(w, seconds: float):
+    """Time the fp64 oracle (naive path) on (sequence, head) pairs of the workload for
+    about `seconds`, and scale to one whole step (all sequences x all heads)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count() or 1
+    H, B = w.dims.heads, w.batch
+    pairs = [(b, h) for h in range(H) for b in range(B)]
+    done, t0 = 0, time.perf_counter()
+    while done < len(pairs) and (done < 4 or time.perf_counter() - t0 < seconds):
+        oracle.workload_naive(w, pairs=[pairs[done]])
+        done += 1
+    el = time.perf_counter() - t0
+    per_pair = el / done
+    return {"value": per_pair * len(pairs) * 1e6, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"{done} of {len(pairs)} (sequence, head) pairs of the same workload, naive fp64 path, "
+                      f"{el:.1f} s, scaled to the whole step"}
+
+
+def run_reference(args, rank, world):
+    from deepseek_mla_latent_b200 import workloads as wl
+    if rank != 0:
+        return
+    w = wl.workload(args.workload)
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count() or 1
+    H, B = w.dims.heads, w.batch
+    pairs = [(b, h) for h in range(H) for b in range(B)]
+    for i in range(args.warmup):
+        oracle.workload_naive(w, pairs=[pairs[i % len(pairs)]])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.workload_naive(w, pairs=[pairs[i % len(pairs)]])
+    el = time.perf_counter() - t0
+    us_step = el / args.steps * len(pairs) * 1e6
+    line = {"metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": us_step / 1e3, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "batch": B, "heads": H, "seq_len_k": max(w.seqlens_k),
+                       "queries_per_seq": 1, "parallelism": "replicas"},
+            "cpu_baseline": {"value": us_step, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+                             "sample": f"each step: one (sequence, head) pair of {len(pairs)}, naive fp64 path, "
+                                       "scaled to the whole step"},
+            "e2e": {"value": us_step, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from deepseek_mla_latent_b200 import mla
+    from deepseek_mla_latent_b200 import workloads as wl
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    w = wl.workload(args.workload)
+    d = mla.dims_from(w.dims)
+    dt = torch.bfloat16 if w.dims.dtype == "bf16" else torch.float32
+    T = lambda a: torch.from_numpy(a).to(device=dev, dtype=dt)
+    q, kv, pe, wkv_b = T(w.q), T(w.kv), T(w.pe), T(w.wkv_b)
+    cu_k = torch.from_numpy(w.cu_seqlens_k).to(dev)
+    B, H, C, Dv = w.batch, w.dims.heads, w.dims.kv_lora_rank, w.dims.v_head
+    max_k = max(w.seqlens_k)
+    bufs = {"q_abs": torch.empty((B, H, C), dtype=dt, device=dev),
+            "o_lat": torch.empty((B, H, C), dtype=dt, device=dev),
+            "out": torch.empty((B, H, Dv), dtype=dt, device=dev),
+            "ws": mla.workspace(d, B, B, max_k, 0, device=dev)}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        q_abs = mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
+        ev_a0.record(stream)
+        o_lat = mla.attn_decode(d, q_abs, q, kv, pe, cu_k, max_k, bufs["o_lat"], bufs["ws"])
+        ev_a1.record(stream)
+        return mla.out_proj(d, o_lat, wkv_b, bufs["out"])
+
+    n_ev = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_as = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_ae = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+
+    ev_a0, ev_a1 = ev_as[0], ev_ae[0]
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    mla.device_status()
+
+    sampler = None
+    if rank == 0:
+        try:
+            gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
+            gpu_id = gpu_id if gpu_id.startswith("GPU-") else "GPU-" + gpu_id
+        except Exception:  # noqa: BLE001
+            gpu_id = str(local)
+        sampler = ClockSampler(gpu_id)
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev_a0, ev_a1 = ev_as[i], ev_ae[i]
+        ev_s[i].record(stream)
+        step()
+        ev_e[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    mla.device_status()
+
+    step_ms = [s.elapsed_time(e) for s, e in zip(ev_s, ev_e)]
+    attn_ms = [s.elapsed_time(e) for s, e in zip(ev_as, ev_ae)]
+    total_ms = sum(step_ms)
+    mean_attn_ms = sum(attn_ms) / len(attn_ms)
+    if world > 1:
+        t = torch.tensor([total_ms, mean_attn_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, mean_attn_ms = float(t[0]), float(t[1])
+    us_step = total_ms / args.steps * 1e3
+
+    # End to end through the same public calls: pinned host q -> device, step, out -> pinned host.
+    q_host = w.q if dt == torch.float32 else None
+    q_pinned = torch.from_numpy(w.q).to(dt).pin_memory()
+    out_pinned = torch.empty((B, H, Dv), dtype=dt).pin_memory()
+    q_dev = torch.empty_like(q)
+    e2e_steps = min(args.steps, 500)
+    e2e_s = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e2e_e = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    for i in range(e2e_steps):
+        flush.zero_()
+        e2e_s[i].record(stream)
+        q_dev.copy_(q_pinned, non_blocking=True)
+        q_abs = mla.absorb_q(d, q_dev, wkv_b, bufs["q_abs"])
+        o_lat = mla.attn_decode(d, q_abs, q_dev, kv, pe, cu_k, max_k, bufs["o_lat"], bufs["ws"])
+        out = mla.out_proj(d, o_lat, wkv_b, bufs["out"])
+        out_pinned.copy_(out, non_blocking=True)
+        e2e_e[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_us = e2e_ms / e2e_steps * 1e3
+    del q_host
+
+    if rank == 0:
+        hbm, tf, peak_kind = load_peaks()
+        tokens = w.total_k
+        alg_bytes = tokens * KV_BYTES_PER_TOKEN + B * H * (C + w.dims.qk_rope + C) * 2
+        alg_flop = tokens * H * FLOP_PER_TOKEN_PER_HEAD
+        attn_s = mean_attn_ms / 1e3
+        achieved_gbs = alg_bytes / attn_s / 1e9
+        traffic = profiled_traffic(w.name)
+        line = {
+            "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": us_step / 1e3, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "batch": B, "heads": H, "kv_lora_rank": C, "qk_rope": w.dims.qk_rope,
+                       "seq_len_k": max_k, "queries_per_seq": 1, "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+            "tokens_per_s": world * B / (us_step / 1e6),
+            "attn_kernel_us": mean_attn_ms * 1e3,
+            "attn_cache_gbs": achieved_gbs,
+            "attn_tflops": alg_flop / attn_s / 1e12,
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved_gbs / hbm, "traffic": traffic, "peak_kind": peak_kind,
+                         "tensor_frac": alg_flop / attn_s / 1e12 / tf},
+            "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": int(q_pinned.numel() * q_pinned.element_size()),
+                    "d2h_bytes_per_step": int(out_pinned.numel() * out_pinned.element_size())},
+            "gpu_launches": None,
+            "clocks": clocks,
+            "kernel_family": mla.kernel_family(d),
+            "kernel_source_hash": kernel_source_hash(),
+        }
+        # absorb_q + attention + (merge when split) + out_proj, each one launch of ours
+        splits = mla.decode_num_splits(d, B, max_k, 0)
+        line["gpu_launches"] = args.steps * (3 + (1 if splits > 1 else 0))
+        line["config"]["num_splits"] = splits
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_oracle(w, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,285 @@
+// mla_lib.cu -- the C ABI declared in include/mla.h: argument checks, kernel
+// choice, workspace layout and launches.  Every arithmetic step runs in the
+// kernels included below; this file only marshals.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "mla.h"
+#include "common.cuh"
+#include "simt.cuh"
+#include "sm100.cuh"
+
+namespace {
+
+using mla_bf16 = __nv_bfloat16;
+
+struct Geo {
+  int H, C, Dn, R, Dv;
+  bool bf16;
+  float scale;
+  int family;   // 1 tensor-core kernels, 0 CUDA-core kernels, -1 unsupported
+};
+
+int pick_family(const mla_dims_t* d) {
+  if (!d) return -1;
+  if (d->num_heads <= 0 || d->kv_lora_rank <= 0 || d->qk_nope_head_dim <= 0 || d->qk_rope_head_dim < 0 ||
+      d->v_head_dim <= 0)
+    return -1;
+  if (d->dtype != MLA_DTYPE_BF16 && d->dtype != MLA_DTYPE_F32) return -1;
+  if (d->dtype == MLA_DTYPE_BF16 && mla::sm100::supports(d->num_heads, d->kv_lora_rank, d->qk_nope_head_dim,
+                                                          d->qk_rope_head_dim, d->v_head_dim))
+    return 1;
+  if (d->kv_lora_rank > mla::simt::kMaxC || d->qk_rope_head_dim > mla::simt::kMaxR ||
+      d->qk_nope_head_dim > mla::simt::kMaxD || d->v_head_dim > mla::simt::kMaxD || d->num_heads > 1024)
+    return -1;
+  return 0;
+}
+
+bool geo_of(const mla_dims_t* d, Geo* g) {
+  g->family = pick_family(d);
+  if (g->family < 0) return false;
+  g->H = d->num_heads; g->C = d->kv_lora_rank; g->Dn = d->qk_nope_head_dim;
+  g->R = d->qk_rope_head_dim; g->Dv = d->v_head_dim;
+  g->bf16 = d->dtype == MLA_DTYPE_BF16;
+  g->scale = d->softmax_scale;
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mla_status_t launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int device_sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// ---- split-t planning (CUDA-core kernels) ----------------------------------
+int simt_auto_splits(int64_t n_q_rows, int H, int64_t max_seqlen_k) {
+  const int64_t blocks = n_q_rows * H;
+  const int64_t want = 4LL * device_sm_count();
+  int splits = 1;
+  while (splits < 64 && blocks * splits < want && max_seqlen_k / (splits * 2) >= 1024) splits *= 2;
+  return splits;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t simt_workspace(const Geo& g, int64_t n_q_rows, int splits) {
+  if (splits <= 1) return 0;
+  return align256((size_t)splits * n_q_rows * g.H * g.C * sizeof(float)) +
+         align256((size_t)splits * n_q_rows * g.H * 2 * sizeof(float));
+}
+
+template <typename T>
+mla_status_t simt_attention(const Geo& g, const void* q_abs, const void* q, int64_t q_row_stride,
+                            const void* kv, const void* pe, const int32_t* cu_q, const int32_t* cu_k, int batch,
+                            int64_t n_rows, int splits, void* o_lat, void* ws, cudaStream_t stream) {
+  float* part_o = nullptr;
+  float* part_ml = nullptr;
+  if (splits > 1) {
+    part_o = static_cast<float*>(ws);
+    part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                       align256((size_t)splits * n_rows * g.H * g.C * sizeof(float)));
+  }
+  dim3 grid((unsigned)n_rows, g.H, splits);
+  size_t smem = (size_t)(2 * g.C + g.R + mla::simt::kThreads + 32) * sizeof(float);
+  mla::simt::attn_kernel<T><<<grid, mla::simt::kThreads, smem, stream>>>(
+      static_cast<const T*>(q_abs), static_cast<const T*>(q), q_row_stride, static_cast<const T*>(kv),
+      static_cast<const T*>(pe), cu_q, cu_k, batch, n_rows, g.H, g.C, g.R, g.Dn, g.scale, splits,
+      static_cast<T*>(o_lat), part_o, part_ml);
+  if (splits > 1) {
+    mla::simt::combine_kernel<T><<<dim3((unsigned)n_rows, g.H), mla::simt::kThreads, 0, stream>>>(
+        part_o, part_ml, splits, n_rows, g.H, g.C, static_cast<T*>(o_lat));
+  }
+  return launch_status();
+}
+
+int resolve_splits(const Geo& g, int32_t batch, int64_t n_q_rows, int64_t max_seqlen_k, int32_t num_splits,
+                   bool decode) {
+  if (!decode) return g.family == 1 ? mla::sm100::prefill_splits() : 1;
+  if (num_splits > 0) return num_splits;
+  if (g.family == 1) return mla::sm100::auto_decode_splits(batch, max_seqlen_k, device_sm_count());
+  return simt_auto_splits(n_q_rows, g.H, max_seqlen_k);
+}
+
+size_t workspace_bytes_for(const Geo& g, int32_t batch, int64_t n_q_rows, int64_t max_seqlen_k, int splits,
+                           bool decode) {
+  if (g.family == 1) return mla::sm100::workspace_bytes(g.H, g.C, batch, n_q_rows, max_seqlen_k, splits, decode);
+  return simt_workspace(g, n_q_rows, splits);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t mla_api_version(void) { return MLA_API_VERSION; }
+
+int32_t mla_kernel_family(const mla_dims_t* dims) { return pick_family(dims); }
+
+const char* mla_status_string(mla_status_t s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported head geometry or dtype";
+    case MLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_DEVICE_TIMEOUT: return "a bounded device wait ran out";
+  }
+  return "unknown status";
+}
+
+mla_status_t mla_absorb_q(const mla_dims_t* dims, const void* q, int64_t q_row_stride, const void* wkv_b,
+                          void* q_abs, int64_t n_rows, cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (n_rows < 0 || q_row_stride < (int64_t)g.H * (g.Dn + g.R)) return MLA_ERR_INVALID_ARG;
+  if (n_rows == 0) return MLA_OK;
+  if (!q || !wkv_b || !q_abs || !aligned16(q) || !aligned16(wkv_b) || !aligned16(q_abs)) return MLA_ERR_INVALID_ARG;
+  if (g.family == 1) {
+    if ((q_row_stride * 2) % 16 != 0) return MLA_ERR_INVALID_ARG;
+    return mla::sm100::absorb_q(q, q_row_stride, wkv_b, q_abs, n_rows, g.H, stream);
+  }
+  dim3 grid((unsigned)((n_rows + mla::simt::kRowsPerBlock - 1) / mla::simt::kRowsPerBlock), g.H);
+  if (g.bf16)
+    mla::simt::absorb_q_kernel<mla_bf16><<<grid, mla::simt::kThreads, 0, stream>>>(
+        static_cast<const mla_bf16*>(q), q_row_stride, static_cast<const mla_bf16*>(wkv_b),
+        static_cast<mla_bf16*>(q_abs), n_rows, g.H, g.C, g.Dn, g.R, g.Dv);
+  else
+    mla::simt::absorb_q_kernel<float><<<grid, mla::simt::kThreads, 0, stream>>>(
+        static_cast<const float*>(q), q_row_stride, static_cast<const float*>(wkv_b), static_cast<float*>(q_abs),
+        n_rows, g.H, g.C, g.Dn, g.R, g.Dv);
+  return launch_status();
+}
+
+mla_status_t mla_out_proj(const mla_dims_t* dims, const void* o_lat, const void* wkv_b, void* out, int64_t n_rows,
+                          cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (n_rows < 0) return MLA_ERR_INVALID_ARG;
+  if (n_rows == 0) return MLA_OK;
+  if (!o_lat || !wkv_b || !out || !aligned16(o_lat) || !aligned16(wkv_b) || !aligned16(out))
+    return MLA_ERR_INVALID_ARG;
+  if (g.family == 1) return mla::sm100::out_proj(o_lat, wkv_b, out, n_rows, g.H, stream);
+  dim3 grid((unsigned)((n_rows + mla::simt::kRowsPerBlock - 1) / mla::simt::kRowsPerBlock), g.H);
+  size_t smem = (size_t)mla::simt::kRowsPerBlock * g.C * sizeof(float);
+  if (g.bf16)
+    mla::simt::out_proj_kernel<mla_bf16><<<grid, mla::simt::kThreads, smem, stream>>>(
+        static_cast<const mla_bf16*>(o_lat), static_cast<const mla_bf16*>(wkv_b), static_cast<mla_bf16*>(out),
+        n_rows, g.H, g.C, g.Dn, g.Dv);
+  else
+    mla::simt::out_proj_kernel<float><<<grid, mla::simt::kThreads, smem, stream>>>(
+        static_cast<const float*>(o_lat), static_cast<const float*>(wkv_b), static_cast<float*>(out), n_rows, g.H,
+        g.C, g.Dn, g.Dv);
+  return launch_status();
+}
+
+size_t mla_workspace_size(const mla_dims_t* dims, int32_t batch, int64_t n_q_rows, int64_t max_seqlen_k,
+                          int32_t num_splits) {
+  Geo g;
+  if (!dims || !geo_of(dims, &g) || batch < 0 || n_q_rows < 0 || max_seqlen_k < 0 || num_splits < 0) return 0;
+  // A decode call has exactly one query row per sequence.
+  const bool decode = n_q_rows == batch;
+  const int splits = resolve_splits(g, batch, n_q_rows, max_seqlen_k, num_splits, decode);
+  size_t a = workspace_bytes_for(g, batch, n_q_rows, max_seqlen_k, splits, decode);
+  if (decode) {
+    // the same sizes may also be served as a chunked prefill
+    size_t b = workspace_bytes_for(g, batch, n_q_rows, max_seqlen_k,
+                                   resolve_splits(g, batch, n_q_rows, max_seqlen_k, 0, false), false);
+    a = std::max(a, b);
+  }
+  return a;
+}
+
+int32_t mla_decode_num_splits(const mla_dims_t* dims, int32_t batch, int64_t max_seqlen_k, int32_t num_splits) {
+  Geo g;
+  if (!dims || !geo_of(dims, &g) || batch < 0 || max_seqlen_k < 0 || num_splits < 0) return 0;
+  return resolve_splits(g, batch, batch, max_seqlen_k, num_splits, true);
+}
+
+mla_status_t mla_attn_decode(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
+                             const void* kv_cache, const void* pe_cache, const int32_t* cu_seqlens_k, int32_t batch,
+                             int64_t max_seqlen_k, void* o_lat, void* workspace, size_t workspace_bytes,
+                             int32_t num_splits, cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (batch < 0 || max_seqlen_k < 0 || num_splits < 0 || num_splits > 256 ||
+      q_row_stride < (int64_t)g.H * (g.Dn + g.R))
+    return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!q_abs || !q || !cu_seqlens_k || !o_lat || !aligned16(q_abs) || !aligned16(q) || !aligned16(o_lat))
+    return MLA_ERR_INVALID_ARG;
+  if (max_seqlen_k > 0 && (!kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
+    return MLA_ERR_INVALID_ARG;
+  const int splits = resolve_splits(g, batch, batch, max_seqlen_k, num_splits, true);
+  const size_t need = workspace_bytes_for(g, batch, batch, max_seqlen_k, splits, true);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return MLA_ERR_WORKSPACE;
+  if (g.family == 1) {
+    if ((q_row_stride * 2) % 16 != 0) return MLA_ERR_INVALID_ARG;
+    return mla::sm100::attention(q_abs, q, q_row_stride, kv_cache, pe_cache, nullptr, cu_seqlens_k, batch, batch,
+                                 1, max_seqlen_k, splits, g.scale, o_lat, workspace, stream);
+  }
+  if (g.bf16)
+    return simt_attention<mla_bf16>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, nullptr, cu_seqlens_k, batch,
+                                    batch, splits, o_lat, workspace, stream);
+  return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, nullptr, cu_seqlens_k, batch, batch,
+                               splits, o_lat, workspace, stream);
+}
+
+mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
+                                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch,
+                                    int64_t n_q_rows, int64_t max_seqlen_q, int64_t max_seqlen_k,
+                                    const void* kv_cache, const void* pe_cache, void* o_lat, void* workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (batch < 0 || n_q_rows < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 ||
+      q_row_stride < (int64_t)g.H * (g.Dn + g.R))
+    return MLA_ERR_INVALID_ARG;
+  if (batch == 0 || n_q_rows == 0) return MLA_OK;
+  if (!q_abs || !q || !cu_seqlens_q || !cu_seqlens_k || !o_lat || !aligned16(q_abs) || !aligned16(q) ||
+      !aligned16(o_lat))
+    return MLA_ERR_INVALID_ARG;
+  if (max_seqlen_k > 0 && (!kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
+    return MLA_ERR_INVALID_ARG;
+  const int splits = resolve_splits(g, batch, n_q_rows, max_seqlen_k, 0, false);
+  const size_t need = workspace_bytes_for(g, batch, n_q_rows, max_seqlen_k, splits, false);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return MLA_ERR_WORKSPACE;
+  if (g.family == 1) {
+    if ((q_row_stride * 2) % 16 != 0) return MLA_ERR_INVALID_ARG;
+    return mla::sm100::attention(q_abs, q, q_row_stride, kv_cache, pe_cache, cu_seqlens_q, cu_seqlens_k, batch,
+                                 n_q_rows, max_seqlen_q, max_seqlen_k, splits, g.scale, o_lat, workspace, stream);
+  }
+  if (g.bf16)
+    return simt_attention<mla_bf16>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, cu_seqlens_q, cu_seqlens_k,
+                                    batch, n_q_rows, splits, o_lat, workspace, stream);
+  return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, cu_seqlens_q, cu_seqlens_k, batch,
+                               n_q_rows, splits, o_lat, workspace, stream);
+}
+
+mla_status_t mla_device_status(cudaStream_t stream, uint32_t* code_out) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MLA_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpyFromSymbol(&word, mla::g_mla_error_word, sizeof(word)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (code_out) *code_out = word;
+  if (word != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(mla::g_mla_error_word, &zero, sizeof(zero)) != cudaSuccess) return MLA_ERR_CUDA;
+    return MLA_ERR_DEVICE_TIMEOUT;
+  }
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,214 @@
+// simt.cuh -- CUDA-core kernels for any head geometry, fp32 or bf16 storage,
+// fp32 arithmetic.  They serve the fp32 dtype (whose 1e-5 relative bound no
+// bf16/TF32 tensor-core product meets) and bf16 shapes the tensor-core kernels
+// are not built for.
+//
+// Operation: "Naive vs Absorb Attention Implementations in DeepSeek-V3",
+// section "Absorb Path Execution" (absorbed query, two-term scores, latent
+// value sum, output up-projection), with a softmax over the visible keys.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+namespace simt {
+
+constexpr int kThreads = 128;
+constexpr int kRowsPerBlock = 8;   // query rows sharing one weight read in the projections
+constexpr int kMaxC = 1024, kMaxR = 128, kMaxD = 256;
+
+// q_abs[n,h,c] = sum_{d<Dn} q[n,h,d] * W[h,d,c].  grid (ceil(n/8), H), 128 threads.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) absorb_q_kernel(
+    const T* __restrict__ q, int64_t q_row_stride, const T* __restrict__ wkv_b, T* __restrict__ q_abs,
+    int64_t n_rows, int H, int C, int Dn, int R, int Dv) {
+  __shared__ float qn[kRowsPerBlock][kMaxD];
+  const int h = blockIdx.y;
+  const int64_t n0 = (int64_t)blockIdx.x * kRowsPerBlock;
+  const int rows = (int)min64(kRowsPerBlock, n_rows - n0);
+  for (int i = threadIdx.x; i < kRowsPerBlock * Dn; i += kThreads) {
+    int r = i / Dn, d = i % Dn;
+    qn[r][d] = r < rows ? Elem<T>::load(q + (n0 + r) * q_row_stride + (int64_t)h * (Dn + R) + d) : 0.f;
+  }
+  __syncthreads();
+  const T* w = wkv_b + (int64_t)h * (Dn + Dv) * C;
+  for (int c = threadIdx.x; c < C; c += kThreads) {
+    float acc[kRowsPerBlock];
+#pragma unroll
+    for (int r = 0; r < kRowsPerBlock; ++r) acc[r] = 0.f;
+    for (int d = 0; d < Dn; ++d) {
+      float wv = Elem<T>::load(w + (int64_t)d * C + c);
+#pragma unroll
+      for (int r = 0; r < kRowsPerBlock; ++r) acc[r] = fmaf(qn[r][d], wv, acc[r]);
+    }
+    for (int r = 0; r < rows; ++r) Elem<T>::store(q_abs + ((n0 + r) * H + h) * (int64_t)C + c, acc[r]);
+  }
+}
+
+// out[n,h,d] = sum_c o_lat[n,h,c] * W[h,Dn+d,c].  grid (ceil(n/8), H), 128 threads.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) out_proj_kernel(
+    const T* __restrict__ o_lat, const T* __restrict__ wkv_b, T* __restrict__ out, int64_t n_rows, int H,
+    int C, int Dn, int Dv) {
+  extern __shared__ float o_s[];   // [kRowsPerBlock][C]
+  const int h = blockIdx.y;
+  const int64_t n0 = (int64_t)blockIdx.x * kRowsPerBlock;
+  const int rows = (int)min64(kRowsPerBlock, n_rows - n0);
+  for (int i = threadIdx.x; i < kRowsPerBlock * C; i += kThreads) {
+    int r = i / C, c = i % C;
+    o_s[i] = r < rows ? Elem<T>::load(o_lat + ((n0 + r) * H + h) * (int64_t)C + c) : 0.f;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const T* w = wkv_b + ((int64_t)h * (Dn + Dv) + Dn) * C;
+  for (int d = warp; d < Dv; d += kThreads / 32) {
+    float acc[kRowsPerBlock];
+#pragma unroll
+    for (int r = 0; r < kRowsPerBlock; ++r) acc[r] = 0.f;
+    for (int c = lane; c < C; c += 32) {
+      float wv = Elem<T>::load(w + (int64_t)d * C + c);
+#pragma unroll
+      for (int r = 0; r < kRowsPerBlock; ++r) acc[r] = fmaf(o_s[r * C + c], wv, acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < kRowsPerBlock; ++r) acc[r] = warp_sum(acc[r]);
+    if (lane == 0)
+      for (int r = 0; r < rows; ++r) Elem<T>::store(out + ((n0 + r) * H + h) * (int64_t)Dv + d, acc[r]);
+  }
+}
+
+__device__ __forceinline__ float block_reduce_max(float v, float* red) {
+  v = warp_max(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int i = 1; i < kThreads / 32; ++i) r = fmaxf(r, red[i]);
+  return r;
+}
+__device__ __forceinline__ float block_reduce_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = 0.f;
+  for (int i = 0; i < kThreads / 32; ++i) r += red[i];
+  return r;
+}
+
+// Attention for one (query row, head, split) per block, online softmax over
+// 128-key chunks.  With num_splits == 1 the normalised result goes straight to
+// o_lat; otherwise the unnormalised partial (o, running max m, running sum l)
+// goes to the workspace for attn_combine_kernel.  Keys visible to query i of
+// a chunk of s over a cache of t: j < t - s + i + 1.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) attn_kernel(
+    const T* __restrict__ q_abs, const T* __restrict__ q, int64_t q_row_stride, const T* __restrict__ kv,
+    const T* __restrict__ pe, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int batch,
+    int64_t n_rows, int H, int C, int R, int Dn, float scale, int num_splits, T* __restrict__ o_lat,
+    float* __restrict__ part_o, float* __restrict__ part_ml) {
+  extern __shared__ float sm[];
+  float* qa = sm;            // [C]
+  float* qp = qa + C;        // [R]
+  float* o = qp + R;         // [C]
+  float* p = o + C;          // [kThreads]
+  float* red = p + kThreads; // [32]
+  const int64_t n = blockIdx.x;
+  const int h = blockIdx.y, split = blockIdx.z;
+  const int b = cu_q ? find_sequence(cu_q, batch, n) : (int)n;
+  const int64_t k0 = __ldg(cu_k + b);
+  const int64_t t = max64(0, (int64_t)__ldg(cu_k + b + 1) - k0);
+  int64_t s = 1, i = 0;
+  if (cu_q) {
+    const int64_t q0 = __ldg(cu_q + b);
+    s = max64(0, (int64_t)__ldg(cu_q + b + 1) - q0);
+    i = n - q0;
+  }
+  const int64_t visible = min64(t, max64(0, t - s + i + 1));
+  const int64_t per = (visible + num_splits - 1) / num_splits;
+  const int64_t j_begin = min64(visible, (int64_t)split * per);
+  const int64_t j_end = min64(visible, j_begin + per);
+
+  for (int c = threadIdx.x; c < C; c += kThreads) {
+    qa[c] = Elem<T>::load(q_abs + (n * H + h) * (int64_t)C + c);
+    o[c] = 0.f;
+  }
+  for (int r = threadIdx.x; r < R; r += kThreads)
+    qp[r] = Elem<T>::load(q + n * q_row_stride + (int64_t)h * (Dn + R) + Dn + r);
+  __syncthreads();
+
+  float m = -INFINITY, l = 0.f;
+  for (int64_t j0 = j_begin; j0 < j_end; j0 += kThreads) {
+    const int64_t j = j0 + threadIdx.x;
+    float sc = -INFINITY;
+    if (j < j_end) {
+      const T* kr = kv + (k0 + j) * (int64_t)C;
+      const T* pr = pe + (k0 + j) * (int64_t)R;
+      float acc = 0.f;
+      for (int c = 0; c < C; ++c) acc = fmaf(qa[c], Elem<T>::load(kr + c), acc);
+      for (int r = 0; r < R; ++r) acc = fmaf(qp[r], Elem<T>::load(pr + r), acc);
+      sc = acc * scale;
+    }
+    const float cmax = block_reduce_max(sc, red);
+    const float m_new = fmaxf(m, cmax);
+    const float alpha = expf(m - m_new);   // m = -inf on the first chunk gives 0
+    const float pj = (j < j_end) ? expf(sc - m_new) : 0.f;
+    p[threadIdx.x] = pj;
+    const float psum = block_reduce_sum(pj, red);   // also orders the p[] writes
+    l = l * alpha + psum;
+    m = m_new;
+    const int cnt = (int)min64(kThreads, j_end - j0);
+    for (int c = threadIdx.x; c < C; c += kThreads) {
+      float acc = o[c] * alpha;
+      const T* kc = kv + (k0 + j0) * (int64_t)C + c;
+      for (int jj = 0; jj < cnt; ++jj) acc = fmaf(p[jj], Elem<T>::load(kc + (int64_t)jj * C), acc);
+      o[c] = acc;
+    }
+    __syncthreads();
+  }
+
+  if (num_splits == 1) {
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    for (int c = threadIdx.x; c < C; c += kThreads) Elem<T>::store(o_lat + (n * H + h) * (int64_t)C + c, o[c] * inv);
+  } else {
+    const int64_t slot = ((int64_t)split * n_rows + n) * H + h;
+    for (int c = threadIdx.x; c < C; c += kThreads) part_o[slot * C + c] = o[c];
+    if (threadIdx.x == 0) {
+      part_ml[slot * 2 + 0] = m;
+      part_ml[slot * 2 + 1] = l;
+    }
+  }
+}
+
+// Merge split partials: o = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s, M = max_s m_s.
+// grid (n_rows, H), 128 threads.  A row with no key anywhere gets zeros.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) combine_kernel(
+    const float* __restrict__ part_o, const float* __restrict__ part_ml, int num_splits, int64_t n_rows,
+    int H, int C, T* __restrict__ o_lat) {
+  const int64_t n = blockIdx.x;
+  const int h = blockIdx.y;
+  float mx = -INFINITY;
+  for (int s = 0; s < num_splits; ++s) mx = fmaxf(mx, part_ml[(((int64_t)s * n_rows + n) * H + h) * 2]);
+  float L = 0.f;
+  for (int s = 0; s < num_splits; ++s) {
+    const int64_t slot = ((int64_t)s * n_rows + n) * H + h;
+    const float ms = part_ml[slot * 2];
+    if (ms != -INFINITY) L += expf(ms - mx) * part_ml[slot * 2 + 1];
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  for (int c = threadIdx.x; c < C; c += kThreads) {
+    float acc = 0.f;
+    for (int s = 0; s < num_splits; ++s) {
+      const int64_t slot = ((int64_t)s * n_rows + n) * H + h;
+      const float ms = part_ml[slot * 2];
+      if (ms != -INFINITY) acc = fmaf(expf(ms - mx), part_o[slot * C + c], acc);
+    }
+    Elem<T>::store(o_lat + (n * H + h) * (int64_t)C + c, acc * inv);
+  }
+}
+
+}  // namespace simt
+}  // namespace mla

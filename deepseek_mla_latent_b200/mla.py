@@ -1,0 +1,184 @@
+"""Torch-facing wrappers of the C ABI (same names as include/mla.h, without the prefix).
+
+PyTorch only supplies device memory and the current stream; each wrapper checks
+shapes and dtypes, allocates outputs when the caller gives none, and calls the
+library.  Layouts are those of include/mla.h:
+
+  q      [N_q, H, Dn+R] (rows may be strided), q_abs / o_lat [N_q, H, C],
+  kv     [sum_t, C], pe [sum_t, R], wkv_b [H*(Dn+Dv), C], out [N_q, H, Dv],
+  cu_seqlens_* int32 [batch+1] on the device.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from ._lib import LIB, MLA_DTYPE_BF16, MlaDims, MlaError, _check, dims_from, make_dims  # noqa: F401
+
+
+def _dtype(d: MlaDims) -> torch.dtype:
+    return torch.bfloat16 if d.dtype == MLA_DTYPE_BF16 else torch.float32
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, contiguous=True) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _q_row_stride(q: torch.Tensor, d: MlaDims) -> int:
+    H, W = d.num_heads, d.qk_nope_head_dim + d.qk_rope_head_dim
+    if q.dim() != 3 or q.shape[1] != H or q.shape[2] != W or q.stride(2) != 1 or q.stride(1) != W:
+        raise ValueError(f"q must be [N, {H}, {W}] with contiguous heads (row stride free)")
+    return q.stride(0) if q.shape[0] > 1 else H * W
+
+
+def kernel_family(d: MlaDims) -> int:
+    return LIB.mla_kernel_family(ctypes.byref(d))
+
+
+def decode_num_splits(d: MlaDims, batch: int, max_seqlen_k: int, num_splits: int = 0) -> int:
+    return int(LIB.mla_decode_num_splits(ctypes.byref(d), batch, max_seqlen_k, num_splits))
+
+
+def absorb_q(d: MlaDims, q: torch.Tensor, wkv_b: torch.Tensor, q_abs: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    dt = _dtype(d)
+    n = q.shape[0]
+    rs = _q_row_stride(q, d)
+    _need(q, "q", dt, contiguous=False)
+    _need(wkv_b, "wkv_b", dt, (d.num_heads * (d.qk_nope_head_dim + d.v_head_dim), d.kv_lora_rank))
+    if q_abs is None:
+        q_abs = torch.empty((n, d.num_heads, d.kv_lora_rank), dtype=dt, device=q.device)
+    _need(q_abs, "q_abs", dt, (n, d.num_heads, d.kv_lora_rank))
+    _check(LIB.mla_absorb_q(ctypes.byref(d), _ptr(q), rs, _ptr(wkv_b), _ptr(q_abs), n, _stream(stream)),
+           "mla_absorb_q")
+    return q_abs
+
+
+def workspace_size(d: MlaDims, batch: int, n_q_rows: int, max_seqlen_k: int, num_splits: int = 0) -> int:
+    return int(LIB.mla_workspace_size(ctypes.byref(d), batch, n_q_rows, max_seqlen_k, num_splits))
+
+
+def workspace(d: MlaDims, batch: int, n_q_rows: int, max_seqlen_k: int, num_splits: int = 0,
+              device="cuda") -> Optional[torch.Tensor]:
+    nbytes = workspace_size(d, batch, n_q_rows, max_seqlen_k, num_splits)
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device) if nbytes else None
+
+
+def attn_decode(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, kv: torch.Tensor, pe: torch.Tensor,
+                cu_seqlens_k: torch.Tensor, max_seqlen_k: int, o_lat: Optional[torch.Tensor] = None,
+                ws: Optional[torch.Tensor] = None, num_splits: int = 0, stream=None) -> torch.Tensor:
+    dt = _dtype(d)
+    batch = cu_seqlens_k.numel() - 1
+    H, C, R = d.num_heads, d.kv_lora_rank, d.qk_rope_head_dim
+    rs = _q_row_stride(q, d)
+    _need(q_abs, "q_abs", dt, (batch, H, C))
+    _need(q, "q", dt, contiguous=False)
+    _need(kv, "kv", dt)
+    _need(pe, "pe", dt)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    if kv.dim() != 2 or kv.shape[1] != C or pe.dim() != 2 or pe.shape[1] != R or pe.shape[0] != kv.shape[0]:
+        raise ValueError("kv must be [T, C] and pe [T, R]")
+    if o_lat is None:
+        o_lat = torch.empty((batch, H, C), dtype=dt, device=q_abs.device)
+    _need(o_lat, "o_lat", dt, (batch, H, C))
+    if ws is None:
+        ws = workspace(d, batch, batch, max_seqlen_k, num_splits, device=q_abs.device)
+    wsb = ws.numel() if ws is not None else 0
+    _check(LIB.mla_attn_decode(ctypes.byref(d), _ptr(q_abs), _ptr(q), rs, _ptr(kv), _ptr(pe), _ptr(cu_seqlens_k),
+                               batch, int(max_seqlen_k), _ptr(o_lat), _ptr(ws), wsb, num_splits, _stream(stream)),
+           "mla_attn_decode")
+    return o_lat
+
+
+def attn_prefill_chunk(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                       cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int, kv: torch.Tensor,
+                       pe: torch.Tensor, o_lat: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    dt = _dtype(d)
+    batch = cu_seqlens_k.numel() - 1
+    n = q_abs.shape[0]
+    H, C, R = d.num_heads, d.kv_lora_rank, d.qk_rope_head_dim
+    rs = _q_row_stride(q, d)
+    _need(q_abs, "q_abs", dt, (n, H, C))
+    _need(q, "q", dt, contiguous=False)
+    _need(kv, "kv", dt)
+    _need(pe, "pe", dt)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, (batch + 1,))
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    if kv.dim() != 2 or kv.shape[1] != C or pe.dim() != 2 or pe.shape[1] != R or pe.shape[0] != kv.shape[0]:
+        raise ValueError("kv must be [T, C] and pe [T, R]")
+    if o_lat is None:
+        o_lat = torch.empty((n, H, C), dtype=dt, device=q_abs.device)
+    _need(o_lat, "o_lat", dt, (n, H, C))
+    if ws is None:
+        ws = workspace(d, batch, n, max_seqlen_k, 0, device=q_abs.device)
+    wsb = ws.numel() if ws is not None else 0
+    _check(LIB.mla_attn_prefill_chunk(ctypes.byref(d), _ptr(q_abs), _ptr(q), rs, _ptr(cu_seqlens_q),
+                                      _ptr(cu_seqlens_k), batch, n, int(max_seqlen_q), int(max_seqlen_k), _ptr(kv),
+                                      _ptr(pe), _ptr(o_lat), _ptr(ws), wsb, _stream(stream)),
+           "mla_attn_prefill_chunk")
+    return o_lat
+
+
+def out_proj(d: MlaDims, o_lat: torch.Tensor, wkv_b: torch.Tensor, out: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    dt = _dtype(d)
+    n = o_lat.shape[0]
+    _need(o_lat, "o_lat", dt, (n, d.num_heads, d.kv_lora_rank))
+    _need(wkv_b, "wkv_b", dt, (d.num_heads * (d.qk_nope_head_dim + d.v_head_dim), d.kv_lora_rank))
+    if out is None:
+        out = torch.empty((n, d.num_heads, d.v_head_dim), dtype=dt, device=o_lat.device)
+    _need(out, "out", dt, (n, d.num_heads, d.v_head_dim))
+    _check(LIB.mla_out_proj(ctypes.byref(d), _ptr(o_lat), _ptr(wkv_b), _ptr(out), n, _stream(stream)),
+           "mla_out_proj")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and raise MlaError if a device wait ran out; returns the error word."""
+    word = ctypes.c_uint32(0)
+    st = LIB.mla_device_status(_stream(stream), ctypes.byref(word))
+    _check(st, f"mla_device_status (device word {word.value:#x})")
+    return word.value
+
+
+def decode_step(d: MlaDims, q: torch.Tensor, wkv_b: torch.Tensor, kv: torch.Tensor, pe: torch.Tensor,
+                cu_seqlens_k: torch.Tensor, max_seqlen_k: int, num_splits: int = 0, bufs: Optional[dict] = None,
+                stream=None) -> torch.Tensor:
+    """The whole absorb decode path: mla_absorb_q -> mla_attn_decode -> mla_out_proj.
+
+    ``bufs`` may hold preallocated "q_abs", "o_lat", "out", "ws" tensors."""
+    bufs = bufs or {}
+    q_abs = absorb_q(d, q, wkv_b, bufs.get("q_abs"), stream)
+    o_lat = attn_decode(d, q_abs, q, kv, pe, cu_seqlens_k, max_seqlen_k, bufs.get("o_lat"), bufs.get("ws"),
+                        num_splits, stream)
+    return out_proj(d, o_lat, wkv_b, bufs.get("out"), stream)
+
+
+def prefill_step(d: MlaDims, q: torch.Tensor, wkv_b: torch.Tensor, kv: torch.Tensor, pe: torch.Tensor,
+                 cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int,
+                 bufs: Optional[dict] = None, stream=None) -> torch.Tensor:
+    """The whole chunked-prefill path: mla_absorb_q -> mla_attn_prefill_chunk -> mla_out_proj."""
+    bufs = bufs or {}
+    q_abs = absorb_q(d, q, wkv_b, bufs.get("q_abs"), stream)
+    o_lat = attn_prefill_chunk(d, q_abs, q, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, kv, pe,
+                               bufs.get("o_lat"), bufs.get("ws"), stream)
+    return out_proj(d, o_lat, wkv_b, bufs.get("out"), stream)

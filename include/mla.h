@@ -1,0 +1,183 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) multi-head latent attention library.
+ *
+ * The operation is DeepSeek-V3 multi-head latent attention in its "absorb"
+ * form, as set out in "Naive vs Absorb Attention Implementations in
+ * DeepSeek-V3", section "Absorb Path Execution":
+ *
+ *   W       = wkv_b viewed as [H, Dn + Dv, C]      (rows 0..Dn-1: key part,
+ *                                                   rows Dn..Dn+Dv-1: value part)
+ *   q_abs   = q_nope . W[:, :Dn]                    mla_absorb_q
+ *   scores  = (q_abs . kv^T + q_pe . pe^T) * scale  mla_attn_decode /
+ *   P       = softmax over keys (causal, aligned    mla_attn_prefill_chunk
+ *             to the end of the cache)
+ *   o_lat   = P . kv
+ *   out     = o_lat . W[:, Dn:]^T                   mla_out_proj
+ *
+ * The cache layout is the page's absorb cache design ("Absorb Implementation
+ * Cache Design"): kv_cache holds the compressed latent (C = kv_lora_rank
+ * values per token) and pe_cache the rotary key (R = qk_rope_head_dim values
+ * per token); neither has a head axis.  Here sequences are packed one after
+ * another along the token axis and located by cu_seqlens (an exclusive
+ * prefix sum of per-sequence lengths, batch + 1 entries, device memory).
+ *
+ * Conventions common to every call:
+ *  - Every pointer argument except `dims` and the `*_out` results is a
+ *    DEVICE pointer owned by the caller; the library never allocates, frees
+ *    or synchronises on these calls.  All calls are asynchronous on `stream`
+ *    and keep no state between calls, so they may be issued from several
+ *    host threads on different streams.
+ *  - Element types follow dims->dtype: MLA_DTYPE_BF16 (bfloat16 storage,
+ *    fp32 accumulation) or MLA_DTYPE_F32 (fp32 throughout).  cu_seqlens are
+ *    int32.
+ *  - Device buffers must be 16-byte aligned.
+ *  - The host checks sizes, alignment and the workspace before launching and
+ *    returns a status without launching on failure.  Sequence lengths live on
+ *    the device and are not read by the host: a negative length is treated
+ *    as 0, and a query row that sees no key gets zeros.
+ *  - Device-side waits are bounded.  A wait that runs out sets a device
+ *    error word instead of trapping; mla_device_status reports it.
+ */
+#ifndef MLA_B200_H_
+#define MLA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t; 0 is the legacy default stream. */
+#ifndef __DRIVER_TYPES_H__
+typedef struct CUstream_st* cudaStream_t;
+#endif
+
+#define MLA_API_VERSION 1
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+typedef enum mla_status {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,     /* null pointer, bad size, misaligned pointer, bad stride */
+  MLA_ERR_UNSUPPORTED = 2,     /* dims not compiled in (see each call) */
+  MLA_ERR_WORKSPACE = 3,       /* workspace missing or smaller than mla_workspace_size */
+  MLA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
+  MLA_ERR_DEVICE_TIMEOUT = 5   /* a bounded device wait ran out (see mla_device_status) */
+} mla_status_t;
+
+typedef enum mla_dtype { MLA_DTYPE_BF16 = 0, MLA_DTYPE_F32 = 1 } mla_dtype_t;
+
+/* Head geometry.  H = num_heads, C = kv_lora_rank, Dn = qk_nope_head_dim,
+ * R = qk_rope_head_dim, Dv = v_head_dim.  softmax_scale multiplies the scores
+ * (DeepSeek-V3 without YaRN: 1/sqrt(Dn + R)).
+ *
+ * bf16 runs on the tcgen05 tensor-core kernels when C = 512, R = 64,
+ * Dn = Dv = 128 and H is a multiple of 128 (the DeepSeek-V3 shapes); other
+ * bf16 shapes and every fp32 shape run on CUDA-core kernels, which need
+ * C <= 1024, R <= 128, Dn <= 256, Dv <= 256 and H <= 1024. */
+typedef struct mla_dims {
+  int32_t num_heads;
+  int32_t kv_lora_rank;
+  int32_t qk_nope_head_dim;
+  int32_t qk_rope_head_dim;
+  int32_t v_head_dim;
+  int32_t dtype;        /* mla_dtype_t */
+  float softmax_scale;
+} mla_dims_t;
+
+/* Absorbed query: q_abs[n,h,c] = sum_{d<Dn} q[n,h,d] * wkv_b[h*(Dn+Dv)+d, c].
+ * ("Absorb Path Execution", the einsum that folds q_nope through the key
+ * rows of wkv_b.)
+ *   q        [n_rows, H, Dn+R], row n starts at q + n*q_row_stride elements,
+ *            head h of a row at + h*(Dn+R); only dims 0..Dn-1 are read.
+ *   wkv_b    [H*(Dn+Dv), C] row-major.
+ *   q_abs    [n_rows, H, C] contiguous, written.
+ *   n_rows   >= 0 (0 is a no-op).  q_row_stride >= H*(Dn+R).  */
+MLA_API mla_status_t mla_absorb_q(const mla_dims_t* dims, const void* q, int64_t q_row_stride,
+                          const void* wkv_b, void* q_abs, int64_t n_rows, cudaStream_t stream);
+
+/* Bytes of workspace mla_attn_decode / mla_attn_prefill_chunk need for these
+ * sizes.  num_splits = 0 means the automatic choice the attention call makes
+ * for the same arguments.  n_q_rows = total query rows (batch for decode). */
+MLA_API size_t mla_workspace_size(const mla_dims_t* dims, int32_t batch, int64_t n_q_rows,
+                          int64_t max_seqlen_k, int32_t num_splits);
+
+/* Number of key-range splits mla_attn_decode uses for these arguments
+ * (num_splits = 0: the automatic choice).  With more than one split the
+ * call launches a merge kernel after the attention kernel. */
+MLA_API int32_t mla_decode_num_splits(const mla_dims_t* dims, int32_t batch, int64_t max_seqlen_k,
+                                      int32_t num_splits);
+
+/* Decode attention: one query per sequence over its whole cache (no mask).
+ * ("Absorb Path Execution", the score einsums and the latent value einsum;
+ * the softmax between them is the reading documented with the oracle.)
+ *   q_abs        [batch, H, C] (from mla_absorb_q).
+ *   q            [batch, H, Dn+R] with row stride q_row_stride; the rotary
+ *                part q_pe is read from dims Dn..Dn+R-1.
+ *   kv_cache     [total_k, C], pe_cache [total_k, R]; sequence b owns rows
+ *                cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1.
+ *   cu_seqlens_k device int32 [batch+1], non-decreasing.
+ *   max_seqlen_k host upper bound of every sequence length (keys past it
+ *                are not read); it sizes the split-t partition.
+ *   o_lat        [batch, H, C] written: softmax-weighted sum of latent rows.
+ *   workspace    device scratch of at least mla_workspace_size(dims, batch,
+ *                batch, max_seqlen_k, num_splits) bytes (may be NULL when
+ *                that is 0).  Contents on entry are ignored.
+ *   num_splits   0 = automatic; otherwise the key range of each sequence is
+ *                cut into that many parts that are merged afterwards (1..256).
+ */
+MLA_API mla_status_t mla_attn_decode(const mla_dims_t* dims, const void* q_abs, const void* q,
+                             int64_t q_row_stride, const void* kv_cache, const void* pe_cache,
+                             const int32_t* cu_seqlens_k, int32_t batch, int64_t max_seqlen_k,
+                             void* o_lat, void* workspace, size_t workspace_bytes,
+                             int32_t num_splits, cudaStream_t stream);
+
+/* Chunked-prefill attention: sequence b has s_b = cu_seqlens_q[b+1]-cu_seqlens_q[b]
+ * new queries whose keys are already the last s_b rows of its cache of
+ * t_b rows; query i (0-based) sees keys j <= t_b - s_b + i.
+ *   q_abs, q     [total_q, H, C] and [total_q, H, Dn+R] (row stride q_row_stride).
+ *   cu_seqlens_q device int32 [batch+1]; cu_seqlens_k as for decode.
+ *   max_seqlen_q, max_seqlen_k  host upper bounds of s_b and t_b.
+ *   o_lat        [total_q, H, C] written.
+ *   workspace    at least mla_workspace_size(dims, batch, total_q, max_seqlen_k, 0)
+ *                bytes, where total_q = cu_seqlens_q[batch] <= n_q_rows given there.
+ *   n_q_rows     host value of cu_seqlens_q[batch] (rows of q_abs / o_lat). */
+MLA_API mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* q_abs, const void* q,
+                                    int64_t q_row_stride, const int32_t* cu_seqlens_q,
+                                    const int32_t* cu_seqlens_k, int32_t batch, int64_t n_q_rows,
+                                    int64_t max_seqlen_q, int64_t max_seqlen_k,
+                                    const void* kv_cache, const void* pe_cache, void* o_lat,
+                                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Output projection: out[n,h,d] = sum_c o_lat[n,h,c] * wkv_b[h*(Dn+Dv)+Dn+d, c].
+ * ("Absorb Path Execution", the last einsum, with the tail rows of wkv_b.)
+ *   o_lat [n_rows, H, C] contiguous; out [n_rows, H, Dv] contiguous, written. */
+MLA_API mla_status_t mla_out_proj(const mla_dims_t* dims, const void* o_lat, const void* wkv_b, void* out,
+                          int64_t n_rows, cudaStream_t stream);
+
+/* Static text for a status code. */
+MLA_API const char* mla_status_string(mla_status_t status);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns MLA_ERR_DEVICE_TIMEOUT if a bounded wait in an
+ * earlier kernel ran out (its code is stored in *code_out when non-NULL),
+ * MLA_ERR_CUDA if the stream reports an error, MLA_OK otherwise. */
+MLA_API mla_status_t mla_device_status(cudaStream_t stream, uint32_t* code_out);
+
+/* Which kernel family a call with these dims runs: 1 = tcgen05 tensor-core
+ * kernels, 0 = CUDA-core kernels, -1 = unsupported dims. */
+MLA_API int32_t mla_kernel_family(const mla_dims_t* dims);
+
+/* MLA_API_VERSION of the built library. */
+MLA_API int32_t mla_api_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H_ */

@@ -1,0 +1,104 @@
+"""The C ABI without a GPU: the library loads, exports what include/mla.h declares,
+and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MLA_API\s+[\w\s\*]*?\b(mla_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from deepseek_mla_latent_b200 import build
+    build.build()
+    from deepseek_mla_latent_b200 import _lib
+    return _lib
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("mla_absorb_q", "mla_attn_decode", "mla_attn_prefill_chunk", "mla_out_proj",
+                     "mla_workspace_size", "mla_status_string", "mla_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib.LIB, n), n
+        assert n in lib.SIGNATURES, f"binding lacks {n}"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.LIB.mla_api_version() == 1
+    for s in range(6):
+        assert lib.LIB.mla_status_string(s)
+
+
+V3 = dict(heads=128, kv_lora_rank=512, qk_nope=128, qk_rope=64, v_head=128)
+
+
+def test_kernel_family_selection(lib):
+    d = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
+    assert lib.LIB.mla_kernel_family(ctypes.byref(d)) in (0, 1)
+    d = lib.make_dims(8, 64, 32, 16, 32, "f32", 0.1)
+    assert lib.LIB.mla_kernel_family(ctypes.byref(d)) == 0
+    d = lib.make_dims(8, 4096, 32, 16, 32, "f32", 0.1)
+    assert lib.LIB.mla_kernel_family(ctypes.byref(d)) == -1
+    d = lib.make_dims(8, 64, 32, 16, 32, "f32", 0.1)
+    d.dtype = 7
+    assert lib.LIB.mla_kernel_family(ctypes.byref(d)) == -1
+
+
+# Fake but aligned device addresses: every call below must return before touching them.
+A = 0x10000
+
+
+def test_host_validation_rejects_before_launch(lib):
+    L = lib.LIB
+    d = lib.make_dims(8, 64, 32, 16, 32, "f32", 0.1)
+    bad = lib.make_dims(8, 4096, 32, 16, 32, "f32", 0.1)
+    assert L.mla_absorb_q(None, A, 384, A, A, 4, None) == lib.MLA_ERR_INVALID_ARG
+    assert L.mla_absorb_q(ctypes.byref(bad), A, 384, A, A, 4, None) == lib.MLA_ERR_UNSUPPORTED
+    assert L.mla_absorb_q(ctypes.byref(d), A, 100, A, A, 4, None) == lib.MLA_ERR_INVALID_ARG   # stride < H*(Dn+R)
+    assert L.mla_absorb_q(ctypes.byref(d), None, 384, A, A, 4, None) == lib.MLA_ERR_INVALID_ARG
+    assert L.mla_absorb_q(ctypes.byref(d), A + 4, 384, A, A, 4, None) == lib.MLA_ERR_INVALID_ARG  # misaligned
+    assert L.mla_absorb_q(ctypes.byref(d), A, 384, A, A, -1, None) == lib.MLA_ERR_INVALID_ARG
+    assert L.mla_absorb_q(ctypes.byref(d), None, 384, None, None, 0, None) == lib.MLA_OK        # empty
+    assert L.mla_out_proj(ctypes.byref(d), A, None, A, 3, None) == lib.MLA_ERR_INVALID_ARG
+    assert L.mla_out_proj(ctypes.byref(d), None, None, None, 0, None) == lib.MLA_OK
+    # decode: too many splits, negative batch, missing cache
+    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, A, 2, 128, A, A, 1 << 20, 300, None) \
+        == lib.MLA_ERR_INVALID_ARG
+    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, A, -1, 128, A, A, 1 << 20, 0, None) \
+        == lib.MLA_ERR_INVALID_ARG
+    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, None, A, A, 2, 128, A, A, 1 << 20, 0, None) \
+        == lib.MLA_ERR_INVALID_ARG
+    assert L.mla_attn_decode(ctypes.byref(d), None, None, 384, None, None, None, 0, 0, None, None, 0, 0, None) \
+        == lib.MLA_OK
+    # prefill: missing cu_seqlens_q
+    assert L.mla_attn_prefill_chunk(ctypes.byref(d), A, A, 384, None, A, 2, 8, 4, 128, A, A, A, A, 1 << 20,
+                                    None) == lib.MLA_ERR_INVALID_ARG
+
+
+def test_workspace_is_checked(lib):
+    L = lib.LIB
+    d = lib.make_dims(8, 64, 32, 16, 32, "f32", 0.1)
+    need = L.mla_workspace_size(ctypes.byref(d), 2, 2, 1 << 16, 4)
+    assert need > 0
+    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, A, 2, 1 << 16, A, A, need - 16, 4, None) \
+        == lib.MLA_ERR_WORKSPACE
+    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, A, 2, 1 << 16, A, None, need, 4, None) \
+        == lib.MLA_ERR_WORKSPACE
+    assert L.mla_workspace_size(ctypes.byref(d), 2, 2, 1 << 16, 1) == 0
+    v3 = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
+    assert L.mla_workspace_size(ctypes.byref(v3), 8, 8, 4096, 0) >= 0

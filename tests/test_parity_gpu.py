@@ -1,0 +1,113 @@
+"""GPU parity: the library's CUDA path against the fp64 oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from deepseek_mla_latent_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from deepseek_mla_latent_b200 import mla
+    from gpu_util import TOL, assert_close, run_path, to_dev
+
+
+def _check_full(w, num_splits=0):
+    got = run_path(w, num_splits=num_splits)
+    q_abs, o_lat, _ = oracle.workload_absorb(w)
+    ref = oracle.workload_naive(w)
+    dt = w.dims.dtype
+    assert_close(got["q_abs"], q_abs, dt, "q_abs")
+    assert_close(got["o_lat"], o_lat, dt, "o_lat")
+    return assert_close(got["out"], ref, dt, "out")
+
+
+def test_tiny_fp32_workload():
+    """Workload 0 in full: fp32 path within 1e-5 relative of the fp64 oracle."""
+    _check_full(wl.workload(0))
+
+
+@pytest.mark.parametrize("splits", [0, 1, 3])
+def test_fp32_small_decode_and_splits(splits):
+    w = wl.make_workload("f32", wl.TINY, [1, 1, 1], [1, 300, 129], seed=1)
+    _check_full(w, splits)
+
+
+def test_fp32_prefill():
+    w = wl.make_workload("f32p", wl.TINY, [4, 9], [4, 200], seed=2)
+    _check_full(w)
+
+
+V3 = wl.V3
+
+
+@pytest.mark.parametrize("seqlens", [[1, 200, 777], [129], [4096, 33]])
+def test_v3_decode_ragged(seqlens):
+    """DeepSeek-V3 shapes, several 128-key tiles with ragged tails, whole output compared."""
+    w = wl.make_workload("v3d", V3, [1] * len(seqlens), seqlens, seed=3)
+    _check_full(w)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 7, 64])
+def test_v3_decode_split_invariance(splits):
+    w = wl.make_workload("v3s", V3, [1, 1], [1000, 260], seed=4)
+    _check_full(w, splits)
+
+
+def test_v3_decode_more_splits_than_keys():
+    w = wl.make_workload("v3k", V3, [1, 1, 1], [1, 2, 5], seed=5)
+    _check_full(w, 8)
+
+
+def test_v3_decode_empty_sequence_gives_zeros():
+    w = wl.make_workload("v3e", V3, [1, 1, 1], [0, 70, 0], seed=6)
+    got = run_path(w)
+    assert np.all(got["out"][0] == 0) and np.all(got["out"][2] == 0)
+    ref = oracle.workload_naive(w)
+    assert_close(got["out"], ref, "bf16", "out")
+
+
+@pytest.mark.parametrize("sq,sk", [([5, 130], [300, 700]), ([128], [128]), ([1, 257], [1, 1000]),
+                                   ([3, 0, 64], [64, 10, 200])])
+def test_v3_prefill_causal(sq, sk):
+    w = wl.make_workload("v3p", V3, sq, sk, seed=7)
+    _check_full(w)
+
+
+def test_v3_prefill_equals_decode_for_single_query():
+    w = wl.make_workload("v3pd", V3, [1, 1], [500, 77], seed=8)
+    a = run_path(w, decode=True)["out"]
+    b = run_path(w, decode=False)["out"]
+    ref = oracle.workload_naive(w)
+    assert_close(a, ref, "bf16", "decode")
+    assert_close(b, ref, "bf16", "prefill")
+
+
+def _sampled(index, pairs, num_splits=0):
+    """A full-size workload run in the benchmark's launch configuration, checked
+    on (sequence, head) pairs the oracle computes one by one."""
+    w = wl.workload(index)
+    got = run_path(w, num_splits=num_splits)["out"]
+    ref = oracle.workload_naive(w, pairs=pairs)
+    cq = w.cu_seqlens_q
+    for (b, h), r in ref.items():
+        assert_close(got[cq[b]:cq[b + 1], h, :], r, w.dims.dtype, f"workload {index} seq {b} head {h}")
+
+
+def test_full_v3_decode_sampled():
+    _sampled(1, [(0, 0), (3, 77), (7, 127)])
+
+
+def test_full_ragged_sampled():
+    _, _, _, sk = wl.workload_shape(2)
+    longest, shortest = int(np.argmax(sk)), int(np.argmin(sk))
+    _sampled(2, [(longest, 5), (shortest, 100), (31, 64)])
+
+
+def test_full_long_context_sampled():
+    _sampled(3, [(0, 1), (1, 126)])
+
+
+def test_full_prefill_sampled():
+    _sampled(4, [(0, 3), (3, 120)])
