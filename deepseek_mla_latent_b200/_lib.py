@@ -31,8 +31,9 @@ _DP = ctypes.POINTER(MlaDims)
 SIGNATURES = {
     "mla_absorb_q": (_I32, [_DP, _P, _I64, _P, _P, _I64, _P]),
     "mla_workspace_size": (_SZ, [_DP, _I32, _I64, _I64, _I32]),
-    "mla_attn_decode": (_I32, [_DP, _P, _P, _I64, _P, _P, _P, _I32, _I64, _P, _P, _SZ, _I32, _P]),
-    "mla_attn_prefill_chunk": (_I32, [_DP, _P, _P, _I64, _P, _P, _I32, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
+    "mla_attn_decode": (_I32, [_DP, _P, _P, _I64, _P, _P, _I64, _P, _I32, _I64, _P, _P, _SZ, _I32, _P]),
+    "mla_attn_prefill_chunk": (_I32, [_DP, _P, _P, _I64, _P, _P, _I32, _I64, _I64, _I64, _P, _P, _I64, _P, _P, _SZ,
+                                      _P]),
     "mla_out_proj": (_I32, [_DP, _P, _P, _P, _I64, _P]),
     "mla_status_string": (ctypes.c_char_p, [_I32]),
     "mla_device_status": (_I32, [_P, ctypes.POINTER(ctypes.c_uint32)]),

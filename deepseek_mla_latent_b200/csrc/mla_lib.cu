@@ -81,7 +81,8 @@ size_t simt_workspace(const Geo& g, int64_t n_q_rows, int splits) {
 
 template <typename T>
 mla_status_t simt_attention(const Geo& g, const void* q_abs, const void* q, int64_t q_row_stride,
-                            const void* kv, const void* pe, const int32_t* cu_q, const int32_t* cu_k, int batch,
+                            const void* kv, const void* pe, int64_t kv_rows, const int32_t* cu_q, const int32_t* cu_k,
+                            int batch,
                             int64_t n_rows, int splits, void* o_lat, void* ws, cudaStream_t stream) {
   float* part_o = nullptr;
   float* part_ml = nullptr;
@@ -94,7 +95,7 @@ mla_status_t simt_attention(const Geo& g, const void* q_abs, const void* q, int6
   size_t smem = (size_t)(2 * g.C + g.R + mla::simt::kThreads + 32) * sizeof(float);
   mla::simt::attn_kernel<T><<<grid, mla::simt::kThreads, smem, stream>>>(
       static_cast<const T*>(q_abs), static_cast<const T*>(q), q_row_stride, static_cast<const T*>(kv),
-      static_cast<const T*>(pe), cu_q, cu_k, batch, n_rows, g.H, g.C, g.R, g.Dn, g.scale, splits,
+      static_cast<const T*>(pe), kv_rows, cu_q, cu_k, batch, n_rows, g.H, g.C, g.R, g.Dn, g.scale, splits,
       static_cast<T*>(o_lat), part_o, part_ml);
   if (splits > 1) {
     mla::simt::combine_kernel<T><<<dim3((unsigned)n_rows, g.H), mla::simt::kThreads, 0, stream>>>(
@@ -107,13 +108,13 @@ int resolve_splits(const Geo& g, int32_t batch, int64_t n_q_rows, int64_t max_se
                    bool decode) {
   if (!decode) return g.family == 1 ? mla::sm100::prefill_splits() : 1;
   if (num_splits > 0) return num_splits;
-  if (g.family == 1) return mla::sm100::auto_decode_splits(batch, max_seqlen_k, device_sm_count());
+  if (g.family == 1) return mla::sm100::auto_decode_splits(batch, g.H, max_seqlen_k, device_sm_count());
   return simt_auto_splits(n_q_rows, g.H, max_seqlen_k);
 }
 
 size_t workspace_bytes_for(const Geo& g, int32_t batch, int64_t n_q_rows, int64_t max_seqlen_k, int splits,
                            bool decode) {
-  if (g.family == 1) return mla::sm100::workspace_bytes(g.H, g.C, batch, n_q_rows, max_seqlen_k, splits, decode);
+  if (g.family == 1) return mla::sm100::workspace_bytes(g.H, n_q_rows, splits);
   return simt_workspace(g, n_q_rows, splits);
 }
 
@@ -208,65 +209,67 @@ int32_t mla_decode_num_splits(const mla_dims_t* dims, int32_t batch, int64_t max
 }
 
 mla_status_t mla_attn_decode(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
-                             const void* kv_cache, const void* pe_cache, const int32_t* cu_seqlens_k, int32_t batch,
+                             const void* kv_cache, const void* pe_cache, int64_t kv_rows,
+                             const int32_t* cu_seqlens_k, int32_t batch,
                              int64_t max_seqlen_k, void* o_lat, void* workspace, size_t workspace_bytes,
                              int32_t num_splits, cudaStream_t stream) {
   Geo g;
   if (!dims) return MLA_ERR_INVALID_ARG;
   if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
-  if (batch < 0 || max_seqlen_k < 0 || num_splits < 0 || num_splits > 256 ||
+  if (batch < 0 || max_seqlen_k < 0 || kv_rows < 0 || num_splits < 0 || num_splits > 256 ||
       q_row_stride < (int64_t)g.H * (g.Dn + g.R))
     return MLA_ERR_INVALID_ARG;
   if (batch == 0) return MLA_OK;
   if (!q_abs || !q || !cu_seqlens_k || !o_lat || !aligned16(q_abs) || !aligned16(q) || !aligned16(o_lat))
     return MLA_ERR_INVALID_ARG;
-  if (max_seqlen_k > 0 && (!kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
+  if (kv_rows > 0 && (!kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
     return MLA_ERR_INVALID_ARG;
   const int splits = resolve_splits(g, batch, batch, max_seqlen_k, num_splits, true);
   const size_t need = workspace_bytes_for(g, batch, batch, max_seqlen_k, splits, true);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return MLA_ERR_WORKSPACE;
   if (g.family == 1) {
     if ((q_row_stride * 2) % 16 != 0) return MLA_ERR_INVALID_ARG;
-    return mla::sm100::attention(q_abs, q, q_row_stride, kv_cache, pe_cache, nullptr, cu_seqlens_k, batch, batch,
-                                 1, max_seqlen_k, splits, g.scale, o_lat, workspace, stream);
+    return mla::sm100::attention(q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, nullptr, cu_seqlens_k, batch,
+                                 batch, g.H, splits, g.scale, o_lat, workspace, stream);
   }
   if (g.bf16)
-    return simt_attention<mla_bf16>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, nullptr, cu_seqlens_k, batch,
-                                    batch, splits, o_lat, workspace, stream);
-  return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, nullptr, cu_seqlens_k, batch, batch,
-                               splits, o_lat, workspace, stream);
+    return simt_attention<mla_bf16>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, nullptr, cu_seqlens_k,
+                                    batch, batch, splits, o_lat, workspace, stream);
+  return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, nullptr, cu_seqlens_k, batch,
+                               batch, splits, o_lat, workspace, stream);
 }
 
 mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
                                     const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch,
                                     int64_t n_q_rows, int64_t max_seqlen_q, int64_t max_seqlen_k,
-                                    const void* kv_cache, const void* pe_cache, void* o_lat, void* workspace,
+                                    const void* kv_cache, const void* pe_cache, int64_t kv_rows, void* o_lat,
+                                    void* workspace,
                                     size_t workspace_bytes, cudaStream_t stream) {
   Geo g;
   if (!dims) return MLA_ERR_INVALID_ARG;
   if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
-  if (batch < 0 || n_q_rows < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 ||
+  if (batch < 0 || n_q_rows < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || kv_rows < 0 ||
       q_row_stride < (int64_t)g.H * (g.Dn + g.R))
     return MLA_ERR_INVALID_ARG;
   if (batch == 0 || n_q_rows == 0) return MLA_OK;
   if (!q_abs || !q || !cu_seqlens_q || !cu_seqlens_k || !o_lat || !aligned16(q_abs) || !aligned16(q) ||
       !aligned16(o_lat))
     return MLA_ERR_INVALID_ARG;
-  if (max_seqlen_k > 0 && (!kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
+  if (kv_rows > 0 && (!kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
     return MLA_ERR_INVALID_ARG;
   const int splits = resolve_splits(g, batch, n_q_rows, max_seqlen_k, 0, false);
   const size_t need = workspace_bytes_for(g, batch, n_q_rows, max_seqlen_k, splits, false);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return MLA_ERR_WORKSPACE;
   if (g.family == 1) {
     if ((q_row_stride * 2) % 16 != 0) return MLA_ERR_INVALID_ARG;
-    return mla::sm100::attention(q_abs, q, q_row_stride, kv_cache, pe_cache, cu_seqlens_q, cu_seqlens_k, batch,
-                                 n_q_rows, max_seqlen_q, max_seqlen_k, splits, g.scale, o_lat, workspace, stream);
+    return mla::sm100::attention(q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, cu_seqlens_k,
+                                 batch, n_q_rows, g.H, splits, g.scale, o_lat, workspace, stream);
   }
   if (g.bf16)
-    return simt_attention<mla_bf16>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, cu_seqlens_q, cu_seqlens_k,
-                                    batch, n_q_rows, splits, o_lat, workspace, stream);
-  return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, cu_seqlens_q, cu_seqlens_k, batch,
-                               n_q_rows, splits, o_lat, workspace, stream);
+    return simt_attention<mla_bf16>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q,
+                                    cu_seqlens_k, batch, n_q_rows, splits, o_lat, workspace, stream);
+  return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, cu_seqlens_k,
+                               batch, n_q_rows, splits, o_lat, workspace, stream);
 }
 
 mla_status_t mla_device_status(cudaStream_t stream, uint32_t* code_out) {

@@ -106,7 +106,7 @@ __device__ __forceinline__ float block_reduce_sum(float v, float* red) {
 template <typename T>
 __global__ void __launch_bounds__(kThreads) attn_kernel(
     const T* __restrict__ q_abs, const T* __restrict__ q, int64_t q_row_stride, const T* __restrict__ kv,
-    const T* __restrict__ pe, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int batch,
+    const T* __restrict__ pe, int64_t kv_rows, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int batch,
     int64_t n_rows, int H, int C, int R, int Dn, float scale, int num_splits, T* __restrict__ o_lat,
     float* __restrict__ part_o, float* __restrict__ part_ml) {
   extern __shared__ float sm[];
@@ -118,8 +118,8 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(
   const int64_t n = blockIdx.x;
   const int h = blockIdx.y, split = blockIdx.z;
   const int b = cu_q ? find_sequence(cu_q, batch, n) : (int)n;
-  const int64_t k0 = __ldg(cu_k + b);
-  const int64_t t = max64(0, (int64_t)__ldg(cu_k + b + 1) - k0);
+  const int64_t k0 = min64(max64(0, __ldg(cu_k + b)), kv_rows);
+  const int64_t t = max64(0, min64((int64_t)__ldg(cu_k + b + 1), kv_rows) - k0);
   int64_t s = 1, i = 0;
   if (cu_q) {
     const int64_t q0 = __ldg(cu_q + b);

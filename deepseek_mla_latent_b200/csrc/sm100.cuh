@@ -1,24 +1,193 @@
-// sm100.cuh -- tensor-core (tcgen05) kernels for the DeepSeek-V3 head shapes.
+// sm100.cuh -- host side of the tensor-core (tcgen05) path for the
+// DeepSeek-V3 head shapes: TMA descriptor encoding, launch shapes, split-t
+// planning and the workspace layout.
 #pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "mla.h"
+#include "sm100_attn.cuh"
+#include "sm100_proj.cuh"
 
 namespace mla {
 namespace sm100 {
 
-inline bool supports(int H, int C, int Dn, int R, int Dv) { return false; }
-inline int prefill_splits() { return 1; }
-inline int auto_decode_splits(int batch, int64_t max_seqlen_k, int sms) { return 1; }
-inline size_t workspace_bytes(int H, int C, int batch, int64_t n_q_rows, int64_t max_seqlen_k, int splits,
-                              bool decode) { return 0; }
-inline mla_status_t absorb_q(const void*, int64_t, const void*, void*, int64_t, int, cudaStream_t) {
-  return MLA_ERR_UNSUPPORTED;
+inline bool supports(int H, int C, int Dn, int R, int Dv) {
+  return C == 512 && R == 64 && Dn == 128 && Dv == 128 && H > 0 && H % 128 == 0 && H <= 128 * 64;
 }
-inline mla_status_t out_proj(const void*, const void*, void*, int64_t, int, cudaStream_t) { return MLA_ERR_UNSUPPORTED; }
-inline mla_status_t attention(const void*, const void*, int64_t, const void*, const void*, const int32_t*,
-                              const int32_t*, int, int64_t, int64_t, int64_t, int, float, void*, void*, cudaStream_t) {
-  return MLA_ERR_UNSUPPORTED;
+
+// ---------------------------------------------------------------- TMA maps --
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map: dims/strides innermost first, strides in bytes (rank-1 of them).
+inline bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                     const uint32_t* box, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[3], s[2];
+  cuuint32_t b[3], e[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
+  for (int i = 0; i < rank - 1; ++i) s[i] = strides[i];
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, b, e,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline mla_status_t last_launch() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+template <typename K>
+inline bool set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+}
+
+// --------------------------------------------------------------- projections
+template <bool A_MN, int N_TILE, int STAGES>
+inline mla_status_t launch_proj(const CUtensorMap& tw, const CUtensorMap& tx, dim3 grid, int k_chunks, int w_row_base,
+                                int n_rows, void* out, int64_t out_row_stride, int out_head_stride,
+                                cudaStream_t stream) {
+  constexpr size_t smem = proj_smem_bytes<N_TILE, STAGES>();
+  auto kern = proj_kernel<A_MN, N_TILE, STAGES>;
+  if (!set_smem(kern, smem)) return MLA_ERR_CUDA;
+  kern<<<grid, kProjThreads, smem, stream>>>(tw, tx, k_chunks, w_row_base, 256, n_rows,
+                                             static_cast<__nv_bfloat16*>(out), out_row_stride, out_head_stride);
+  return last_launch();
+}
+
+template <bool A_MN, int STAGES>
+inline mla_status_t dispatch_proj(const CUtensorMap& tw, const CUtensorMap& tx, int m_tiles, int H, int64_t n_rows,
+                                  int k_chunks, int w_row_base, void* out, int64_t out_row_stride,
+                                  int out_head_stride, cudaStream_t stream) {
+  auto go = [&](auto tile) {
+    constexpr int NT = decltype(tile)::value;
+    dim3 grid(m_tiles, H, (unsigned)((n_rows + NT - 1) / NT));
+    return launch_proj<A_MN, NT, STAGES>(tw, tx, grid, k_chunks, w_row_base, (int)n_rows, out, out_row_stride,
+                                         out_head_stride, stream);
+  };
+  if (n_rows <= 16) return go(std::integral_constant<int, 16>{});
+  if (n_rows <= 32) return go(std::integral_constant<int, 32>{});
+  if (n_rows <= 64) return go(std::integral_constant<int, 64>{});
+  if (n_rows <= 128) return go(std::integral_constant<int, 128>{});
+  return go(std::integral_constant<int, 256>{});
+}
+
+inline mla_status_t absorb_q(const void* q, int64_t q_row_stride, const void* wkv_b, void* q_abs, int64_t n_rows,
+                             int H, cudaStream_t stream) {
+  if (n_rows >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  CUtensorMap tw, tx;
+  const uint64_t wd[2] = {512, (uint64_t)H * 256}, ws[1] = {1024};
+  const uint32_t wb[2] = {64, 64};   // 64 latent columns x 64 key rows (M-major A)
+  const uint64_t xd[3] = {192, (uint64_t)H, (uint64_t)n_rows}, xs[2] = {384, (uint64_t)q_row_stride * 2};
+  const uint32_t xb[3] = {64, 1, 0};
+  uint32_t box[3] = {xb[0], xb[1], (uint32_t)(n_rows <= 16 ? 16 : n_rows <= 32 ? 32 : n_rows <= 64 ? 64 : n_rows <= 128 ? 128 : 256)};
+  if (!make_map(&tw, wkv_b, 2, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  if (!make_map(&tx, q, 3, xd, xs, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  return dispatch_proj<true, 2>(tw, tx, 4, H, n_rows, 2, 0, q_abs, (int64_t)H * 512, 512, stream);
+}
+
+inline mla_status_t out_proj(const void* o_lat, const void* wkv_b, void* out, int64_t n_rows, int H,
+                             cudaStream_t stream) {
+  if (n_rows >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  CUtensorMap tw, tx;
+  const uint64_t wd[2] = {512, (uint64_t)H * 256}, ws[1] = {1024};
+  const uint32_t wb[2] = {64, 128};  // 64 latent columns x 128 value rows (K-major A)
+  const uint64_t xd[3] = {512, (uint64_t)H, (uint64_t)n_rows}, xs[2] = {1024, (uint64_t)H * 1024};
+  uint32_t box[3] = {64, 1, (uint32_t)(n_rows <= 16 ? 16 : n_rows <= 32 ? 32 : n_rows <= 64 ? 64 : n_rows <= 128 ? 128 : 256)};
+  if (!make_map(&tw, wkv_b, 2, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  if (!make_map(&tx, o_lat, 3, xd, xs, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  return dispatch_proj<false, 4>(tw, tx, 1, H, n_rows, 8, 128, out, (int64_t)H * 128, 128, stream);
+}
+
+// ----------------------------------------------------------------- attention
+inline int prefill_splits() { return 1; }
+
+// Split-t plan for decode: enough (row, head group, split) units to give
+// each CTA pair of the GPU one, splits never shorter than one 64-key tile.
+inline int auto_decode_splits(int batch, int H, int64_t max_seqlen_k, int sms) {
+  if (batch <= 0) return 1;
+  const int64_t pairs = sms / 2;
+  const int64_t rows = (int64_t)batch * (H / 128);
+  int64_t s = pairs / rows;
+  const int64_t max_tiles = (max_seqlen_k + kTileN - 1) / kTileN;
+  if (s > max_tiles) s = max_tiles;
+  if (s > 256) s = 256;
+  return s < 1 ? 1 : (int)s;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline size_t workspace_bytes(int H, int64_t n_q, int splits) {
+  if (splits <= 1) return 0;
+  return align256((size_t)splits * n_q * H * 512 * sizeof(float)) + align256((size_t)splits * n_q * H * 2 * sizeof(float));
+}
+
+inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_stride, const void* kv, const void* pe,
+                              int64_t kv_rows, const int32_t* cu_q, const int32_t* cu_k, int batch, int64_t n_q,
+                              int H, int splits, float scale, void* o_lat, void* ws, cudaStream_t stream) {
+  if (kv_rows >= (1LL << 31) || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  const int64_t units = n_q * (H / 128) * splits;
+  if (units == 0) return MLA_OK;
+  if (2 * units >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  CUtensorMap tkv, tpe, tqpe;
+  // kv_rows may be 0 (every sequence empty); the maps still need one row.
+  const uint64_t rows = kv_rows > 0 ? (uint64_t)kv_rows : 1;
+  const uint64_t kd[2] = {512, rows}, ks[1] = {1024};
+  const uint32_t kb[2] = {64, (uint32_t)kTileN};
+  const uint64_t pd[2] = {64, rows}, ps[1] = {128};
+  const uint32_t pb[2] = {32, (uint32_t)kTileN};
+  const uint64_t qd[3] = {192, (uint64_t)H, (uint64_t)n_q}, qs[2] = {384, (uint64_t)q_row_stride * 2};
+  const uint32_t qb[3] = {32, 128, 1};
+  const void* kv_base = kv_rows > 0 ? kv : q_abs;   // any valid 16-byte aligned address for an unused map
+  const void* pe_base = kv_rows > 0 ? pe : q_abs;
+  if (!make_map(&tkv, kv_base, 2, kd, ks, kb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  if (!make_map(&tpe, pe_base, 2, pd, ps, pb, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
+  if (!make_map(&tqpe, q, 3, qd, qs, qb, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
+
+  AttnParams p;
+  p.q_abs = static_cast<const __nv_bfloat16*>(q_abs);
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.batch = batch;
+  p.heads = H;
+  p.head_groups = H / 128;
+  p.num_splits = splits;
+  p.kv_rows = kv_rows;
+  p.n_q = n_q;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_lat = static_cast<__nv_bfloat16*>(o_lat);
+  p.part_o = nullptr;
+  p.part_ml = nullptr;
+  if (splits > 1) {
+    p.part_o = static_cast<float*>(ws);
+    p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)splits * n_q * H * 512 * 4));
+  }
+  if (!set_smem(latent_attn_kernel, AttnLayout::kAlloc)) return MLA_ERR_CUDA;
+  latent_attn_kernel<<<(unsigned)(2 * units), kAttnThreads, AttnLayout::kAlloc, stream>>>(tkv, tpe, tqpe, p);
+  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  if (splits > 1) {
+    merge_splits_kernel<<<dim3((unsigned)n_q, H), 128, 0, stream>>>(p.part_o, p.part_ml, splits, n_q, H,
+                                                                    static_cast<__nv_bfloat16*>(o_lat));
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
 }
 
 }  // namespace sm100

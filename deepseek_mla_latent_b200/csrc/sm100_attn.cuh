@@ -1,0 +1,483 @@
+// sm100_attn.cuh -- latent attention on tcgen05 for the DeepSeek-V3 shapes
+// (C = 512 latent columns, R = 64 rotary columns, 128 heads per row block).
+//
+// Operation ("Naive vs Absorb Attention Implementations in DeepSeek-V3",
+// section "Absorb Path Execution"): for one query row and 128 heads
+//   S[h,t] = (q_abs[h,:] . kv[t,:] + q_pe[h,:] . pe[t,:]) * scale
+//   P      = softmax_t(S)   (keys past the row's visible limit masked)
+//   o[h,:] = sum_t P[h,t] kv[t,:]
+// The latent cache serves as both key and value, so one shared-memory tile
+// of kv feeds both products: K-major for S = Q K^T, MN-major for O = P V.
+//
+// Why a CTA pair: the fp32 accumulator O for 128 heads x 512 columns is
+// 256 KB, all of one SM's tensor memory, leaving nothing for S.  So the two
+// CTAs of a cluster split the latent columns: CTA r keeps O[:, 256r..256r+255]
+// in TMEM and loads only those kv columns (plus rotary columns 32r..32r+31),
+// so no cache byte is read twice.  Each CTA computes the partial score over
+// its 288 contraction columns; the two partials (rounded to fp16 on both
+// sides, so both CTAs add the same two numbers) are exchanged through
+// distributed shared memory with st.async, summed, and both CTAs run the
+// same softmax, getting bit-identical P.
+//
+// Tensor memory (512 columns x 128 lanes, lane = head):
+//   [  0,256) O accumulator (fp32)       [256,384) this CTA's half of q_abs (bf16 pairs, MMA A operand)
+//   [384,448) S buffer 0 (fp32; P overwrites its first 32 columns as bf16 pairs)
+//   [448,512) S buffer 1
+// Shared memory: a 4-stage ring of 64-key tiles (4 x 8 KB latent boxes with
+// 128-byte swizzle + 4 KB rotary box with 64-byte swizzle), this CTA's
+// q_pe half (128 x 32), and a 2-slot inbox for the partner's partial scores.
+//
+// Warps: 0-3 softmax / epilogue (thread h owns head h), 4 TMA producer,
+// 5 MMA issuer and TMEM owner.  The softmax is online with a lazily updated
+// reference max: O is rescaled only when a row max grows by more than 2^8.
+// Every wait is bounded; a wait that runs out raises the device error word
+// and the CTA takes its exit path.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace mla {
+namespace sm100 {
+
+constexpr int kAttnThreads = 192;
+constexpr int kTileN = 64;     // keys per tile
+constexpr int kStages = 4;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+struct AttnLayout {
+  static constexpr int kKvBox = kTileN * 128;           // 64 keys x 64 bf16 latent columns
+  static constexpr int kKv = 4 * kKvBox;                // this CTA's 256 latent columns
+  static constexpr int kPe = kTileN * 64;               // 64 keys x 32 bf16 rotary columns
+  static constexpr int kStage = kKv + kPe;              // 36 KB, a multiple of 1024
+  static constexpr int kQpe = 128 * 64;                 // 128 heads x 32 bf16
+  static constexpr int kInboxSlot = 128 * kTileN * 2;   // 128 heads x 64 fp16 partial scores
+  static constexpr int kOffQpe = kStages * kStage;
+  static constexpr int kOffInbox = kOffQpe + kQpe;
+  static constexpr int kOffBars = kOffInbox + 2 * kInboxSlot;
+  static constexpr int kBytes = kOffBars + 256;
+  static constexpr int kAlloc = kBytes + 1024;          // room to align the base to 1024
+};
+
+struct AttnParams {
+  const __nv_bfloat16* q_abs;   // [n_q, H, 512]
+  const int* cu_q;              // [batch+1] for chunked prefill, nullptr for decode
+  const int* cu_k;              // [batch+1]
+  int batch;
+  int heads;
+  int head_groups;              // heads / 128
+  int num_splits;
+  int64_t kv_rows;
+  int64_t n_q;
+  float scale_log2;             // softmax_scale * log2(e)
+  __nv_bfloat16* o_lat;         // [n_q, H, 512], written when num_splits == 1
+  float* part_o;                // [splits, n_q, H, 512]
+  float* part_ml;               // [splits, n_q, H, 2] = (reference max in log2 units, sum)
+};
+
+__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float2 f16x2_to_f2(uint32_t v) {
+  __half2 h = *reinterpret_cast<__half2*>(&v);
+  return __half22float2(h);
+}
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
+    latent_attn_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_pe,
+                       const __grid_constant__ CUtensorMap tmap_qpe, const AttnParams p) {
+  using L = AttnLayout;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* qpe_s = smem + L::kOffQpe;
+  uint8_t* inbox = smem + L::kOffInbox;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBars);
+  uint64_t* kv_full = bars;             // [kStages]
+  uint64_t* kv_empty = bars + 4;        // [kStages]
+  uint64_t* s_full = bars + 8;          // [2]  QK committed
+  uint64_t* p_ready = bars + 10;        // [2]  P written (128 arrivals)
+  uint64_t* xchg_full = bars + 12;      // [2]  partner's partial scores landed in my inbox
+  uint64_t* xchg_free = bars + 14;      // [2]  partner consumed what I sent (4 arrivals)
+  uint64_t* o_done = bars + 16;         // one phase per PV product
+  uint64_t* q_ready = bars + 17;        // q_abs half stored in TMEM (128 arrivals)
+  uint64_t* qpe_full = bars + 18;
+  uint64_t* mma_idle = bars + 19;       // every MMA of this CTA finished
+  uint64_t* o_final = bars + 20;        // the last PV product finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+
+  const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id();
+  const uint32_t rank = ptx::cluster_rank(), peer = rank ^ 1u;
+
+  // ---- work unit: (query row, head group, split) -------------------------
+  const int64_t unit = blockIdx.x >> 1;
+  const int per_row = p.head_groups * p.num_splits;
+  const int64_t row = unit / per_row;
+  const int hg = (int)((unit % per_row) / p.num_splits);
+  const int sp = (int)(unit % p.num_splits);
+  const int b = p.cu_q ? find_sequence(p.cu_q, p.batch, row) : (int)row;
+  const int64_t k0 = min64(max64(0, __ldg(p.cu_k + b)), p.kv_rows);
+  const int64_t t = max64(0, min64((int64_t)__ldg(p.cu_k + b + 1), p.kv_rows) - k0);
+  int64_t visible = t;
+  if (p.cu_q) {
+    const int64_t q0 = __ldg(p.cu_q + b);
+    const int64_t s = max64(0, (int64_t)__ldg(p.cu_q + b + 1) - q0);
+    visible = min64(t, max64(0, t - s + (row - q0) + 1));
+  }
+  const int64_t per = ((visible + p.num_splits - 1) / p.num_splits + kTileN - 1) / kTileN * kTileN;
+  const int64_t j_begin = min64(visible, (int64_t)sp * per);
+  const int64_t j_end = min64(visible, j_begin + per);
+  const int nt = (int)((j_end - j_begin + kTileN - 1) / kTileN);
+  const int head0 = hg * 128;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(&kv_full[s], 1);
+      ptx::mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&s_full[s], 1);
+      ptx::mbar_init(&p_ready[s], 128);
+      ptx::mbar_init(&xchg_full[s], 1);
+      ptx::mbar_init(&xchg_free[s], 4);
+    }
+    ptx::mbar_init(o_done, 1);
+    ptx::mbar_init(q_ready, 128);
+    ptx::mbar_init(qpe_full, 1);
+    ptx::mbar_init(mma_idle, 1);
+    ptx::mbar_init(o_final, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  ptx::cluster_sync();   // the partner's barriers exist before anything remote touches them
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t kColO = 0, kColQ = 256, kColS = 384;
+
+  if (warp == 4) {
+    // ================================================= TMA producer ======
+    int issued = 0;
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmap_kv);
+      ptx::prefetch_tmap(&tmap_pe);
+      if (nt > 0) {
+        ptx::mbar_arrive_expect_tx(qpe_full, L::kQpe);
+        ptx::tma_load_3d(qpe_s, &tmap_qpe, qpe_full, 128 + 32 * (int)rank, head0, (int)row);
+      }
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % kStages;
+        if (!ptx::mbar_wait(&kv_empty[s], ((j / kStages) & 1) ^ 1, kErrTimeoutStageFree)) break;
+        uint8_t* st = smem + s * L::kStage;
+        ptx::mbar_arrive_expect_tx(&kv_full[s], L::kStage);
+        const int key = (int)(k0 + j_begin + (int64_t)j * kTileN);
+#pragma unroll
+        for (int bx = 0; bx < 4; ++bx)
+          ptx::tma_load_2d(st + bx * L::kKvBox, &tmap_kv, &kv_full[s], 256 * (int)rank + 64 * bx, key);
+        ptx::tma_load_2d(st + L::kKv, &tmap_pe, &kv_full[s], 32 * (int)rank, key);
+        issued = j + 1;
+      }
+      // exit path: every copy this CTA started has landed before its smem goes away
+      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+        ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, kErrTimeoutDrain);
+      if (nt > 0) ptx::mbar_wait(qpe_full, 0, kErrTimeoutDrain);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ================================================= MMA issuer ========
+    if (lane == 0 && nt > 0) {
+      constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(128, kTileN, false, false);
+      constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(128, 256, false, true);
+      bool ok = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax) && ptx::mbar_wait(qpe_full, 0, kErrTimeoutTmaFull);
+      const uint32_t qpe_addr = ptx::smem_u32(qpe_s);
+      auto issue_pv = [&](int j) {
+        const uint32_t st = ptx::smem_u32(smem + (j % kStages) * L::kStage);
+        const uint32_t pcol = tmem + kColS + (j & 1) * kTileN;
+#pragma unroll
+        for (int ks = 0; ks < kTileN / 16; ++ks)
+          ptx::mma_ts(tmem + kColO, pcol + ks * 8, ptx::smem_desc(st + ks * 2048, L::kKvBox, 1024, ptx::kSwizzle128),
+                      idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+        ptx::mma_commit(&kv_empty[j % kStages]);
+        ptx::mma_commit(o_done);
+      };
+      ptx::tc_fence_after();
+      for (int j = 0; ok && j < nt; ++j) {
+        const int s = j % kStages;
+        if (!ptx::mbar_wait(&kv_full[s], (j / kStages) & 1, kErrTimeoutTmaFull)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t st = ptx::smem_u32(smem + s * L::kStage);
+        const uint32_t scol = tmem + kColS + (j & 1) * kTileN;
+#pragma unroll
+        for (int ks = 0; ks < 16; ++ks)
+          ptx::mma_ts(scol, tmem + kColQ + ks * 8,
+                      ptx::smem_desc(st + (ks >> 2) * L::kKvBox + (ks & 3) * 32, 16, 1024, ptx::kSwizzle128),
+                      idesc_qk, ks > 0 ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          ptx::mma_ss(scol, ptx::smem_desc(qpe_addr + ks * 32, 16, 512, ptx::kSwizzle64),
+                      ptx::smem_desc(st + L::kKv + ks * 32, 16, 512, ptx::kSwizzle64), idesc_qk, 1u);
+        ptx::mma_commit(&s_full[j & 1]);
+        if (j > 0) {
+          if (!ptx::mbar_wait(&p_ready[(j - 1) & 1], ((j - 1) >> 1) & 1, kErrTimeoutSoftmax)) { ok = false; break; }
+          ptx::tc_fence_after();
+          issue_pv(j - 1);
+        }
+      }
+      if (ok) {
+        if (ptx::mbar_wait(&p_ready[(nt - 1) & 1], ((nt - 1) >> 1) & 1, kErrTimeoutSoftmax)) {
+          ptx::tc_fence_after();
+          issue_pv(nt - 1);
+          ptx::mma_commit(o_final);
+        }
+      }
+      // nothing of ours may still be running in the tensor core when TMEM is freed
+      ptx::mma_commit(mma_idle);
+      ptx::mbar_wait(mma_idle, 0, kErrTimeoutDrain);
+    }
+    __syncwarp();
+  } else {
+    // ================================================= softmax (warps 0-3)
+    const int h = threadIdx.x;                         // head within the group = TMEM lane
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int64_t head = head0 + h;
+    bool ok = true;
+    float m_ref = -INFINITY, l = 0.f;
+    if (nt > 0) {
+      // this CTA's half of q_abs into TMEM columns [256, 384)
+      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (row * p.heads + head) * 512 + 256 * rank);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint4 x = __ldg(src + c * 8 + v);
+          r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+        }
+        ptx::tmem_st32(tmem + lane_base + kColQ + c * 32, r);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(q_ready);
+
+      const uint32_t inbox_addr = ptx::smem_u32(inbox);
+      const uint32_t peer_inbox = ptx::map_peer(inbox_addr, peer);
+      uint32_t cur[32], nxt[32];
+
+      // Stage A of tile j: read my partial scores, keep them (fp16), send them to the partner.
+      auto stage_a = [&](int j, uint32_t (&own)[32]) -> bool {
+        bool w = ptx::mbar_wait(&s_full[j & 1], (j >> 1) & 1, kErrTimeoutMma);
+        if (!__all_sync(0xffffffffu, w)) return false;
+        ptx::tc_fence_after();
+        uint32_t a[32], c2[32];
+        ptx::tmem_ld32(tmem + lane_base + kColS + (j & 1) * kTileN, a);
+        ptx::tmem_ld32(tmem + lane_base + kColS + (j & 1) * kTileN + 32, c2);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          own[i] = cvt_f16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+          own[16 + i] = cvt_f16x2(__uint_as_float(c2[2 * i]), __uint_as_float(c2[2 * i + 1]));
+        }
+        w = ptx::mbar_wait<true>(&xchg_free[j & 1], ((j >> 1) & 1) ^ 1, kErrTimeoutPeer);
+        if (!__all_sync(0xffffffffu, w)) return false;
+        const uint32_t dst = peer_inbox + (j & 1) * L::kInboxSlot + h * 128;
+        const uint32_t rbar = ptx::map_peer(ptx::smem_u32(&xchg_full[j & 1]), peer);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          ptx::st_async_v4(dst + ((k ^ (h & 7)) << 4), rbar, own[4 * k], own[4 * k + 1], own[4 * k + 2],
+                           own[4 * k + 3]);
+        return true;
+      };
+
+      // Stage B of tile j: add the partner's partial, online softmax, P into TMEM.
+      auto stage_b = [&](int j, const uint32_t (&own)[32]) -> bool {
+        if (h == 0) ptx::mbar_arrive_expect_tx(&xchg_full[j & 1], L::kInboxSlot);
+        bool w = ptx::mbar_wait<true>(&xchg_full[j & 1], (j >> 1) & 1, kErrTimeoutPeer);
+        if (!__all_sync(0xffffffffu, w)) return false;
+        const uint8_t* mine = inbox + (j & 1) * L::kInboxSlot + h * 128;
+        float x[64];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 v = *reinterpret_cast<const uint4*>(mine + ((k ^ (h & 7)) << 4));
+          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 a = f16x2_to_f2(own[4 * k + e]);
+            const float2 c = f16x2_to_f2(pv[e]);
+            x[8 * k + 2 * e] = (a.x + c.x) * p.scale_log2;
+            x[8 * k + 2 * e + 1] = (a.y + c.y) * p.scale_log2;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(&xchg_free[j & 1], peer);
+        const int64_t key0 = j_begin + (int64_t)j * kTileN;
+        const int n_valid = (int)min64(kTileN, j_end - key0);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          if (i >= n_valid) x[i] = -INFINITY;
+          mx = fmaxf(mx, x[i]);
+        }
+        if (j == 0) {
+          m_ref = mx;
+        } else {
+          const bool grow = mx > m_ref + kRescaleThreshold;
+          // TMEM loads/stores are warp-wide: the warp rescales together, lanes
+          // whose row max did not grow use factor 1.
+          if (__any_sync(0xffffffffu, grow)) {
+            // O must not change under us: wait for the PV product of tile j-1
+            w = ptx::mbar_wait(o_done, (j - 1) & 1, kErrTimeoutMma);
+            if (!__all_sync(0xffffffffu, w)) return false;
+            ptx::tc_fence_after();
+            const float f = grow ? fast_exp2(m_ref - mx) : 1.f;
+            l *= f;
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+              uint32_t r[32];
+              ptx::tmem_ld32(tmem + lane_base + kColO + c * 32, r);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+              ptx::tmem_st32(tmem + lane_base + kColO + c * 32, r);
+            }
+            if (grow) m_ref = mx;
+          }
+        }
+        uint32_t pk[32];
+        float psum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float e0 = fast_exp2(x[2 * i] - m_ref), e1 = fast_exp2(x[2 * i + 1] - m_ref);
+          pk[i] = ptx::pack_bf16x2(e0, e1);
+          const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
+          psum += r.x + r.y;
+        }
+        l += psum;
+        ptx::tmem_st32(tmem + lane_base + kColS + (j & 1) * kTileN, pk);
+        if (n_valid < kTileN) {
+          // keys past the end get P = 0, but 0 * NaN is NaN: clear their latent rows
+          uint8_t* st = smem + (j % kStages) * L::kStage;
+          const int rows = kTileN - n_valid;
+          for (int idx = h; idx < rows * 4 * 8; idx += 128) {
+            const int bx = idx / (rows * 8), rem = idx % (rows * 8);
+            *reinterpret_cast<uint4*>(st + bx * L::kKvBox + (n_valid + rem / 8) * 128 + (rem % 8) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&p_ready[j & 1]);
+        return true;
+      };
+
+      ok = stage_a(0, cur);
+      for (int j = 0; ok && j < nt; ++j) {
+        if (j + 1 < nt) {
+          ok = stage_a(j + 1, nxt);
+          if (!ok) break;
+        }
+        ok = stage_b(j, cur);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) cur[i] = nxt[i];
+      }
+    }
+
+    // ---- epilogue ----------------------------------------------------------
+    const int64_t out_row = (row * p.heads + head) * 512 + 256 * rank;
+    if (nt == 0) {
+      if (p.num_splits == 1) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o_lat + out_row);
+        for (int v = 0; v < 32; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+      } else if (rank == 0) {
+        float* ml = p.part_ml + (((int64_t)sp * p.n_q + row) * p.heads + head) * 2;
+        ml[0] = -INFINITY;
+        ml[1] = 0.f;
+      }
+    } else if (ok) {
+      const bool w = ptx::mbar_wait(o_final, 0, kErrTimeoutMma);
+      if (__all_sync(0xffffffffu, w)) {
+        ptx::tc_fence_after();
+        if (p.num_splits == 1) {
+          const float inv = 1.f / l;
+          uint4* dst = reinterpret_cast<uint4*>(p.o_lat + out_row);
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tmem + lane_base + kColO + c * 32, r);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint32_t q4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                q4[e] = ptx::pack_bf16x2(__uint_as_float(r[8 * v + 2 * e]) * inv,
+                                         __uint_as_float(r[8 * v + 2 * e + 1]) * inv);
+              dst[c * 4 + v] = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+            }
+          }
+        } else {
+          const int64_t slot = ((int64_t)sp * p.n_q + row) * p.heads + head;
+          float4* dst = reinterpret_cast<float4*>(p.part_o + slot * 512 + 256 * rank);
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tmem + lane_base + kColO + c * 32, r);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[c * 8 + v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                           __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          }
+          if (rank == 0) {
+            p.part_ml[slot * 2] = m_ref;
+            p.part_ml[slot * 2 + 1] = l;
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 5) ptx::tmem_dealloc(tmem, 512);
+  ptx::cluster_sync();   // the partner no longer writes into this CTA's shared memory
+}
+
+// Merge split partials: o = sum_s 2^{m_s - M} o_s / sum_s 2^{m_s - M} l_s.
+// One block of 128 threads per (row, head); thread i owns columns 4i..4i+3.
+__global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restrict__ part_o,
+                                                           const float* __restrict__ part_ml, int num_splits,
+                                                           int64_t n_q, int heads, __nv_bfloat16* __restrict__ o_lat) {
+  const int64_t row = blockIdx.x;
+  const int head = blockIdx.y;
+  float M = -INFINITY;
+  for (int s = 0; s < num_splits; ++s) M = fmaxf(M, part_ml[(((int64_t)s * n_q + row) * heads + head) * 2]);
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < num_splits; ++s) {
+    const int64_t slot = ((int64_t)s * n_q + row) * heads + head;
+    const float ms = part_ml[slot * 2];
+    if (ms == -INFINITY) continue;
+    const float wgt = exp2f(ms - M);
+    L += wgt * part_ml[slot * 2 + 1];
+    const float4 v = reinterpret_cast<const float4*>(part_o + slot * 512)[threadIdx.x];
+    acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  uint2 o;
+  o.x = ptx::pack_bf16x2(acc.x * inv, acc.y * inv);
+  o.y = ptx::pack_bf16x2(acc.z * inv, acc.w * inv);
+  reinterpret_cast<uint2*>(o_lat + (row * heads + head) * 512)[threadIdx.x] = o;
+}
+
+}  // namespace sm100
+}  // namespace mla

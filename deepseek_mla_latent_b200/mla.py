@@ -102,7 +102,8 @@ def attn_decode(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, kv: torch.Tens
     if ws is None:
         ws = workspace(d, batch, batch, max_seqlen_k, num_splits, device=q_abs.device)
     wsb = ws.numel() if ws is not None else 0
-    _check(LIB.mla_attn_decode(ctypes.byref(d), _ptr(q_abs), _ptr(q), rs, _ptr(kv), _ptr(pe), _ptr(cu_seqlens_k),
+    _check(LIB.mla_attn_decode(ctypes.byref(d), _ptr(q_abs), _ptr(q), rs, _ptr(kv), _ptr(pe), kv.shape[0],
+                               _ptr(cu_seqlens_k),
                                batch, int(max_seqlen_k), _ptr(o_lat), _ptr(ws), wsb, num_splits, _stream(stream)),
            "mla_attn_decode")
     return o_lat
@@ -133,7 +134,7 @@ def attn_prefill_chunk(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, cu_seql
     wsb = ws.numel() if ws is not None else 0
     _check(LIB.mla_attn_prefill_chunk(ctypes.byref(d), _ptr(q_abs), _ptr(q), rs, _ptr(cu_seqlens_q),
                                       _ptr(cu_seqlens_k), batch, n, int(max_seqlen_q), int(max_seqlen_k), _ptr(kv),
-                                      _ptr(pe), _ptr(o_lat), _ptr(ws), wsb, _stream(stream)),
+                                      _ptr(pe), kv.shape[0], _ptr(o_lat), _ptr(ws), wsb, _stream(stream)),
            "mla_attn_prefill_chunk")
     return o_lat
 

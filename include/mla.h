@@ -119,8 +119,10 @@ MLA_API int32_t mla_decode_num_splits(const mla_dims_t* dims, int32_t batch, int
  *   q_abs        [batch, H, C] (from mla_absorb_q).
  *   q            [batch, H, Dn+R] with row stride q_row_stride; the rotary
  *                part q_pe is read from dims Dn..Dn+R-1.
- *   kv_cache     [total_k, C], pe_cache [total_k, R]; sequence b owns rows
+ *   kv_cache     [kv_rows, C], pe_cache [kv_rows, R]; sequence b owns rows
  *                cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1.
+ *   kv_rows      host count of rows in both cache buffers (>= cu_seqlens_k[batch]);
+ *                nothing past it is read (sequence ranges are clamped to it).
  *   cu_seqlens_k device int32 [batch+1], non-decreasing.
  *   max_seqlen_k host upper bound of every sequence length (keys past it
  *                are not read); it sizes the split-t partition.
@@ -133,7 +135,7 @@ MLA_API int32_t mla_decode_num_splits(const mla_dims_t* dims, int32_t batch, int
  */
 MLA_API mla_status_t mla_attn_decode(const mla_dims_t* dims, const void* q_abs, const void* q,
                              int64_t q_row_stride, const void* kv_cache, const void* pe_cache,
-                             const int32_t* cu_seqlens_k, int32_t batch, int64_t max_seqlen_k,
+                             int64_t kv_rows, const int32_t* cu_seqlens_k, int32_t batch, int64_t max_seqlen_k,
                              void* o_lat, void* workspace, size_t workspace_bytes,
                              int32_t num_splits, cudaStream_t stream);
 
@@ -141,7 +143,8 @@ MLA_API mla_status_t mla_attn_decode(const mla_dims_t* dims, const void* q_abs, 
  * new queries whose keys are already the last s_b rows of its cache of
  * t_b rows; query i (0-based) sees keys j <= t_b - s_b + i.
  *   q_abs, q     [total_q, H, C] and [total_q, H, Dn+R] (row stride q_row_stride).
- *   cu_seqlens_q device int32 [batch+1]; cu_seqlens_k as for decode.
+ *   cu_seqlens_q device int32 [batch+1]; cu_seqlens_k, kv_cache, pe_cache,
+ *                kv_rows as for decode.
  *   max_seqlen_q, max_seqlen_k  host upper bounds of s_b and t_b.
  *   o_lat        [total_q, H, C] written.
  *   workspace    at least mla_workspace_size(dims, batch, total_q, max_seqlen_k, 0)
@@ -151,7 +154,7 @@ MLA_API mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* 
                                     int64_t q_row_stride, const int32_t* cu_seqlens_q,
                                     const int32_t* cu_seqlens_k, int32_t batch, int64_t n_q_rows,
                                     int64_t max_seqlen_q, int64_t max_seqlen_k,
-                                    const void* kv_cache, const void* pe_cache, void* o_lat,
+                                    const void* kv_cache, const void* pe_cache, int64_t kv_rows, void* o_lat,
                                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Output projection: out[n,h,d] = sum_c o_lat[n,h,c] * wkv_b[h*(Dn+Dv)+Dn+d, c].

@@ -77,16 +77,16 @@ def test_host_validation_rejects_before_launch(lib):
     assert L.mla_out_proj(ctypes.byref(d), A, None, A, 3, None) == lib.MLA_ERR_INVALID_ARG
     assert L.mla_out_proj(ctypes.byref(d), None, None, None, 0, None) == lib.MLA_OK
     # decode: too many splits, negative batch, missing cache
-    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, A, 2, 128, A, A, 1 << 20, 300, None) \
+    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, 256, A, 2, 128, A, A, 1 << 20, 300, None) \
         == lib.MLA_ERR_INVALID_ARG
-    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, A, -1, 128, A, A, 1 << 20, 0, None) \
+    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, 256, A, -1, 128, A, A, 1 << 20, 0, None) \
         == lib.MLA_ERR_INVALID_ARG
-    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, None, A, A, 2, 128, A, A, 1 << 20, 0, None) \
+    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, None, A, 256, A, 2, 128, A, A, 1 << 20, 0, None) \
         == lib.MLA_ERR_INVALID_ARG
-    assert L.mla_attn_decode(ctypes.byref(d), None, None, 384, None, None, None, 0, 0, None, None, 0, 0, None) \
+    assert L.mla_attn_decode(ctypes.byref(d), None, None, 384, None, None, 0, None, 0, 0, None, None, 0, 0, None) \
         == lib.MLA_OK
     # prefill: missing cu_seqlens_q
-    assert L.mla_attn_prefill_chunk(ctypes.byref(d), A, A, 384, None, A, 2, 8, 4, 128, A, A, A, A, 1 << 20,
+    assert L.mla_attn_prefill_chunk(ctypes.byref(d), A, A, 384, None, A, 2, 8, 4, 128, A, A, 256, A, A, 1 << 20,
                                     None) == lib.MLA_ERR_INVALID_ARG
 
 
@@ -95,9 +95,9 @@ def test_workspace_is_checked(lib):
     d = lib.make_dims(8, 64, 32, 16, 32, "f32", 0.1)
     need = L.mla_workspace_size(ctypes.byref(d), 2, 2, 1 << 16, 4)
     assert need > 0
-    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, A, 2, 1 << 16, A, A, need - 16, 4, None) \
+    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, 1 << 17, A, 2, 1 << 16, A, A, need - 16, 4, None) \
         == lib.MLA_ERR_WORKSPACE
-    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, A, 2, 1 << 16, A, None, need, 4, None) \
+    assert L.mla_attn_decode(ctypes.byref(d), A, A, 384, A, A, 1 << 17, A, 2, 1 << 16, A, None, need, 4, None) \
         == lib.MLA_ERR_WORKSPACE
     assert L.mla_workspace_size(ctypes.byref(d), 2, 2, 1 << 16, 1) == 0
     v3 = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
