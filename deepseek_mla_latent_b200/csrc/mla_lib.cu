@@ -42,6 +42,7 @@ int pick_family(const mla_dims_t* d) {
 bool geo_of(const mla_dims_t* d, Geo* g) {
   g->family = pick_family(d);
   if (g->family < 0) return false;
+  if (!(d->softmax_scale >= 0.f && d->softmax_scale < INFINITY)) return false;
   g->H = d->num_heads; g->C = d->kv_lora_rank; g->Dn = d->qk_nope_head_dim;
   g->R = d->qk_rope_head_dim; g->Dv = d->v_head_dim;
   g->bf16 = d->dtype == MLA_DTYPE_BF16;

@@ -147,6 +147,7 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   if (units == 0) return MLA_OK;
   if (2 * units >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
   CUtensorMap tkv, tpe, tqpe;
+  if ((uint64_t)n_q * H >= (1ULL << 31)) return MLA_ERR_INVALID_ARG;
   // kv_rows may be 0 (every sequence empty); the maps still need one row.
   const uint64_t rows = kv_rows > 0 ? (uint64_t)kv_rows : 1;
   const uint64_t kd[2] = {512, rows}, ks[1] = {1024};
@@ -160,6 +161,10 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   if (!make_map(&tkv, kv_base, 2, kd, ks, kb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   if (!make_map(&tpe, pe_base, 2, pd, ps, pb, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
   if (!make_map(&tqpe, q, 3, qd, qs, qb, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
+  CUtensorMap tqa;   // q_abs viewed as [n_q * H, 512]: boxes of 128 heads x 64 latent columns
+  const uint64_t ad[2] = {512, (uint64_t)n_q * H}, as[1] = {1024};
+  const uint32_t ab[2] = {64, 128};
+  if (!make_map(&tqa, q_abs, 2, ad, as, ab, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
 
   AttnParams p;
   p.q_abs = static_cast<const __nv_bfloat16*>(q_abs);
@@ -180,7 +185,7 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
     p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)splits * n_q * H * 512 * 4));
   }
   if (!set_smem(latent_attn_kernel, AttnLayout::kAlloc)) return MLA_ERR_CUDA;
-  latent_attn_kernel<<<(unsigned)(2 * units), kAttnThreads, AttnLayout::kAlloc, stream>>>(tkv, tpe, tqpe, p);
+  latent_attn_kernel<<<(unsigned)(2 * units), kAttnThreads, AttnLayout::kAlloc, stream>>>(tkv, tpe, tqpe, tqa, p);
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
   if (splits > 1) {
     merge_splits_kernel<<<dim3((unsigned)n_q, H), 128, 0, stream>>>(p.part_o, p.part_ml, splits, n_q, H,

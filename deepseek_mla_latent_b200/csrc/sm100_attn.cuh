@@ -50,10 +50,15 @@ struct AttnLayout {
   static constexpr int kPe = kTileN * 64;               // 64 keys x 32 bf16 rotary columns
   static constexpr int kStage = kKv + kPe;              // 36 KB, a multiple of 1024
   static constexpr int kQpe = 128 * 64;                 // 128 heads x 32 bf16
-  static constexpr int kInboxSlot = 128 * kTileN * 2;   // 128 heads x 64 fp16 partial scores
+  static constexpr int kXchgSlot = 128 * kTileN * 2;    // 128 heads x 64 fp16 partial scores = 16 KB
+  // Exchange area: outbox slots 0,1 then inbox slots 0,1.  Before the first
+  // tile it is the landing zone of this CTA's q_abs half (4 boxes of 128 heads
+  // x 64 latent columns, 16 KB each) on its way into TMEM.
   static constexpr int kOffQpe = kStages * kStage;
-  static constexpr int kOffInbox = kOffQpe + kQpe;
-  static constexpr int kOffBars = kOffInbox + 2 * kInboxSlot;
+  static constexpr int kOffXchg = kOffQpe + kQpe;
+  static constexpr int kOffOutbox = kOffXchg;
+  static constexpr int kOffInbox = kOffXchg + 2 * kXchgSlot;
+  static constexpr int kOffBars = kOffXchg + 4 * kXchgSlot;
   static constexpr int kBytes = kOffBars + 256;
   static constexpr int kAlloc = kBytes + 1024;          // room to align the base to 1024
 };
@@ -91,11 +96,14 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_pe,
-                       const __grid_constant__ CUtensorMap tmap_qpe, const AttnParams p) {
+                       const __grid_constant__ CUtensorMap tmap_qpe, const __grid_constant__ CUtensorMap tmap_qabs,
+                       const AttnParams p) {
   using L = AttnLayout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qpe_s = smem + L::kOffQpe;
+  uint8_t* xchg = smem + L::kOffXchg;
+  uint8_t* outbox = smem + L::kOffOutbox;
   uint8_t* inbox = smem + L::kOffInbox;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBars);
   uint64_t* kv_full = bars;             // [kStages]
@@ -103,13 +111,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   uint64_t* s_full = bars + 8;          // [2]  QK committed
   uint64_t* p_ready = bars + 10;        // [2]  P written (128 arrivals)
   uint64_t* xchg_full = bars + 12;      // [2]  partner's partial scores landed in my inbox
-  uint64_t* xchg_free = bars + 14;      // [2]  partner consumed what I sent (4 arrivals)
+  uint64_t* xchg_free = bars + 14;      // [2]  partner's inbox slot is free (4 arrivals from its warps)
   uint64_t* o_done = bars + 16;         // one phase per PV product
   uint64_t* q_ready = bars + 17;        // q_abs half stored in TMEM (128 arrivals)
   uint64_t* qpe_full = bars + 18;
   uint64_t* mma_idle = bars + 19;       // every MMA of this CTA finished
   uint64_t* o_final = bars + 20;        // the last PV product finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+  uint64_t* q_full = bars + 21;         // q_abs half landed in the exchange area
+  uint64_t* outbox_ready = bars + 22;   // [2]  all 128 rows of my partial written (128 arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
 
   const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id();
   const uint32_t rank = ptx::cluster_rank(), peer = rank ^ 1u;
@@ -151,6 +161,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     ptx::mbar_init(qpe_full, 1);
     ptx::mbar_init(mma_idle, 1);
     ptx::mbar_init(o_final, 1);
+    ptx::mbar_init(q_full, 1);
+    ptx::mbar_init(&outbox_ready[0], 128);
+    ptx::mbar_init(&outbox_ready[1], 128);
     ptx::fence_mbar_init();
   }
   if (warp == 5) {
@@ -171,6 +184,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       ptx::prefetch_tmap(&tmap_kv);
       ptx::prefetch_tmap(&tmap_pe);
       if (nt > 0) {
+        ptx::mbar_arrive_expect_tx(q_full, 4 * L::kXchgSlot);
+#pragma unroll
+        for (int bx = 0; bx < 4; ++bx)
+          ptx::tma_load_2d(xchg + bx * L::kXchgSlot, &tmap_qabs, q_full, 256 * (int)rank + 64 * bx,
+                           (int)(row * p.heads + head0));
         ptx::mbar_arrive_expect_tx(qpe_full, L::kQpe);
         ptx::tma_load_3d(qpe_s, &tmap_qpe, qpe_full, 128 + 32 * (int)rank, head0, (int)row);
       }
@@ -189,7 +207,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       // exit path: every copy this CTA started has landed before its smem goes away
       for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
         ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, kErrTimeoutDrain);
-      if (nt > 0) ptx::mbar_wait(qpe_full, 0, kErrTimeoutDrain);
+      if (nt > 0) {
+        ptx::mbar_wait(qpe_full, 0, kErrTimeoutDrain);
+        ptx::mbar_wait(q_full, 0, kErrTimeoutDrain);
+      }
     }
     __syncwarp();
   } else if (warp == 5) {
@@ -252,72 +273,95 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     bool ok = true;
     float m_ref = -INFINITY, l = 0.f;
     if (nt > 0) {
-      // this CTA's half of q_abs into TMEM columns [256, 384)
-      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (row * p.heads + head) * 512 + 256 * rank);
+      // this CTA's half of q_abs: exchange area (TMA, 128-byte swizzle) -> TMEM columns [256, 384)
+      bool w = ptx::mbar_wait(q_full, 0, kErrTimeoutTmaFull);
+      ok = __all_sync(0xffffffffu, w);
+      if (ok) {
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
+        for (int c = 0; c < 4; ++c) {
+          const uint8_t* src = xchg + c * L::kXchgSlot + h * 128;
+          uint32_t r[32];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          uint4 x = __ldg(src + c * 8 + v);
-          r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+          for (int v = 0; v < 8; ++v) {
+            const uint4 x = *reinterpret_cast<const uint4*>(src + ((v ^ (h & 7)) << 4));
+            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+          }
+          ptx::tmem_st32(tmem + lane_base + kColQ + c * 32, r);
         }
-        ptx::tmem_st32(tmem + lane_base + kColQ + c * 32, r);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(q_ready);
+        // the exchange area is free again: tell the partner it may send into my inbox
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive_cluster(&xchg_free[0], peer);
+          ptx::mbar_arrive_cluster(&xchg_free[1], peer);
+        }
       }
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(q_ready);
 
-      const uint32_t inbox_addr = ptx::smem_u32(inbox);
-      const uint32_t peer_inbox = ptx::map_peer(inbox_addr, peer);
-      uint32_t cur[32], nxt[32];
+      const uint32_t peer_inbox = ptx::map_peer(ptx::smem_u32(inbox), peer);
+      const uint32_t peer_full0 = ptx::map_peer(ptx::smem_u32(&xchg_full[0]), peer);
+      const uint32_t peer_full1 = ptx::map_peer(ptx::smem_u32(&xchg_full[1]), peer);
+      const float sl2 = p.scale_log2;
 
-      // Stage A of tile j: read my partial scores, keep them (fp16), send them to the partner.
-      auto stage_a = [&](int j, uint32_t (&own)[32]) -> bool {
-        bool w = ptx::mbar_wait(&s_full[j & 1], (j >> 1) & 1, kErrTimeoutMma);
-        if (!__all_sync(0xffffffffu, w)) return false;
+      for (int j = 0; ok && j < nt; ++j) {
+        const int slot = j & 1;
+        const uint32_t par = (j >> 1) & 1;
+        // --- my partial scores: TMEM -> fp16 -> outbox -> one bulk copy into the partner's inbox
+        w = ptx::mbar_wait(&s_full[slot], par, kErrTimeoutMma);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         ptx::tc_fence_after();
-        uint32_t a[32], c2[32];
-        ptx::tmem_ld32(tmem + lane_base + kColS + (j & 1) * kTileN, a);
-        ptx::tmem_ld32(tmem + lane_base + kColS + (j & 1) * kTileN + 32, c2);
-        ptx::tmem_wait_ld();
+        uint32_t own[32];
+        {
+          uint32_t a[32], c2[32];
+          ptx::tmem_ld32(tmem + lane_base + kColS + slot * kTileN, a);
+          ptx::tmem_ld32(tmem + lane_base + kColS + slot * kTileN + 32, c2);
+          ptx::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          own[i] = cvt_f16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
-          own[16 + i] = cvt_f16x2(__uint_as_float(c2[2 * i]), __uint_as_float(c2[2 * i + 1]));
+          for (int i = 0; i < 16; ++i) {
+            own[i] = cvt_f16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+            own[16 + i] = cvt_f16x2(__uint_as_float(c2[2 * i]), __uint_as_float(c2[2 * i + 1]));
+          }
         }
-        w = ptx::mbar_wait<true>(&xchg_free[j & 1], ((j >> 1) & 1) ^ 1, kErrTimeoutPeer);
-        if (!__all_sync(0xffffffffu, w)) return false;
-        const uint32_t dst = peer_inbox + (j & 1) * L::kInboxSlot + h * 128;
-        const uint32_t rbar = ptx::map_peer(ptx::smem_u32(&xchg_full[j & 1]), peer);
+        w = ptx::mbar_wait<true>(&xchg_free[slot], par, kErrTimeoutPeer);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        {
+          uint8_t* dst = outbox + slot * L::kXchgSlot + h * 128;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          ptx::st_async_v4(dst + ((k ^ (h & 7)) << 4), rbar, own[4 * k], own[4 * k + 1], own[4 * k + 2],
-                           own[4 * k + 3]);
-        return true;
-      };
-
-      // Stage B of tile j: add the partner's partial, online softmax, P into TMEM.
-      auto stage_b = [&](int j, const uint32_t (&own)[32]) -> bool {
-        if (h == 0) ptx::mbar_arrive_expect_tx(&xchg_full[j & 1], L::kInboxSlot);
-        bool w = ptx::mbar_wait<true>(&xchg_full[j & 1], (j >> 1) & 1, kErrTimeoutPeer);
-        if (!__all_sync(0xffffffffu, w)) return false;
-        const uint8_t* mine = inbox + (j & 1) * L::kInboxSlot + h * 128;
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint4*>(dst + ((k ^ (h & 7)) << 4)) =
+                make_uint4(own[4 * k], own[4 * k + 1], own[4 * k + 2], own[4 * k + 3]);
+        }
+        ptx::fence_async_smem();
+        ptx::mbar_arrive(&outbox_ready[slot]);
+        if (h == 0) {
+          // every row is in the outbox (a bounded wait, unlike a named barrier) -> one bulk copy
+          if (ptx::mbar_wait(&outbox_ready[slot], par, kErrTimeoutSoftmax))
+            ptx::bulk_copy_to_peer(peer_inbox + slot * L::kXchgSlot, ptx::smem_u32(outbox + slot * L::kXchgSlot),
+                                   L::kXchgSlot, slot ? peer_full1 : peer_full0);
+          ptx::mbar_arrive_expect_tx(&xchg_full[slot], L::kXchgSlot);
+        }
+        // --- the partner's partial: add, online softmax, P into TMEM
+        w = ptx::mbar_wait<true>(&xchg_full[slot], par, kErrTimeoutPeer);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         float x[64];
+        {
+          const uint8_t* mine = inbox + slot * L::kXchgSlot + h * 128;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint4 v = *reinterpret_cast<const uint4*>(mine + ((k ^ (h & 7)) << 4));
-          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+          for (int k = 0; k < 8; ++k) {
+            const uint4 v = *reinterpret_cast<const uint4*>(mine + ((k ^ (h & 7)) << 4));
+            const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 a = f16x2_to_f2(own[4 * k + e]);
-            const float2 c = f16x2_to_f2(pv[e]);
-            x[8 * k + 2 * e] = (a.x + c.x) * p.scale_log2;
-            x[8 * k + 2 * e + 1] = (a.y + c.y) * p.scale_log2;
+            for (int e = 0; e < 4; ++e) {
+              const float2 a = f16x2_to_f2(own[4 * k + e]);
+              const float2 c = f16x2_to_f2(pv[e]);
+              x[8 * k + 2 * e] = a.x + c.x;
+              x[8 * k + 2 * e + 1] = a.y + c.y;
+            }
           }
         }
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_cluster(&xchg_free[j & 1], peer);
+        if (lane == 0) ptx::mbar_arrive_cluster(&xchg_free[slot], peer);   // my inbox slot is free again
         const int64_t key0 = j_begin + (int64_t)j * kTileN;
         const int n_valid = (int)min64(kTileN, j_end - key0);
         float mx = -INFINITY;
@@ -326,6 +370,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           if (i >= n_valid) x[i] = -INFINITY;
           mx = fmaxf(mx, x[i]);
         }
+        mx *= sl2;   // scale >= 0: the max of scaled scores is the scaled max
         if (j == 0) {
           m_ref = mx;
         } else {
@@ -335,7 +380,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           if (__any_sync(0xffffffffu, grow)) {
             // O must not change under us: wait for the PV product of tile j-1
             w = ptx::mbar_wait(o_done, (j - 1) & 1, kErrTimeoutMma);
-            if (!__all_sync(0xffffffffu, w)) return false;
+            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             ptx::tc_fence_after();
             const float f = grow ? fast_exp2(m_ref - mx) : 1.f;
             l *= f;
@@ -355,13 +400,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         float psum = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float e0 = fast_exp2(x[2 * i] - m_ref), e1 = fast_exp2(x[2 * i + 1] - m_ref);
+          const float e0 = fast_exp2(fmaf(x[2 * i], sl2, -m_ref));
+          const float e1 = fast_exp2(fmaf(x[2 * i + 1], sl2, -m_ref));
           pk[i] = ptx::pack_bf16x2(e0, e1);
-          const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
-          psum += r.x + r.y;
+          psum += e0 + e1;
         }
         l += psum;
-        ptx::tmem_st32(tmem + lane_base + kColS + (j & 1) * kTileN, pk);
+        ptx::tmem_st32(tmem + lane_base + kColS + slot * kTileN, pk);
         if (n_valid < kTileN) {
           // keys past the end get P = 0, but 0 * NaN is NaN: clear their latent rows
           uint8_t* st = smem + (j % kStages) * L::kStage;
@@ -371,23 +416,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
             *reinterpret_cast<uint4*>(st + bx * L::kKvBox + (n_valid + rem / 8) * 128 + (rem % 8) * 16) =
                 make_uint4(0, 0, 0, 0);
           }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          ptx::fence_async_smem();
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&p_ready[j & 1]);
-        return true;
-      };
-
-      ok = stage_a(0, cur);
-      for (int j = 0; ok && j < nt; ++j) {
-        if (j + 1 < nt) {
-          ok = stage_a(j + 1, nxt);
-          if (!ok) break;
-        }
-        ok = stage_b(j, cur);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) cur[i] = nxt[i];
+        ptx::mbar_arrive(&p_ready[slot]);
       }
     }
 

@@ -226,15 +226,20 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-// 16-byte store into the peer CTA's shared memory; completion is counted in
-// bytes on the peer's mbarrier (both addresses from map_peer).
-__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t remote_bar, uint32_t a, uint32_t b,
-                                            uint32_t c, uint32_t d) {
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into the
+// shared memory of another CTA of the cluster; completion is counted in bytes
+// on the destination CTA's mbarrier (dst and bar from map_peer).
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
   asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%2, %3, %4, %5}, [%1];" ::"r"(
-          remote_addr),
-      "r"(remote_bar), "r"(a), "r"(b), "r"(c), "r"(d)
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "r"(src), "r"(bytes), "r"(bar)
       : "memory");
+}
+// Make this thread's generic-proxy shared-memory writes visible to async-proxy readers (TMA, bulk copy, MMA).
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Named barrier over `count` threads (id 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

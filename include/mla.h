@@ -74,7 +74,8 @@ typedef enum mla_dtype { MLA_DTYPE_BF16 = 0, MLA_DTYPE_F32 = 1 } mla_dtype_t;
 
 /* Head geometry.  H = num_heads, C = kv_lora_rank, Dn = qk_nope_head_dim,
  * R = qk_rope_head_dim, Dv = v_head_dim.  softmax_scale multiplies the scores
- * (DeepSeek-V3 without YaRN: 1/sqrt(Dn + R)).
+ * (DeepSeek-V3 without YaRN: 1/sqrt(Dn + R)); it must be finite and >= 0
+ * (calls with other values return MLA_ERR_UNSUPPORTED).
  *
  * bf16 runs on the tcgen05 tensor-core kernels when C = 512, R = 64,
  * Dn = Dv = 128 and H is a multiple of 128 (the DeepSeek-V3 shapes); other
