@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "mla.h"
 #include "common.cuh"
@@ -117,6 +118,28 @@ size_t workspace_bytes_for(const Geo& g, int32_t batch, int64_t n_q_rows, int64_
                            bool decode) {
   if (g.family == 1) return mla::sm100::workspace_bytes(g.H, n_q_rows, splits);
   return simt_workspace(g, n_q_rows, splits);
+}
+
+// Scratch for mla_attn_decode_static_scratch: one array per device that loads
+// the library, for callers that cannot allocate.  Host code only ever uses
+// the device address looked up below, never this symbol directly.
+static __device__ __align__(256) unsigned char g_static_scratch[MLA_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device (looked up once per device).
+void* static_scratch_for_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev] = ptr;
+  }
+  return g_scratch_ptr[dev];
 }
 
 }  // namespace
@@ -238,6 +261,29 @@ mla_status_t mla_attn_decode(const mla_dims_t* dims, const void* q_abs, const vo
                                     batch, batch, splits, o_lat, workspace, stream);
   return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, nullptr, cu_seqlens_k, batch,
                                batch, splits, o_lat, workspace, stream);
+}
+
+mla_status_t mla_attn_decode_static_scratch(const mla_dims_t* dims, const void* q_abs, const void* q,
+                                            int64_t q_row_stride, const void* kv_cache, const void* pe_cache,
+                                            int64_t kv_rows, const int32_t* cu_seqlens_k, int32_t batch,
+                                            int64_t max_seqlen_k, void* o_lat, int32_t num_splits,
+                                            cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (batch < 0 || max_seqlen_k < 0 || num_splits < 0 || num_splits > 256) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  const int splits = resolve_splits(g, batch, batch, max_seqlen_k, num_splits, true);
+  const size_t need = workspace_bytes_for(g, batch, batch, max_seqlen_k, splits, true);
+  if (need > (size_t)MLA_STATIC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (need > 0) {
+    ws = static_scratch_for_current_device();
+    if (!ws) return MLA_ERR_CUDA;
+  }
+  return mla_attn_decode(dims, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_k, batch,
+                         max_seqlen_k, o_lat, ws, need > 0 ? (size_t)MLA_STATIC_SCRATCH_BYTES : 0, num_splits,
+                         stream);
 }
 
 mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,

@@ -140,6 +140,35 @@ MLA_API mla_status_t mla_attn_decode(const mla_dims_t* dims, const void* q_abs, 
                              void* o_lat, void* workspace, size_t workspace_bytes,
                              int32_t num_splits, cudaStream_t stream);
 
+/* Size of the device scratch array behind mla_attn_decode_static_scratch. */
+#define MLA_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* mla_attn_decode without a caller-provided workspace.  The paper has no
+ * counterpart to this call; it exists for callers that cannot allocate
+ * device memory: code that only receives input and output buffers from a
+ * host framework with no allocator to call, and code on a path where
+ * cudaMalloc is not allowed or would synchronise the device (inside a
+ * stream capture in global mode, a latency-bound decode loop).
+ *
+ * Arguments are those of mla_attn_decode minus the workspace.  The split-t
+ * partials go to one library-owned device array of MLA_STATIC_SCRATCH_BYTES
+ * per GPU, held from the library's first use on that GPU until the process
+ * exits.  The call allocates and frees nothing.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - If the split plan needs more than MLA_STATIC_SCRATCH_BYTES (as
+ *     mla_workspace_size would report), the call returns MLA_ERR_WORKSPACE
+ *     and launches nothing; pass a smaller num_splits or use mla_attn_decode.
+ *   - Every call on a device shares the array and leaves its partials there;
+ *     nothing in it needs to start at zero.  Calls that overlap on the GPU
+ *     (other streams, other host threads) race on it: serialise them. */
+MLA_API mla_status_t mla_attn_decode_static_scratch(const mla_dims_t* dims, const void* q_abs, const void* q,
+                                                    int64_t q_row_stride, const void* kv_cache,
+                                                    const void* pe_cache, int64_t kv_rows,
+                                                    const int32_t* cu_seqlens_k, int32_t batch,
+                                                    int64_t max_seqlen_k, void* o_lat, int32_t num_splits,
+                                                    cudaStream_t stream);
+
 /* Chunked-prefill attention: sequence b has s_b = cu_seqlens_q[b+1]-cu_seqlens_q[b]
  * new queries whose keys are already the last s_b rows of its cache of
  * t_b rows; query i (0-based) sees keys j <= t_b - s_b + i.
