@@ -72,12 +72,15 @@ inline mla_status_t launch_proj(const CUtensorMap& tw, const CUtensorMap& tx, di
   return last_launch();
 }
 
-template <bool A_MN, int STAGES>
+// STAGES: the K ring depth; with few query rows the whole weight tile of a
+// CTA is kept in flight (the projection is a weight stream at decode sizes).
+template <bool A_MN, int MAX_STAGES>
 inline mla_status_t dispatch_proj(const CUtensorMap& tw, const CUtensorMap& tx, int m_tiles, int H, int64_t n_rows,
                                   int k_chunks, int w_row_base, void* out, int64_t out_row_stride,
                                   int out_head_stride, cudaStream_t stream) {
   auto go = [&](auto tile) {
     constexpr int NT = decltype(tile)::value;
+    constexpr int STAGES = NT <= 64 ? MAX_STAGES : (MAX_STAGES < 4 ? MAX_STAGES : 4);
     dim3 grid(m_tiles, H, (unsigned)((n_rows + NT - 1) / NT));
     return launch_proj<A_MN, NT, STAGES>(tw, tx, grid, k_chunks, w_row_base, (int)n_rows, out, out_row_stride,
                                          out_head_stride, stream);
@@ -113,7 +116,7 @@ inline mla_status_t out_proj(const void* o_lat, const void* wkv_b, void* out, in
   uint32_t box[3] = {64, 1, (uint32_t)(n_rows <= 16 ? 16 : n_rows <= 32 ? 32 : n_rows <= 64 ? 64 : n_rows <= 128 ? 128 : 256)};
   if (!make_map(&tw, wkv_b, 2, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   if (!make_map(&tx, o_lat, 3, xd, xs, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-  return dispatch_proj<false, 4>(tw, tx, 1, H, n_rows, 8, 128, out, (int64_t)H * 128, 128, stream);
+  return dispatch_proj<false, 8>(tw, tx, 1, H, n_rows, 8, 128, out, (int64_t)H * 128, 128, stream);
 }
 
 // ----------------------------------------------------------------- attention

@@ -21,17 +21,22 @@
 //
 // Tensor memory (512 columns x 128 lanes, lane = head):
 //   [  0,256) O accumulator (fp32)       [256,384) this CTA's half of q_abs (bf16 pairs, MMA A operand)
-//   [384,448) S buffer 0 (fp32; P overwrites its first 32 columns as bf16 pairs)
-//   [448,512) S buffer 1
-// Shared memory: a 4-stage ring of 64-key tiles (4 x 8 KB latent boxes with
-// 128-byte swizzle + 4 KB rotary box with 64-byte swizzle), this CTA's
-// q_pe half (128 x 32), and a 2-slot inbox for the partner's partial scores.
+//   [384,448) S buffer 0 (fp32)          [448,512) S buffer 1
+// Shared memory: a 3-stage ring of 64-key tiles (4 x 8 KB latent boxes with
+// 128-byte swizzle + 4 KB rotary box with 64-byte swizzle), this CTA's q_pe
+// half (128 x 32), two P buffers (128 heads x 64 keys bf16, the A operand of
+// O += P V), and the exchange area (2-slot outbox and inbox of fp16 partial
+// scores, one 16 KB bulk copy per tile).  P lives in shared memory so an S
+// buffer is free as soon as the softmax has read it: QK of tile j+2 does not
+// wait for the P V product of tile j.
 //
 // Warps: 0-3 softmax / epilogue (thread h owns head h), 4 TMA producer,
-// 5 MMA issuer and TMEM owner.  The softmax is online with a lazily updated
-// reference max: O is rescaled only when a row max grows by more than 2^8.
-// Every wait is bounded; a wait that runs out raises the device error word
-// and the CTA takes its exit path.
+// 5 MMA issuer and TMEM owner.  The softmax runs one tile ahead on the
+// exchange: it reads and sends the partial scores of tile j+1 before it
+// finishes tile j, so the partner's data for a tile is usually there when it
+// is needed.  It is online with a lazily updated reference max: O is rescaled
+// only when a row max grows by more than 2^8.  Every wait is bounded; a wait
+// that runs out raises the device error word and the CTA takes its exit path.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -41,7 +46,7 @@ namespace sm100 {
 
 constexpr int kAttnThreads = 192;
 constexpr int kTileN = 64;     // keys per tile
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct AttnLayout {
@@ -50,12 +55,14 @@ struct AttnLayout {
   static constexpr int kPe = kTileN * 64;               // 64 keys x 32 bf16 rotary columns
   static constexpr int kStage = kKv + kPe;              // 36 KB, a multiple of 1024
   static constexpr int kQpe = 128 * 64;                 // 128 heads x 32 bf16
+  static constexpr int kP = 128 * kTileN * 2;           // 128 heads x 64 keys bf16 = 16 KB
   static constexpr int kXchgSlot = 128 * kTileN * 2;    // 128 heads x 64 fp16 partial scores = 16 KB
   // Exchange area: outbox slots 0,1 then inbox slots 0,1.  Before the first
   // tile it is the landing zone of this CTA's q_abs half (4 boxes of 128 heads
   // x 64 latent columns, 16 KB each) on its way into TMEM.
   static constexpr int kOffQpe = kStages * kStage;
-  static constexpr int kOffXchg = kOffQpe + kQpe;
+  static constexpr int kOffP = kOffQpe + kQpe;
+  static constexpr int kOffXchg = kOffP + 2 * kP;
   static constexpr int kOffOutbox = kOffXchg;
   static constexpr int kOffInbox = kOffXchg + 2 * kXchgSlot;
   static constexpr int kOffBars = kOffXchg + 4 * kXchgSlot;
@@ -102,23 +109,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qpe_s = smem + L::kOffQpe;
+  uint8_t* p_s = smem + L::kOffP;
   uint8_t* xchg = smem + L::kOffXchg;
   uint8_t* outbox = smem + L::kOffOutbox;
   uint8_t* inbox = smem + L::kOffInbox;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBars);
-  uint64_t* kv_full = bars;             // [kStages]
-  uint64_t* kv_empty = bars + 4;        // [kStages]
-  uint64_t* s_full = bars + 8;          // [2]  QK committed
+  uint64_t* kv_full = bars;             // [3]  TMA tile landed
+  uint64_t* kv_empty = bars + 3;        // [3]  tile no longer read by the tensor core
+  uint64_t* s_full = bars + 6;          // [2]  QK product committed
+  uint64_t* s_free = bars + 8;          // [2]  softmax read S (128 arrivals)
   uint64_t* p_ready = bars + 10;        // [2]  P written (128 arrivals)
   uint64_t* xchg_full = bars + 12;      // [2]  partner's partial scores landed in my inbox
   uint64_t* xchg_free = bars + 14;      // [2]  partner's inbox slot is free (4 arrivals from its warps)
-  uint64_t* o_done = bars + 16;         // one phase per PV product
-  uint64_t* q_ready = bars + 17;        // q_abs half stored in TMEM (128 arrivals)
-  uint64_t* qpe_full = bars + 18;
-  uint64_t* mma_idle = bars + 19;       // every MMA of this CTA finished
-  uint64_t* o_final = bars + 20;        // the last PV product finished
+  uint64_t* outbox_ready = bars + 16;   // [2]  all 128 rows of my partial written (128 arrivals)
+  uint64_t* o_done = bars + 18;         // one phase per P V product
+  uint64_t* o_final = bars + 19;        // the last P V product finished
+  uint64_t* q_ready = bars + 20;        // q_abs half stored in TMEM (128 arrivals)
   uint64_t* q_full = bars + 21;         // q_abs half landed in the exchange area
-  uint64_t* outbox_ready = bars + 22;   // [2]  all 128 rows of my partial written (128 arrivals)
+  uint64_t* qpe_full = bars + 22;
+  uint64_t* mma_idle = bars + 23;       // every MMA of this CTA finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
 
   const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id();
@@ -152,18 +161,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&s_full[s], 1);
+      ptx::mbar_init(&s_free[s], 128);
       ptx::mbar_init(&p_ready[s], 128);
       ptx::mbar_init(&xchg_full[s], 1);
       ptx::mbar_init(&xchg_free[s], 4);
+      ptx::mbar_init(&outbox_ready[s], 128);
     }
     ptx::mbar_init(o_done, 1);
+    ptx::mbar_init(o_final, 1);
     ptx::mbar_init(q_ready, 128);
+    ptx::mbar_init(q_full, 1);
     ptx::mbar_init(qpe_full, 1);
     ptx::mbar_init(mma_idle, 1);
-    ptx::mbar_init(o_final, 1);
-    ptx::mbar_init(q_full, 1);
-    ptx::mbar_init(&outbox_ready[0], 128);
-    ptx::mbar_init(&outbox_ready[1], 128);
     ptx::fence_mbar_init();
   }
   if (warp == 5) {
@@ -215,18 +224,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else if (warp == 5) {
     // ================================================= MMA issuer ========
+    // Order: QK(0), QK(1), PV(0), QK(2), PV(1), ...  QK(j) needs its tile and
+    // S buffer j&1 read out (tile j-2); PV(j) needs P(j).
     if (lane == 0 && nt > 0) {
       constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(128, kTileN, false, false);
       constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(128, 256, false, true);
       bool ok = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax) && ptx::mbar_wait(qpe_full, 0, kErrTimeoutTmaFull);
       const uint32_t qpe_addr = ptx::smem_u32(qpe_s);
+      const uint32_t p_addr = ptx::smem_u32(p_s);
       auto issue_pv = [&](int j) {
         const uint32_t st = ptx::smem_u32(smem + (j % kStages) * L::kStage);
-        const uint32_t pcol = tmem + kColS + (j & 1) * kTileN;
+        const uint32_t pa = p_addr + (j & 1) * L::kP;
 #pragma unroll
         for (int ks = 0; ks < kTileN / 16; ++ks)
-          ptx::mma_ts(tmem + kColO, pcol + ks * 8, ptx::smem_desc(st + ks * 2048, L::kKvBox, 1024, ptx::kSwizzle128),
-                      idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+          ptx::mma_ss(tmem + kColO, ptx::smem_desc(pa + ks * 32, 16, 1024, ptx::kSwizzle128),
+                      ptx::smem_desc(st + ks * 2048, L::kKvBox, 1024, ptx::kSwizzle128), idesc_pv,
+                      (j > 0 || ks > 0) ? 1u : 0u);
         ptx::mma_commit(&kv_empty[j % kStages]);
         ptx::mma_commit(o_done);
       };
@@ -234,6 +247,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       for (int j = 0; ok && j < nt; ++j) {
         const int s = j % kStages;
         if (!ptx::mbar_wait(&kv_full[s], (j / kStages) & 1, kErrTimeoutTmaFull)) { ok = false; break; }
+        if (j >= 2 && !ptx::mbar_wait(&s_free[j & 1], ((j - 2) >> 1) & 1, kErrTimeoutSoftmax)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint32_t st = ptx::smem_u32(smem + s * L::kStage);
         const uint32_t scol = tmem + kColS + (j & 1) * kTileN;
@@ -253,12 +267,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           issue_pv(j - 1);
         }
       }
-      if (ok) {
-        if (ptx::mbar_wait(&p_ready[(nt - 1) & 1], ((nt - 1) >> 1) & 1, kErrTimeoutSoftmax)) {
-          ptx::tc_fence_after();
-          issue_pv(nt - 1);
-          ptx::mma_commit(o_final);
-        }
+      if (ok && ptx::mbar_wait(&p_ready[(nt - 1) & 1], ((nt - 1) >> 1) & 1, kErrTimeoutSoftmax)) {
+        ptx::tc_fence_after();
+        issue_pv(nt - 1);
+        ptx::mma_commit(o_final);
       }
       // nothing of ours may still be running in the tensor core when TMEM is freed
       ptx::mma_commit(mma_idle);
@@ -270,6 +282,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     const int h = threadIdx.x;                         // head within the group = TMEM lane
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const int64_t head = head0 + h;
+    const uint32_t sw = (uint32_t)(h & 7);             // 128-byte swizzle phase of row h
     bool ok = true;
     float m_ref = -INFINITY, l = 0.f;
     if (nt > 0) {
@@ -283,7 +296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           uint32_t r[32];
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
-            const uint4 x = *reinterpret_cast<const uint4*>(src + ((v ^ (h & 7)) << 4));
+            const uint4 x = *reinterpret_cast<const uint4*>(src + ((v ^ sw) << 4));
             r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
           }
           ptx::tmem_st32(tmem + lane_base + kColQ + c * 32, r);
@@ -304,19 +317,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       const uint32_t peer_full1 = ptx::map_peer(ptx::smem_u32(&xchg_full[1]), peer);
       const float sl2 = p.scale_log2;
 
-      for (int j = 0; ok && j < nt; ++j) {
+      // Send: my partial scores of tile j (TMEM -> fp16 -> outbox -> one bulk
+      // copy into the partner's inbox); they are kept in `own` for the sum.
+      auto send = [&](int j, uint32_t (&own)[32]) -> bool {
         const int slot = j & 1;
         const uint32_t par = (j >> 1) & 1;
-        // --- my partial scores: TMEM -> fp16 -> outbox -> one bulk copy into the partner's inbox
-        w = ptx::mbar_wait(&s_full[slot], par, kErrTimeoutMma);
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        bool w = ptx::mbar_wait(&s_full[slot], par, kErrTimeoutMma);
+        if (!__all_sync(0xffffffffu, w)) return false;
         ptx::tc_fence_after();
-        uint32_t own[32];
         {
           uint32_t a[32], c2[32];
           ptx::tmem_ld32(tmem + lane_base + kColS + slot * kTileN, a);
           ptx::tmem_ld32(tmem + lane_base + kColS + slot * kTileN + 32, c2);
           ptx::tmem_wait_ld();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&s_free[slot]);               // S buffer may take QK(j+2)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             own[i] = cvt_f16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
@@ -324,14 +339,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           }
         }
         w = ptx::mbar_wait<true>(&xchg_free[slot], par, kErrTimeoutPeer);
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        {
-          uint8_t* dst = outbox + slot * L::kXchgSlot + h * 128;
+        if (!__all_sync(0xffffffffu, w)) return false;
+        uint8_t* dst = outbox + slot * L::kXchgSlot + h * 128;
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<uint4*>(dst + ((k ^ (h & 7)) << 4)) =
-                make_uint4(own[4 * k], own[4 * k + 1], own[4 * k + 2], own[4 * k + 3]);
-        }
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4*>(dst + ((k ^ sw) << 4)) =
+              make_uint4(own[4 * k], own[4 * k + 1], own[4 * k + 2], own[4 * k + 3]);
         ptx::fence_async_smem();
         ptx::mbar_arrive(&outbox_ready[slot]);
         if (h == 0) {
@@ -341,15 +354,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
                                    L::kXchgSlot, slot ? peer_full1 : peer_full0);
           ptx::mbar_arrive_expect_tx(&xchg_full[slot], L::kXchgSlot);
         }
-        // --- the partner's partial: add, online softmax, P into TMEM
-        w = ptx::mbar_wait<true>(&xchg_full[slot], par, kErrTimeoutPeer);
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        return true;
+      };
+
+      // Finish tile j: add the partner's partial, online softmax, P into shared memory.
+      auto finish = [&](int j, const uint32_t (&own)[32]) -> bool {
+        const int slot = j & 1;
+        const uint32_t par = (j >> 1) & 1;
+        bool w = ptx::mbar_wait<true>(&xchg_full[slot], par, kErrTimeoutPeer);
+        if (!__all_sync(0xffffffffu, w)) return false;
         float x[64];
         {
           const uint8_t* mine = inbox + slot * L::kXchgSlot + h * 128;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const uint4 v = *reinterpret_cast<const uint4*>(mine + ((k ^ (h & 7)) << 4));
+            const uint4 v = *reinterpret_cast<const uint4*>(mine + ((k ^ sw) << 4));
             const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -360,15 +379,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
             }
           }
         }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_cluster(&xchg_free[slot], peer);   // my inbox slot is free again
         const int64_t key0 = j_begin + (int64_t)j * kTileN;
         const int n_valid = (int)min64(kTileN, j_end - key0);
-        float mx = -INFINITY;
+        if (n_valid < kTileN) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          if (i >= n_valid) x[i] = -INFINITY;
-          mx = fmaxf(mx, x[i]);
+          for (int i = 0; i < 64; ++i)
+            if (i >= n_valid) x[i] = -INFINITY;
+        }
+        float mx;
+        {
+          float m8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fmaxf(x[8 * i], x[8 * i + 1]), fmaxf(x[8 * i + 2], x[8 * i + 3]));
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], fmaxf(fmaxf(x[8 * i + 4], x[8 * i + 5]), fmaxf(x[8 * i + 6], x[8 * i + 7])));
+          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         }
         mx *= sl2;   // scale >= 0: the max of scaled scores is the scaled max
         if (j == 0) {
@@ -378,9 +403,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           // TMEM loads/stores are warp-wide: the warp rescales together, lanes
           // whose row max did not grow use factor 1.
           if (__any_sync(0xffffffffu, grow)) {
-            // O must not change under us: wait for the PV product of tile j-1
+            // O must not change under us: wait for the P V product of tile j-1
             w = ptx::mbar_wait(o_done, (j - 1) & 1, kErrTimeoutMma);
-            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, w)) return false;
             ptx::tc_fence_after();
             const float f = grow ? fast_exp2(m_ref - mx) : 1.f;
             l *= f;
@@ -393,20 +418,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
               for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
               ptx::tmem_st32(tmem + lane_base + kColO + c * 32, r);
             }
+            ptx::tmem_wait_st();
             if (grow) m_ref = mx;
           }
         }
-        uint32_t pk[32];
-        float psum = 0.f;
+        // P = 2^(s*scale*log2e - m_ref) as bf16, row h of the K-major P tile (128-byte swizzle)
+        uint8_t* prow = p_s + slot * L::kP + h * 128;
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float e0 = fast_exp2(fmaf(x[2 * i], sl2, -m_ref));
-          const float e1 = fast_exp2(fmaf(x[2 * i + 1], sl2, -m_ref));
-          pk[i] = ptx::pack_bf16x2(e0, e1);
-          psum += e0 + e1;
+        for (int k = 0; k < 8; ++k) {
+          uint32_t q4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float e0 = fast_exp2(fmaf(x[8 * k + 2 * e], sl2, -m_ref));
+            const float e1 = fast_exp2(fmaf(x[8 * k + 2 * e + 1], sl2, -m_ref));
+            ps[e] += e0 + e1;
+            q4[e] = ptx::pack_bf16x2(e0, e1);
+          }
+          *reinterpret_cast<uint4*>(prow + ((k ^ sw) << 4)) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
         }
-        l += psum;
-        ptx::tmem_st32(tmem + lane_base + kColS + slot * kTileN, pk);
+        l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         if (n_valid < kTileN) {
           // keys past the end get P = 0, but 0 * NaN is NaN: clear their latent rows
           uint8_t* st = smem + (j % kStages) * L::kStage;
@@ -416,11 +447,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
             *reinterpret_cast<uint4*>(st + bx * L::kKvBox + (n_valid + rem / 8) * 128 + (rem % 8) * 16) =
                 make_uint4(0, 0, 0, 0);
           }
-          ptx::fence_async_smem();
         }
-        ptx::tmem_wait_st();
+        ptx::fence_async_smem();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&p_ready[slot]);
+        // my inbox slot is consumed: the partner may send tile j+2 into it
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(&xchg_free[slot], peer);
+        return true;
+      };
+
+      uint32_t cur[32], nxt[32];
+      if (ok) ok = send(0, cur);
+      for (int j = 0; ok && j < nt; ++j) {
+        if (j + 1 < nt) {
+          ok = send(j + 1, nxt);
+          if (!ok) break;
+        }
+        ok = finish(j, cur);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) cur[i] = nxt[i];
       }
     }
 
@@ -485,31 +531,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   ptx::cluster_sync();   // the partner no longer writes into this CTA's shared memory
 }
 
-// Merge split partials: o = sum_s 2^{m_s - M} o_s / sum_s 2^{m_s - M} l_s.
-// One block of 128 threads per (row, head); thread i owns columns 4i..4i+3.
+// Merge split partials: o = sum_s 2^{m_s - M} o_s / sum_s 2^{m_s - M} l_s, M = max_s m_s.
+// One block of 128 threads per (row, head); warp 0 turns the (m, l) pairs into
+// weights, then thread i accumulates columns 4i..4i+3 over the splits with
+// several loads in flight.  Splits with no key (m = -inf) get weight 0 and
+// their (unwritten) partial is never used.
+constexpr int kMaxSplits = 256;
 __global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restrict__ part_o,
                                                            const float* __restrict__ part_ml, int num_splits,
                                                            int64_t n_q, int heads, __nv_bfloat16* __restrict__ o_lat) {
+  __shared__ float s_w[kMaxSplits];
+  __shared__ float s_inv;
   const int64_t row = blockIdx.x;
   const int head = blockIdx.y;
-  float M = -INFINITY;
-  for (int s = 0; s < num_splits; ++s) M = fmaxf(M, part_ml[(((int64_t)s * n_q + row) * heads + head) * 2]);
-  float L = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < num_splits; ++s) {
-    const int64_t slot = ((int64_t)s * n_q + row) * heads + head;
-    const float ms = part_ml[slot * 2];
-    if (ms == -INFINITY) continue;
-    const float wgt = exp2f(ms - M);
-    L += wgt * part_ml[slot * 2 + 1];
-    const float4 v = reinterpret_cast<const float4*>(part_o + slot * 512)[threadIdx.x];
-    acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+  const int64_t split_stride = n_q * heads;
+  const int64_t base = row * heads + head;
+  if (threadIdx.x < 32) {
+    float M = -INFINITY;
+    for (int s = threadIdx.x; s < num_splits; s += 32) M = fmaxf(M, part_ml[(s * split_stride + base) * 2]);
+    M = warp_max(M);
+    float L = 0.f;
+    for (int s = threadIdx.x; s < num_splits; s += 32) {
+      const float ms = part_ml[(s * split_stride + base) * 2];
+      const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
+      s_w[s] = w;
+      L += w * part_ml[(s * split_stride + base) * 2 + 1];
+    }
+    L = warp_sum(L);
+    if (threadIdx.x == 0) s_inv = L > 0.f ? 1.f / L : 0.f;
   }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
+  __syncthreads();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4* src = reinterpret_cast<const float4*>(part_o + base * 512) + threadIdx.x;
+  const int64_t step = split_stride * 512 / 4;
+#pragma unroll 8
+  for (int s = 0; s < num_splits; ++s) {
+    const float w = s_w[s];
+    const float4 v = src[s * step];
+    if (w != 0.f) {
+      acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+    }
+  }
+  const float inv = s_inv;
   uint2 o;
   o.x = ptx::pack_bf16x2(acc.x * inv, acc.y * inv);
   o.y = ptx::pack_bf16x2(acc.z * inv, acc.w * inv);
-  reinterpret_cast<uint2*>(o_lat + (row * heads + head) * 512)[threadIdx.x] = o;
+  reinterpret_cast<uint2*>(o_lat + base * 512)[threadIdx.x] = o;
 }
 
 }  // namespace sm100
