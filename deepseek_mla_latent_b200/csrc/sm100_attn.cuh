@@ -128,7 +128,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   uint64_t* q_full = bars + 21;         // q_abs half landed in the exchange area
   uint64_t* qpe_full = bars + 22;
   uint64_t* mma_idle = bars + 23;       // every MMA of this CTA finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
+  uint64_t* p_free = bars + 24;         // [2]  the P V product that read P buffer s finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
 
   const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id();
   const uint32_t rank = ptx::cluster_rank(), peer = rank ^ 1u;
@@ -166,6 +167,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       ptx::mbar_init(&xchg_full[s], 1);
       ptx::mbar_init(&xchg_free[s], 4);
       ptx::mbar_init(&outbox_ready[s], 128);
+      ptx::mbar_init(&p_free[s], 1);
     }
     ptx::mbar_init(o_done, 1);
     ptx::mbar_init(o_final, 1);
@@ -224,53 +226,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else if (warp == 5) {
     // ================================================= MMA issuer ========
-    // Order: QK(0), QK(1), PV(0), QK(2), PV(1), ...  QK(j) needs its tile and
-    // S buffer j&1 read out (tile j-2); PV(j) needs P(j).
+    // Two streams issued as their inputs arrive: QK(j) needs tile j and S
+    // buffer j&1 read out (tile j-2); PV(j) needs P(j).  QK runs ahead of PV,
+    // so the scores of the next tiles are ready while the softmax works.
     if (lane == 0 && nt > 0) {
       constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(128, kTileN, false, false);
       constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(128, 256, false, true);
       bool ok = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax) && ptx::mbar_wait(qpe_full, 0, kErrTimeoutTmaFull);
-      const uint32_t qpe_addr = ptx::smem_u32(qpe_s);
-      const uint32_t p_addr = ptx::smem_u32(p_s);
-      auto issue_pv = [&](int j) {
-        const uint32_t st = ptx::smem_u32(smem + (j % kStages) * L::kStage);
-        const uint32_t pa = p_addr + (j & 1) * L::kP;
-#pragma unroll
-        for (int ks = 0; ks < kTileN / 16; ++ks)
-          ptx::mma_ss(tmem + kColO, ptx::smem_desc(pa + ks * 32, 16, 1024, ptx::kSwizzle128),
-                      ptx::smem_desc(st + ks * 2048, L::kKvBox, 1024, ptx::kSwizzle128), idesc_pv,
-                      (j > 0 || ks > 0) ? 1u : 0u);
-        ptx::mma_commit(&kv_empty[j % kStages]);
-        ptx::mma_commit(o_done);
-      };
+      // descriptor bases; the start address sits in the low bits, so offsets add directly (>> 4)
+      const uint64_t d_stage0 = ptx::smem_desc(ptx::smem_u32(smem), 16, 1024, ptx::kSwizzle128);
+      const uint64_t d_pe0 = ptx::smem_desc(ptx::smem_u32(smem + L::kKv), 16, 512, ptx::kSwizzle64);
+      const uint64_t d_qpe = ptx::smem_desc(ptx::smem_u32(qpe_s), 16, 512, ptx::kSwizzle64);
+      const uint64_t d_p0 = ptx::smem_desc(ptx::smem_u32(p_s), 16, 1024, ptx::kSwizzle128);
+      const uint64_t d_v0 = ptx::smem_desc(ptx::smem_u32(smem), L::kKvBox, 1024, ptx::kSwizzle128);
+      int qk = 0, pv = 0;
+      uint64_t t_last = global_timer_ns();
       ptx::tc_fence_after();
-      for (int j = 0; ok && j < nt; ++j) {
-        const int s = j % kStages;
-        if (!ptx::mbar_wait(&kv_full[s], (j / kStages) & 1, kErrTimeoutTmaFull)) { ok = false; break; }
-        if (j >= 2 && !ptx::mbar_wait(&s_free[j & 1], ((j - 2) >> 1) & 1, kErrTimeoutSoftmax)) { ok = false; break; }
-        ptx::tc_fence_after();
-        const uint32_t st = ptx::smem_u32(smem + s * L::kStage);
-        const uint32_t scol = tmem + kColS + (j & 1) * kTileN;
-#pragma unroll
-        for (int ks = 0; ks < 16; ++ks)
-          ptx::mma_ts(scol, tmem + kColQ + ks * 8,
-                      ptx::smem_desc(st + (ks >> 2) * L::kKvBox + (ks & 3) * 32, 16, 1024, ptx::kSwizzle128),
-                      idesc_qk, ks > 0 ? 1u : 0u);
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-          ptx::mma_ss(scol, ptx::smem_desc(qpe_addr + ks * 32, 16, 512, ptx::kSwizzle64),
-                      ptx::smem_desc(st + L::kKv + ks * 32, 16, 512, ptx::kSwizzle64), idesc_qk, 1u);
-        ptx::mma_commit(&s_full[j & 1]);
-        if (j > 0) {
-          if (!ptx::mbar_wait(&p_ready[(j - 1) & 1], ((j - 1) >> 1) & 1, kErrTimeoutSoftmax)) { ok = false; break; }
+      while (ok && pv < nt) {
+        bool progressed = false;
+        if (qk < nt && (qk < 2 || ptx::mbar_test(&s_free[qk & 1], ((qk - 2) >> 1) & 1)) &&
+            ptx::mbar_test(&kv_full[qk % kStages], (qk / kStages) & 1)) {
           ptx::tc_fence_after();
-          issue_pv(j - 1);
+          const uint32_t so = (uint32_t)((qk % kStages) * L::kStage) >> 4;
+          const uint32_t scol = tmem + kColS + (qk & 1) * kTileN;
+#pragma unroll
+          for (int ks = 0; ks < 16; ++ks)
+            ptx::mma_ts(scol, tmem + kColQ + ks * 8, d_stage0 + so + (((ks >> 2) * L::kKvBox + (ks & 3) * 32) >> 4),
+                        idesc_qk, ks > 0 ? 1u : 0u);
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks)
+            ptx::mma_ss(scol, d_qpe + ((ks * 32) >> 4), d_pe0 + so + ((ks * 32) >> 4), idesc_qk, 1u);
+          ptx::mma_commit(&s_full[qk & 1]);
+          ++qk;
+          progressed = true;
         }
-      }
-      if (ok && ptx::mbar_wait(&p_ready[(nt - 1) & 1], ((nt - 1) >> 1) & 1, kErrTimeoutSoftmax)) {
-        ptx::tc_fence_after();
-        issue_pv(nt - 1);
-        ptx::mma_commit(o_final);
+        if (pv < qk && ptx::mbar_test(&p_ready[pv & 1], (pv >> 1) & 1)) {
+          ptx::tc_fence_after();
+          const uint32_t so = (uint32_t)((pv % kStages) * L::kStage) >> 4;
+          const uint32_t po = (uint32_t)((pv & 1) * L::kP) >> 4;
+#pragma unroll
+          for (int ks = 0; ks < kTileN / 16; ++ks)
+            ptx::mma_ss(tmem + kColO, d_p0 + po + ((ks * 32) >> 4), d_v0 + so + ((ks * 2048) >> 4), idesc_pv,
+                        (pv > 0 || ks > 0) ? 1u : 0u);
+          ptx::mma_commit(&kv_empty[pv % kStages]);
+          ptx::mma_commit(&p_free[pv & 1]);
+          ptx::mma_commit(o_done);
+          if (pv == nt - 1) ptx::mma_commit(o_final);
+          ++pv;
+          progressed = true;
+        }
+        if (progressed) {
+          t_last = global_timer_ns();
+        } else {
+          __nanosleep(20);
+          if (global_timer_ns() - t_last > kWaitLimitNs) {
+            raise_error(qk < nt ? kErrTimeoutTmaFull : kErrTimeoutSoftmax);
+            ok = false;
+          }
+        }
       }
       // nothing of ours may still be running in the tensor core when TMEM is freed
       ptx::mma_commit(mma_idle);
@@ -363,7 +376,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         const uint32_t par = (j >> 1) & 1;
         bool w = ptx::mbar_wait<true>(&xchg_full[slot], par, kErrTimeoutPeer);
         if (!__all_sync(0xffffffffu, w)) return false;
-        float x[64];
+        // raw scores: my fp16 partial + the partner's fp16 partial (packed fp16 adds)
+        uint32_t sum2[32];
         {
           const uint8_t* mine = inbox + slot * L::kXchgSlot + h * 128;
 #pragma unroll
@@ -372,10 +386,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
             const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 a = f16x2_to_f2(own[4 * k + e]);
-              const float2 c = f16x2_to_f2(pv[e]);
-              x[8 * k + 2 * e] = a.x + c.x;
-              x[8 * k + 2 * e + 1] = a.y + c.y;
+              __half2 a = *reinterpret_cast<const __half2*>(&own[4 * k + e]);
+              __half2 c = *reinterpret_cast<const __half2*>(&pv[e]);
+              __half2 r = __hadd2(a, c);
+              sum2[4 * k + e] = *reinterpret_cast<uint32_t*>(&r);
             }
           }
         }
@@ -383,19 +397,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         const int n_valid = (int)min64(kTileN, j_end - key0);
         if (n_valid < kTileN) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (i >= n_valid) x[i] = -INFINITY;
+          for (int i = 0; i < 32; ++i) {
+            // keys past the end: -inf (fp16 0xFC00) in the masked half(s)
+            if (2 * i >= n_valid) sum2[i] = 0xFC00FC00u;
+            else if (2 * i + 1 >= n_valid) sum2[i] = (sum2[i] & 0x0000FFFFu) | 0xFC000000u;
+          }
         }
         float mx;
         {
-          float m8[8];
+          __half2 m8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fmaxf(x[8 * i], x[8 * i + 1]), fmaxf(x[8 * i + 2], x[8 * i + 3]));
-#pragma unroll
-          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], fmaxf(fmaxf(x[8 * i + 4], x[8 * i + 5]), fmaxf(x[8 * i + 6], x[8 * i + 7])));
-          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          for (int i = 0; i < 8; ++i) {
+            const __half2* v = reinterpret_cast<const __half2*>(&sum2[4 * i]);
+            m8[i] = __hmax2(__hmax2(v[0], v[1]), __hmax2(v[2], v[3]));
+          }
+          const __half2 m2 = __hmax2(__hmax2(__hmax2(m8[0], m8[1]), __hmax2(m8[2], m8[3])),
+                                     __hmax2(__hmax2(m8[4], m8[5]), __hmax2(m8[6], m8[7])));
+          mx = fmaxf(__low2float(m2), __high2float(m2));
         }
         mx *= sl2;   // scale >= 0: the max of scaled scores is the scaled max
+        // P buffer `slot` and O are only touched once the P V product of tile j-2 is done
+        if (j >= 2) {
+          w = ptx::mbar_wait(&p_free[slot], ((j - 2) >> 1) & 1, kErrTimeoutMma);
+          if (!__all_sync(0xffffffffu, w)) return false;
+        }
         if (j == 0) {
           m_ref = mx;
         } else {
@@ -430,8 +455,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           uint32_t q4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float e0 = fast_exp2(fmaf(x[8 * k + 2 * e], sl2, -m_ref));
-            const float e1 = fast_exp2(fmaf(x[8 * k + 2 * e + 1], sl2, -m_ref));
+            const float2 xs = __half22float2(*reinterpret_cast<const __half2*>(&sum2[4 * k + e]));
+            float e0 = fast_exp2(fmaf(xs.x, sl2, -m_ref));
+            float e1 = fast_exp2(fmaf(xs.y, sl2, -m_ref));
+            if (n_valid < kTileN) {   // keys past the end weigh exactly 0 (also when scale is 0)
+              if (8 * k + 2 * e >= n_valid) e0 = 0.f;
+              if (8 * k + 2 * e + 1 >= n_valid) e1 = 0.f;
+            }
             ps[e] += e0 + e1;
             q4[e] = ptx::pack_bf16x2(e0, e1);
           }
