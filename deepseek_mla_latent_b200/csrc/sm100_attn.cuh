@@ -190,8 +190,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
 
   if (warp == 4) {
     // ================================================= TMA producer ======
+    // The whole warp runs the loop (waits are warp-wide); one elected lane issues.
     int issued = 0;
-    if (lane == 0) {
+    if (ptx::elect_one()) {
       ptx::prefetch_tmap(&tmap_kv);
       ptx::prefetch_tmap(&tmap_pe);
       if (nt > 0) {
@@ -203,9 +204,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         ptx::mbar_arrive_expect_tx(qpe_full, L::kQpe);
         ptx::tma_load_3d(qpe_s, &tmap_qpe, qpe_full, 128 + 32 * (int)rank, head0, (int)row);
       }
-      for (int j = 0; j < nt; ++j) {
-        const int s = j % kStages;
-        if (!ptx::mbar_wait(&kv_empty[s], ((j / kStages) & 1) ^ 1, kErrTimeoutStageFree)) break;
+    }
+    __syncwarp();
+    for (int j = 0; j < nt; ++j) {
+      const int s = j % kStages;
+      const bool w = ptx::mbar_wait(&kv_empty[s], ((j / kStages) & 1) ^ 1, kErrTimeoutStageFree);
+      if (!__all_sync(0xffffffffu, w)) break;
+      if (ptx::elect_one()) {
         uint8_t* st = smem + s * L::kStage;
         ptx::mbar_arrive_expect_tx(&kv_full[s], L::kStage);
         const int key = (int)(k0 + j_begin + (int64_t)j * kTileN);
@@ -213,15 +218,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         for (int bx = 0; bx < 4; ++bx)
           ptx::tma_load_2d(st + bx * L::kKvBox, &tmap_kv, &kv_full[s], 256 * (int)rank + 64 * bx, key);
         ptx::tma_load_2d(st + L::kKv, &tmap_pe, &kv_full[s], 32 * (int)rank, key);
-        issued = j + 1;
       }
-      // exit path: every copy this CTA started has landed before its smem goes away
-      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-        ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, kErrTimeoutDrain);
-      if (nt > 0) {
-        ptx::mbar_wait(qpe_full, 0, kErrTimeoutDrain);
-        ptx::mbar_wait(q_full, 0, kErrTimeoutDrain);
-      }
+      __syncwarp();
+      issued = j + 1;
+    }
+    // exit path: every copy this CTA started has landed before its smem goes away
+    for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+      ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, kErrTimeoutDrain);
+    if (nt > 0) {
+      ptx::mbar_wait(qpe_full, 0, kErrTimeoutDrain);
+      ptx::mbar_wait(q_full, 0, kErrTimeoutDrain);
     }
     __syncwarp();
   } else if (warp == 5) {
@@ -229,10 +235,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     // Two streams issued as their inputs arrive: QK(j) needs tile j and S
     // buffer j&1 read out (tile j-2); PV(j) needs P(j).  QK runs ahead of PV,
     // so the scores of the next tiles are ready while the softmax works.
-    if (lane == 0 && nt > 0) {
+    // The whole warp runs the loop with warp-uniform decisions; one elected
+    // lane issues each MMA and commit.
+    if (nt > 0) {
       constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(128, kTileN, false, false);
       constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(128, 256, false, true);
       bool ok = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax) && ptx::mbar_wait(qpe_full, 0, kErrTimeoutTmaFull);
+      ok = __all_sync(0xffffffffu, ok);
       // descriptor bases; the start address sits in the low bits, so offsets add directly (>> 4)
       const uint64_t d_stage0 = ptx::smem_desc(ptx::smem_u32(smem), 16, 1024, ptx::kSwizzle128);
       const uint64_t d_pe0 = ptx::smem_desc(ptx::smem_u32(smem + L::kKv), 16, 512, ptx::kSwizzle64);
@@ -244,34 +253,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       ptx::tc_fence_after();
       while (ok && pv < nt) {
         bool progressed = false;
-        if (qk < nt && (qk < 2 || ptx::mbar_test(&s_free[qk & 1], ((qk - 2) >> 1) & 1)) &&
-            ptx::mbar_test(&kv_full[qk % kStages], (qk / kStages) & 1)) {
+        bool go = qk < nt && (qk < 2 || ptx::mbar_test(&s_free[qk & 1], ((qk - 2) >> 1) & 1)) &&
+                  ptx::mbar_test(&kv_full[qk % kStages], (qk / kStages) & 1);
+        if (__shfl_sync(0xffffffffu, go, 0)) {
           ptx::tc_fence_after();
           const uint32_t so = (uint32_t)((qk % kStages) * L::kStage) >> 4;
           const uint32_t scol = tmem + kColS + (qk & 1) * kTileN;
 #pragma unroll
-          for (int ks = 0; ks < 16; ++ks)
-            ptx::mma_ts(scol, tmem + kColQ + ks * 8, d_stage0 + so + (((ks >> 2) * L::kKvBox + (ks & 3) * 32) >> 4),
-                        idesc_qk, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < 16; ++ks) {
+            if (ptx::elect_one())
+              ptx::mma_ts(scol, tmem + kColQ + ks * 8,
+                          d_stage0 + so + (((ks >> 2) * L::kKvBox + (ks & 3) * 32) >> 4), idesc_qk,
+                          ks > 0 ? 1u : 0u);
+            __syncwarp();
+          }
 #pragma unroll
-          for (int ks = 0; ks < 2; ++ks)
-            ptx::mma_ss(scol, d_qpe + ((ks * 32) >> 4), d_pe0 + so + ((ks * 32) >> 4), idesc_qk, 1u);
-          ptx::mma_commit(&s_full[qk & 1]);
+          for (int ks = 0; ks < 2; ++ks) {
+            if (ptx::elect_one()) ptx::mma_ss(scol, d_qpe + ((ks * 32) >> 4), d_pe0 + so + ((ks * 32) >> 4), idesc_qk, 1u);
+            __syncwarp();
+          }
+          if (ptx::elect_one()) ptx::mma_commit(&s_full[qk & 1]);
+          __syncwarp();
           ++qk;
           progressed = true;
         }
-        if (pv < qk && ptx::mbar_test(&p_ready[pv & 1], (pv >> 1) & 1)) {
+        go = pv < qk && ptx::mbar_test(&p_ready[pv & 1], (pv >> 1) & 1);
+        if (__shfl_sync(0xffffffffu, go, 0)) {
           ptx::tc_fence_after();
           const uint32_t so = (uint32_t)((pv % kStages) * L::kStage) >> 4;
           const uint32_t po = (uint32_t)((pv & 1) * L::kP) >> 4;
 #pragma unroll
-          for (int ks = 0; ks < kTileN / 16; ++ks)
-            ptx::mma_ss(tmem + kColO, d_p0 + po + ((ks * 32) >> 4), d_v0 + so + ((ks * 2048) >> 4), idesc_pv,
-                        (pv > 0 || ks > 0) ? 1u : 0u);
-          ptx::mma_commit(&kv_empty[pv % kStages]);
-          ptx::mma_commit(&p_free[pv & 1]);
-          ptx::mma_commit(o_done);
-          if (pv == nt - 1) ptx::mma_commit(o_final);
+          for (int ks = 0; ks < kTileN / 16; ++ks) {
+            if (ptx::elect_one())
+              ptx::mma_ss(tmem + kColO, d_p0 + po + ((ks * 32) >> 4), d_v0 + so + ((ks * 2048) >> 4), idesc_pv,
+                          (pv > 0 || ks > 0) ? 1u : 0u);
+            __syncwarp();
+          }
+          if (ptx::elect_one()) {
+            ptx::mma_commit(&kv_empty[pv % kStages]);
+            ptx::mma_commit(&p_free[pv & 1]);
+            ptx::mma_commit(o_done);
+            if (pv == nt - 1) ptx::mma_commit(o_final);
+          }
+          __syncwarp();
           ++pv;
           progressed = true;
         }
@@ -279,14 +303,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           t_last = global_timer_ns();
         } else {
           __nanosleep(20);
-          if (global_timer_ns() - t_last > kWaitLimitNs) {
-            raise_error(qk < nt ? kErrTimeoutTmaFull : kErrTimeoutSoftmax);
+          bool late = global_timer_ns() - t_last > kWaitLimitNs;
+          if (__shfl_sync(0xffffffffu, late, 0)) {
+            if (lane == 0) raise_error(qk < nt ? kErrTimeoutTmaFull : kErrTimeoutSoftmax);
             ok = false;
           }
         }
       }
       // nothing of ours may still be running in the tensor core when TMEM is freed
-      ptx::mma_commit(mma_idle);
+      if (ptx::elect_one()) ptx::mma_commit(mma_idle);
+      __syncwarp();
       ptx::mbar_wait(mma_idle, 0, kErrTimeoutDrain);
     }
     __syncwarp();
@@ -320,8 +346,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         // the exchange area is free again: tell the partner it may send into my inbox
         __syncwarp();
         if (lane == 0) {
-          ptx::mbar_arrive_cluster(&xchg_free[0], peer);
-          ptx::mbar_arrive_cluster(&xchg_free[1], peer);
+          ptx::mbar_arrive_cluster_relaxed(&xchg_free[0], peer);
+          ptx::mbar_arrive_cluster_relaxed(&xchg_free[1], peer);
         }
       }
 
@@ -483,7 +509,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         ptx::mbar_arrive(&p_ready[slot]);
         // my inbox slot is consumed: the partner may send tile j+2 into it
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_cluster(&xchg_free[slot], peer);
+        if (lane == 0) ptx::mbar_arrive_cluster_relaxed(&xchg_free[slot], peer);
         return true;
       };
 

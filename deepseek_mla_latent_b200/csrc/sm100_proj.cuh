@@ -10,10 +10,11 @@
 // sizes (n = batch) the weight read is the whole cost, so M on the weight
 // keeps each weight byte read once per call whatever the batch.
 //
-// One CTA per (M tile, head, N tile), four warps: warp 0 lane 0 feeds a
-// STAGES-deep ring of 64-wide K chunks with TMA, warp 1 lane 0 issues the
-// MMAs into a TMEM accumulator (128 lanes x N columns fp32), then all four
-// warps drain TMEM (warp w owns lanes 32w..32w+31) and store bf16.
+// One CTA per (M tile, head, N tile), four warps: warp 0 feeds a
+// STAGES-deep ring of 64-wide K chunks with TMA, warp 1 issues the MMAs into
+// a TMEM accumulator (128 lanes x N columns fp32) -- both loop with the whole
+// warp and issue from one elected lane -- then all four warps drain TMEM
+// (warp w owns lanes 32w..32w+31) and store bf16.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -69,31 +70,38 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(
   ptx::tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
 
-  int issued = 0;  // chunks whose TMA the producer started (thread 0 only)
-  if (warp == 0 && lane == 0) {
+  int issued = 0;  // chunks whose TMA the producer started
+  if (warp == 0) {
+    // producer: the whole warp loops, one elected lane issues
     for (int i = 0; i < k_chunks; ++i) {
       const int s = i % STAGES;
-      if (!ptx::mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, kErrTimeoutStageFree)) break;
-      uint8_t* a = smem + s * L::kStage;
-      uint8_t* b = a + L::kA;
-      ptx::mbar_arrive_expect_tx(&full[s], L::kA + N_TILE * kProjBoxK * 2);
-      if (A_MN) {
-        // two 64(c) x 64(d) boxes: M elements 0..63 and 64..127 of this tile
-        const int c0 = m_tile * 128, row = w_row_base + h * w_rows_per_head + i * kProjBoxK;
-        ptx::tma_load_2d(a, &tmap_w, &full[s], c0, row);
-        ptx::tma_load_2d(a + L::kA / 2, &tmap_w, &full[s], c0 + 64, row);
-      } else {
-        // one 64(c) x 128(d) box: K elements i*64.., all 128 M rows
-        ptx::tma_load_2d(a, &tmap_w, &full[s], i * kProjBoxK, w_row_base + h * w_rows_per_head);
+      const bool w = ptx::mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, kErrTimeoutStageFree);
+      if (!__all_sync(0xffffffffu, w)) break;
+      if (ptx::elect_one()) {
+        uint8_t* a = smem + s * L::kStage;
+        uint8_t* b = a + L::kA;
+        ptx::mbar_arrive_expect_tx(&full[s], L::kA + N_TILE * kProjBoxK * 2);
+        if (A_MN) {
+          // two 64(c) x 64(d) boxes: M elements 0..63 and 64..127 of this tile
+          const int c0 = m_tile * 128, row = w_row_base + h * w_rows_per_head + i * kProjBoxK;
+          ptx::tma_load_2d(a, &tmap_w, &full[s], c0, row);
+          ptx::tma_load_2d(a + L::kA / 2, &tmap_w, &full[s], c0 + 64, row);
+        } else {
+          // one 64(c) x 128(d) box: K elements i*64.., all 128 M rows
+          ptx::tma_load_2d(a, &tmap_w, &full[s], i * kProjBoxK, w_row_base + h * w_rows_per_head);
+        }
+        ptx::tma_load_3d(b, &tmap_x, &full[s], i * kProjBoxK, h, n_tile * N_TILE);
       }
-      ptx::tma_load_3d(b, &tmap_x, &full[s], i * kProjBoxK, h, n_tile * N_TILE);
+      __syncwarp();
       issued = i + 1;
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
+    // MMA issuer: the whole warp loops, one elected lane issues
     constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, N_TILE, A_MN, false);
     for (int i = 0; i < k_chunks; ++i) {
       const int s = i % STAGES;
-      if (!ptx::mbar_wait(&full[s], (i / STAGES) & 1, kErrTimeoutTmaFull)) break;
+      const bool w = ptx::mbar_wait(&full[s], (i / STAGES) & 1, kErrTimeoutTmaFull);
+      if (!__all_sync(0xffffffffu, w)) break;
       ptx::tc_fence_after();
       const uint32_t a = ptx::smem_u32(smem + s * L::kStage);
       const uint32_t b = a + L::kA;
@@ -102,13 +110,15 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(
         const uint64_t da = A_MN ? ptx::smem_desc(a + ks * 2048, L::kA / 2, 1024, ptx::kSwizzle128)
                                  : ptx::smem_desc(a + ks * 32, 16, 1024, ptx::kSwizzle128);
         const uint64_t db = ptx::smem_desc(b + ks * 32, 16, 1024, ptx::kSwizzle128);
-        ptx::mma_ss(tmem_d, da, db, idesc, (i > 0 || ks > 0) ? 1u : 0u);
+        if (ptx::elect_one()) ptx::mma_ss(tmem_d, da, db, idesc, (i > 0 || ks > 0) ? 1u : 0u);
+        __syncwarp();
       }
-      ptx::mma_commit(&empty[s]);
+      if (ptx::elect_one()) ptx::mma_commit(&empty[s]);
+      __syncwarp();
     }
-    ptx::mma_commit(done);
+    if (ptx::elect_one()) ptx::mma_commit(done);
+    __syncwarp();
   }
-  __syncwarp();
 
   // Epilogue: TMEM -> registers -> bf16 -> global.
   const bool ok = ptx::mbar_wait(done, 0, kErrTimeoutMma);
@@ -131,7 +141,7 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(
     }
   }
   // Exit path: let every TMA this CTA started land before the CTA's shared memory is released.
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
       ptx::mbar_wait(&full[i % STAGES], (i / STAGES) & 1, kErrTimeoutDrain);
   }
