@@ -58,6 +58,17 @@ def dist_env():
     return rank, world, local
 
 
+def reduce_max(values, device):
+    """Element-wise max of per-rank float values over all ranks (identity with one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -273,12 +284,7 @@ def main():
 
     step_ms = [s.elapsed_time(e) for s, e in zip(ev_s, ev_e)]
     attn_ms = [s.elapsed_time(e) for s, e in zip(ev_as, ev_ae)]
-    total_ms = sum(step_ms)
-    mean_attn_ms = sum(attn_ms) / len(attn_ms)
-    if world > 1:
-        t = torch.tensor([total_ms, mean_attn_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, mean_attn_ms = float(t[0]), float(t[1])
+    total_ms, mean_attn_ms = reduce_max([sum(step_ms), sum(attn_ms) / len(attn_ms)], dev)
     us_step = total_ms / args.steps * 1e3
 
     # End to end through the same public calls: pinned host q -> device, step, out -> pinned host.
@@ -299,11 +305,7 @@ def main():
         out_pinned.copy_(out, non_blocking=True)
         e2e_e[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms, = reduce_max([sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))], dev)
     e2e_us = e2e_ms / e2e_steps * 1e3
     del q_host
 
