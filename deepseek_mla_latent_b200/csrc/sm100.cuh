@@ -54,6 +54,25 @@ inline bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
 
 inline mla_status_t last_launch() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
+// Launch with programmatic stream serialization (pdl = true): the kernel may
+// start its set-up while the previous kernel in the stream finishes; every
+// kernel here waits (griddepcontrol.wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+inline mla_status_t launch(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 template <typename K>
 inline bool set_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
@@ -63,13 +82,12 @@ inline bool set_smem(K kernel, size_t bytes) {
 template <bool A_MN, int N_TILE, int STAGES>
 inline mla_status_t launch_proj(const CUtensorMap& tw, const CUtensorMap& tx, dim3 grid, int k_chunks, int w_row_base,
                                 int n_rows, void* out, int64_t out_row_stride, int out_head_stride,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, bool pdl) {
   constexpr size_t smem = proj_smem_bytes<N_TILE, STAGES>();
   auto kern = proj_kernel<A_MN, N_TILE, STAGES>;
   if (!set_smem(kern, smem)) return MLA_ERR_CUDA;
-  kern<<<grid, kProjThreads, smem, stream>>>(tw, tx, k_chunks, w_row_base, 256, n_rows,
-                                             static_cast<__nv_bfloat16*>(out), out_row_stride, out_head_stride);
-  return last_launch();
+  return launch(pdl, kern, grid, dim3(kProjThreads), smem, stream, tw, tx, k_chunks, w_row_base, 256, n_rows,
+                static_cast<__nv_bfloat16*>(out), out_row_stride, out_head_stride);
 }
 
 // STAGES: the K ring depth; with few query rows the whole weight tile of a
@@ -77,13 +95,13 @@ inline mla_status_t launch_proj(const CUtensorMap& tw, const CUtensorMap& tx, di
 template <bool A_MN, int MAX_STAGES>
 inline mla_status_t dispatch_proj(const CUtensorMap& tw, const CUtensorMap& tx, int m_tiles, int H, int64_t n_rows,
                                   int k_chunks, int w_row_base, void* out, int64_t out_row_stride,
-                                  int out_head_stride, cudaStream_t stream) {
+                                  int out_head_stride, cudaStream_t stream, bool pdl) {
   auto go = [&](auto tile) {
     constexpr int NT = decltype(tile)::value;
     constexpr int STAGES = NT <= 64 ? MAX_STAGES : (MAX_STAGES < 4 ? MAX_STAGES : 4);
     dim3 grid(m_tiles, H, (unsigned)((n_rows + NT - 1) / NT));
     return launch_proj<A_MN, NT, STAGES>(tw, tx, grid, k_chunks, w_row_base, (int)n_rows, out, out_row_stride,
-                                         out_head_stride, stream);
+                                         out_head_stride, stream, pdl);
   };
   if (n_rows <= 16) return go(std::integral_constant<int, 16>{});
   if (n_rows <= 32) return go(std::integral_constant<int, 32>{});
@@ -103,7 +121,8 @@ inline mla_status_t absorb_q(const void* q, int64_t q_row_stride, const void* wk
   uint32_t box[3] = {xb[0], xb[1], (uint32_t)(n_rows <= 16 ? 16 : n_rows <= 32 ? 32 : n_rows <= 64 ? 64 : n_rows <= 128 ? 128 : 256)};
   if (!make_map(&tw, wkv_b, 2, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   if (!make_map(&tx, q, 3, xd, xs, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-  return dispatch_proj<true, 2>(tw, tx, 4, H, n_rows, 2, 0, q_abs, (int64_t)H * 512, 512, stream);
+  // the first kernel of a step: an ordinary launch, so the step starts after all earlier work
+  return dispatch_proj<true, 2>(tw, tx, 4, H, n_rows, 2, 0, q_abs, (int64_t)H * 512, 512, stream, false);
 }
 
 inline mla_status_t out_proj(const void* o_lat, const void* wkv_b, void* out, int64_t n_rows, int H,
@@ -116,7 +135,7 @@ inline mla_status_t out_proj(const void* o_lat, const void* wkv_b, void* out, in
   uint32_t box[3] = {64, 1, (uint32_t)(n_rows <= 16 ? 16 : n_rows <= 32 ? 32 : n_rows <= 64 ? 64 : n_rows <= 128 ? 128 : 256)};
   if (!make_map(&tw, wkv_b, 2, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   if (!make_map(&tx, o_lat, 3, xd, xs, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-  return dispatch_proj<false, 8>(tw, tx, 1, H, n_rows, 8, 128, out, (int64_t)H * 128, 128, stream);
+  return dispatch_proj<false, 8>(tw, tx, 1, H, n_rows, 8, 128, out, (int64_t)H * 128, 128, stream, true);
 }
 
 // ----------------------------------------------------------------- attention
@@ -188,14 +207,11 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
     p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)splits * n_q * H * 512 * 4));
   }
   if (!set_smem(latent_attn_kernel, AttnLayout::kAlloc)) return MLA_ERR_CUDA;
-  latent_attn_kernel<<<(unsigned)(2 * units), kAttnThreads, AttnLayout::kAlloc, stream>>>(tkv, tpe, tqpe, tqa, p);
-  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-  if (splits > 1) {
-    merge_splits_kernel<<<dim3((unsigned)n_q, H), 128, 0, stream>>>(p.part_o, p.part_ml, splits, n_q, H,
-                                                                    static_cast<__nv_bfloat16*>(o_lat));
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-  }
-  return MLA_OK;
+  mla_status_t st = launch(true, latent_attn_kernel, dim3((unsigned)(2 * units)), dim3(kAttnThreads),
+                           AttnLayout::kAlloc, stream, tkv, tpe, tqpe, tqa, p);
+  if (st != MLA_OK || splits <= 1) return st;
+  return launch(true, merge_splits_kernel, dim3((unsigned)n_q, H), dim3(128), 0, stream,
+                (const float*)p.part_o, (const float*)p.part_ml, splits, n_q, H, static_cast<__nv_bfloat16*>(o_lat));
 }
 
 }  // namespace sm100

@@ -145,27 +145,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id();
   const uint32_t rank = ptx::cluster_rank(), peer = rank ^ 1u;
 
-  // ---- work unit: (query row, head group, split) -------------------------
-  const int64_t unit = blockIdx.x >> 1;
-  const int per_row = p.head_groups * p.num_splits;
-  const int64_t row = unit / per_row;
-  const int hg = (int)((unit % per_row) / p.num_splits);
-  const int sp = (int)(unit % p.num_splits);
-  const int b = p.cu_q ? find_sequence(p.cu_q, p.batch, row) : (int)row;
-  const int64_t k0 = min64(max64(0, __ldg(p.cu_k + b)), p.kv_rows);
-  const int64_t t = max64(0, min64((int64_t)__ldg(p.cu_k + b + 1), p.kv_rows) - k0);
-  int64_t visible = t;
-  if (p.cu_q) {
-    const int64_t q0 = __ldg(p.cu_q + b);
-    const int64_t s = max64(0, (int64_t)__ldg(p.cu_q + b + 1) - q0);
-    visible = min64(t, max64(0, t - s + (row - q0) + 1));
-  }
-  const int64_t per = ((visible + p.num_splits - 1) / p.num_splits + kTileN - 1) / kTileN * kTileN;
-  const int64_t j_begin = min64(visible, (int64_t)sp * per);
-  const int64_t j_end = min64(visible, j_begin + per);
-  const int nt = (int)((j_end - j_begin + kTileN - 1) / kTileN);
-  const int head0 = hg * 128;
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(&kv_full[s], 1);
@@ -199,6 +178,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   ptx::tc_fence_after();
   ptx::cluster_sync();   // the partner's barriers exist before anything remote touches them
   const uint32_t tmem = *tmem_slot;
+  // set-up above touches no global memory; inputs may come from the previous kernel
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+
+  // ---- work unit: (query row, head group, split) -------------------------
+  const int64_t unit = blockIdx.x >> 1;
+  const int per_row = p.head_groups * p.num_splits;
+  const int64_t row = unit / per_row;
+  const int hg = (int)((unit % per_row) / p.num_splits);
+  const int sp = (int)(unit % p.num_splits);
+  const int b = p.cu_q ? find_sequence(p.cu_q, p.batch, row) : (int)row;
+  const int64_t k0 = min64(max64(0, __ldg(p.cu_k + b)), p.kv_rows);
+  const int64_t t = max64(0, min64((int64_t)__ldg(p.cu_k + b + 1), p.kv_rows) - k0);
+  int64_t visible = t;
+  if (p.cu_q) {
+    const int64_t q0 = __ldg(p.cu_q + b);
+    const int64_t s = max64(0, (int64_t)__ldg(p.cu_q + b + 1) - q0);
+    visible = min64(t, max64(0, t - s + (row - q0) + 1));
+  }
+  const int64_t per = ((visible + p.num_splits - 1) / p.num_splits + kTileN - 1) / kTileN * kTileN;
+  const int64_t j_begin = min64(visible, (int64_t)sp * per);
+  const int64_t j_end = min64(visible, j_begin + per);
+  const int nt = (int)((j_end - j_begin + kTileN - 1) / kTileN);
+  const int head0 = hg * 128;
+
+
   constexpr uint32_t kColO = 0, kColQ = 256, kColS = 384;
 
   if (warp == kProducerWarp) {
@@ -631,6 +636,8 @@ __global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restri
                                                            int64_t n_q, int heads, __nv_bfloat16* __restrict__ o_lat) {
   __shared__ float s_w[kMaxSplits];
   __shared__ float s_inv;
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   const int64_t row = blockIdx.x;
   const int head = blockIdx.y;
   const int64_t split_stride = n_q * heads;

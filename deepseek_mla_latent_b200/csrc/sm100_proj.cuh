@@ -69,6 +69,9 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  // set-up above touches no global memory; inputs may come from the previous kernel
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   int issued = 0;  // chunks whose TMA the producer started
   if (warp == 0) {

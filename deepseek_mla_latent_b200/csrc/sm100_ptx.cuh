@@ -34,6 +34,14 @@ __device__ __forceinline__ bool elect_one() {
 }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 
+// ------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while its
+// predecessor in the stream is still running: it must wait here before its
+// first global memory access.  launch_dependents lets the successor start its
+// own set-up early (the successor still waits for this grid to finish).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier --
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
