@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "mla.h"
@@ -73,9 +75,23 @@ inline mla_status_t launch(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 b
   return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device); the
+// call is host-side only, so it is also safe while a stream is being captured.
+inline bool set_smem_once(const void* kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& d : done)
+    if (d.first == kernel && d.second == dev) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) return false;
+  done.emplace_back(kernel, dev);
+  return true;
+}
 template <typename K>
 inline bool set_smem(K kernel, size_t bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+  return set_smem_once(reinterpret_cast<const void*>(kernel), bytes);
 }
 
 // --------------------------------------------------------------- projections
