@@ -40,16 +40,17 @@ inline EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map: dims/strides innermost first, strides in bytes (rank-1 of them).
+// Tensor map (bf16 unless `dt` says otherwise): dims/strides innermost first, strides in bytes (rank-1 of them).
 inline bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-                     const uint32_t* box, CUtensorMapSwizzle swz) {
+                     const uint32_t* box, CUtensorMapSwizzle swz,
+                     CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t d[3], s[2];
   cuuint32_t b[3], e[3] = {1, 1, 1};
   for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
   for (int i = 0; i < rank - 1; ++i) s[i] = strides[i];
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, b, e,
+  return fn(m, dt, rank, const_cast<void*>(base), d, s, b, e,
             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -158,13 +159,13 @@ inline mla_status_t out_proj(const void* o_lat, const void* wkv_b, void* out, in
 inline int prefill_splits() { return 1; }
 
 // Split-t plan for decode: enough (row, head group, split) units to give
-// each CTA pair of the GPU one, splits never shorter than one 64-key tile.
+// each CTA pair of the GPU one, splits never shorter than one 128-key score tile.
 inline int auto_decode_splits(int batch, int H, int64_t max_seqlen_k, int sms) {
   if (batch <= 0) return 1;
   const int64_t pairs = sms / 2;
   const int64_t rows = (int64_t)batch * (H / 128);
   int64_t s = pairs / rows;
-  const int64_t max_tiles = (max_seqlen_k + kTileN - 1) / kTileN;
+  const int64_t max_tiles = (max_seqlen_k + kTileQ - 1) / kTileQ;
   if (s > max_tiles) s = max_tiles;
   if (s > 256) s = 256;
   return s < 1 ? 1 : (int)s;
@@ -174,7 +175,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 inline size_t workspace_bytes(int H, int64_t n_q, int splits) {
   if (splits <= 1) return 0;
-  return align256((size_t)splits * n_q * H * 512 * sizeof(float)) + align256((size_t)splits * n_q * H * 2 * sizeof(float));
+  // bf16 partial O per (split, row, head) + fp32 (reference max, row sum)
+  return align256((size_t)splits * n_q * H * 512 * 2) + align256((size_t)splits * n_q * H * 2 * sizeof(float));
 }
 
 inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_stride, const void* kv, const void* pe,
@@ -184,30 +186,43 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   const int64_t units = n_q * (H / 128) * splits;
   if (units == 0) return MLA_OK;
   if (2 * units >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
-  CUtensorMap tkv, tpe, tqpe;
-  if ((uint64_t)n_q * H >= (1ULL << 31)) return MLA_ERR_INVALID_ARG;
+  if ((uint64_t)n_q * H * (uint64_t)splits >= (1ULL << 31)) return MLA_ERR_INVALID_ARG;
+  CUtensorMap tkv_s, tpe, tqpe, tkv_v, tout;
   // kv_rows may be 0 (every sequence empty); the maps still need one row.
   const uint64_t rows = kv_rows > 0 ? (uint64_t)kv_rows : 1;
-  const uint64_t kd[2] = {512, rows}, ks[1] = {1024};
-  const uint32_t kb[2] = {64, (uint32_t)kTileN};
-  const uint64_t pd[2] = {64, rows}, ps[1] = {128};
-  const uint32_t pb[2] = {32, (uint32_t)kTileN};
-  const uint64_t qd[3] = {192, (uint64_t)H, (uint64_t)n_q}, qs[2] = {384, (uint64_t)q_row_stride * 2};
-  const uint32_t qb[3] = {32, 128, 1};
   const void* kv_base = kv_rows > 0 ? kv : q_abs;   // any valid 16-byte aligned address for an unused map
   const void* pe_base = kv_rows > 0 ? pe : q_abs;
-  if (!make_map(&tkv, kv_base, 2, kd, ks, kb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-  if (!make_map(&tpe, pe_base, 2, pd, ps, pb, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
-  if (!make_map(&tqpe, q, 3, qd, qs, qb, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
-  CUtensorMap tqa;   // q_abs viewed as [n_q * H, 512]: boxes of 128 heads x 64 latent columns
-  const uint64_t ad[2] = {512, (uint64_t)n_q * H}, as[1] = {1024};
-  const uint32_t ab[2] = {64, 128};
-  if (!make_map(&tqa, q_abs, 2, ad, as, ab, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-
+  {
+    const uint64_t d[2] = {512, rows}, st[1] = {1024};
+    const uint32_t bs[2] = {64, (uint32_t)kTileQ};    // score CTA: 64 latent columns x 128 keys
+    const uint32_t bv[2] = {64, (uint32_t)kTileN};    // value CTA: 64 latent columns x 64 keys
+    if (!make_map(&tkv_s, kv_base, 2, d, st, bs, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    if (!make_map(&tkv_v, kv_base, 2, d, st, bv, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
+  {
+    const uint64_t d[2] = {64, rows}, st[1] = {128};
+    const uint32_t b[2] = {64, (uint32_t)kTileQ};     // 64 rotary columns x 128 keys
+    if (!make_map(&tpe, pe_base, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
+  {
+    // q viewed as [n_q, H, 192]; the box is the rotary part (columns 128..191) of 128 heads of one row
+    const uint64_t d[3] = {192, (uint64_t)H, (uint64_t)n_q}, st[2] = {384, (uint64_t)q_row_stride * 2};
+    const uint32_t b[3] = {64, 128, 1};
+    if (!make_map(&tqpe, q, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
+  CUtensorMap tqa;
+  {
+    // q_abs viewed as [n_q * H, 512]: boxes of 64 latent columns x 128 heads
+    const uint64_t d[2] = {512, (uint64_t)n_q * H}, st[1] = {1024};
+    const uint32_t b[2] = {64, 128};
+    if (!make_map(&tqa, q_abs, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
   AttnParams p;
   p.q_abs = static_cast<const __nv_bfloat16*>(q_abs);
   p.cu_q = cu_q;
   p.cu_k = cu_k;
+  p.kv = static_cast<const __nv_bfloat16*>(kv);
+  p.pe = static_cast<const __nv_bfloat16*>(pe);
   p.batch = batch;
   p.heads = H;
   p.head_groups = H / 128;
@@ -216,18 +231,27 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   p.n_q = n_q;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_lat = static_cast<__nv_bfloat16*>(o_lat);
-  p.part_o = nullptr;
   p.part_ml = nullptr;
+  __nv_bfloat16* part_o = nullptr;
   if (splits > 1) {
-    p.part_o = static_cast<float*>(ws);
-    p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)splits * n_q * H * 512 * 4));
+    part_o = static_cast<__nv_bfloat16*>(ws);
+    p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)splits * n_q * H * 512 * 2));
   }
-  if (!set_smem(latent_attn_kernel, AttnLayout::kAlloc)) return MLA_ERR_CUDA;
-  mla_status_t st = launch(true, latent_attn_kernel, dim3((unsigned)(2 * units)), dim3(kAttnThreads),
-                           AttnLayout::kAlloc, stream, tkv, tpe, tqpe, tqa, p);
+  {
+    // the epilogue's output, [rows, 512] bf16 in boxes of 64 columns x 32 rows: the split
+    // partials [splits * n_q * H, 512], or o_lat [n_q * H, 512] directly
+    const uint64_t d[2] = {512, (uint64_t)(splits > 1 ? splits : 1) * n_q * H}, st[1] = {1024};
+    const uint32_t b[2] = {64, 32};
+    if (!make_map(&tout, splits > 1 ? (void*)part_o : o_lat, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  if (!set_smem(latent_attn_kernel, kAttnSmem)) return MLA_ERR_CUDA;
+  mla_status_t st = launch(true, latent_attn_kernel, dim3((unsigned)(2 * units)), dim3(kAttnThreads), kAttnSmem,
+                           stream, tkv_s, tpe, tqpe, tkv_v, tout, tqa, p);
   if (st != MLA_OK || splits <= 1) return st;
   return launch(true, merge_splits_kernel, dim3((unsigned)n_q, H), dim3(128), 0, stream,
-                (const float*)p.part_o, (const float*)p.part_ml, splits, n_q, H, static_cast<__nv_bfloat16*>(o_lat));
+                (const __nv_bfloat16*)part_o, (const float*)p.part_ml, splits, n_q, H,
+                static_cast<__nv_bfloat16*>(o_lat));
 }
 
 }  // namespace sm100

@@ -6,40 +6,51 @@
 //   S[h,t] = (q_abs[h,:] . kv[t,:] + q_pe[h,:] . pe[t,:]) * scale
 //   P      = softmax_t(S)   (keys past the row's visible limit masked)
 //   o[h,:] = sum_t P[h,t] kv[t,:]
-// The latent cache serves as both key and value, so one shared-memory tile
-// of kv feeds both products: K-major for S = Q K^T, MN-major for O = P V.
+// The latent cache is both key and value.
 //
-// Why a CTA pair: the fp32 accumulator O for 128 heads x 512 columns is
-// 256 KB, all of one SM's tensor memory, leaving nothing for S.  So the two
-// CTAs of a cluster split the latent columns: CTA r keeps O[:, 256r..256r+255]
-// in TMEM and loads only those kv columns (plus rotary columns 32r..32r+31),
-// so no cache byte is read twice.  Each CTA computes the partial score over
-// its 288 contraction columns; the two partials (rounded to fp16 on both
-// sides, so both CTAs add the same two numbers) are exchanged through
-// distributed shared memory with st.async, summed, and both CTAs run the
-// same softmax, getting bit-identical P.
+// Why two CTAs: the fp32 accumulator O for 128 heads x 512 columns is 256 KB,
+// all of one SM's tensor memory, and the query needs 256 more columns.  So a
+// work unit runs on a cluster of two CTAs with fixed roles and a one-way
+// hand-off:
 //
-// Tensor memory (512 columns x 128 lanes, lane = head):
-//   [  0,256) O accumulator (fp32)       [256,384) this CTA's half of q_abs (bf16 pairs, MMA A operand)
-//   [384,448) S buffer 0 (fp32)          [448,512) S buffer 1
-// Shared memory: a 4-stage ring of 64-key tiles (4 x 8 KB latent boxes with
-// 128-byte swizzle + 4 KB rotary box with 64-byte swizzle), this CTA's q_pe
-// half (128 x 32), the P buffer (128 heads x 64 keys bf16, the A operand of
-// O += P V), a one-slot outbox and a two-slot inbox of fp16 partial scores
-// (one 16 KB bulk copy per tile).  P lives in shared memory so an S buffer is
-// free as soon as the softmax has read it: QK of tile j+2 does not wait for
-// the P V product of tile j.
+//   score CTA (rank 0): q_abs in TMEM, S = Q K^T over all 576 contraction
+//     columns for 128 keys at a time (36 tcgen05.mma with N = 128), the
+//     online softmax, and P (bf16, 64 keys at a time) staged in shared memory and
+//     sent to the value CTA with one bulk copy per warp.
+//   value CTA (rank 1): O in TMEM, O += P V (8 tcgen05.mma with N = 256 per
+//     64 keys, A = P and B = the kv tile, both from shared memory), the rare O
+//     rescale, and the epilogue (TMA stores of O or of the split partial).
 //
-// Warps: 0-7 softmax / epilogue (two warpgroups; thread (g, h) owns key
-// columns 32g..32g+31 of every tile for head h, and latent columns
-// 128g..128g+127 of O in the epilogue), 8 TMA producer, 9 MMA issuer and TMEM
-// owner.  The two halves of a row agree on its max through shared memory
-// once per tile.  The softmax runs one tile ahead on the
-// exchange: it reads and sends the partial scores of tile j+1 before it
-// finishes tile j, so the partner's data for a tile is usually there when it
-// is needed.  It is online with a lazily updated reference max: O is rescaled
-// only when a row max grows by more than 2^8.  Every wait is bounded; a wait
-// that runs out raises the device error word and the CTA takes its exit path.
+// The score CTA never waits for the value CTA except for a free P slot (two
+// slots), so the pair forms a pipeline instead of exchanging partial scores
+// every tile.  Each CTA streams its own copy of the kv rows: the score CTA
+// from HBM (it also prefetches its key range into L2), the value CTA a little
+// later from L2, so HBM sees each cache byte once.  N = 128 matters: with one
+// elected lane issuing, a 128 x 64 x 16 MMA takes 48 cycles where 32 would be
+// full rate, while N >= 128 runs at full rate.
+//
+// Score CTA.  TMEM: [0,256) q_abs (bf16 pairs; it lands by TMA in ring units
+// 5-10 and the staging slots and the softmax threads move it into TMEM), two S buffers of 128 columns at 256 and 384.  Shared
+// memory: a ring of eleven 16 KB units, a unit being one 64-column block of
+// 128 keys (eight latent blocks and the rotary block make a score tile) with
+// 128-byte swizzle, q_pe (128 heads x 64, the A operand of the rotary
+// products) and two P staging slots.  Warps 0-3 and 4-7 are two softmax warpgroups that take
+// alternate score tiles (thread = head row, all 128 keys); warp 8 loads,
+// warp 9 issues the MMAs.  The running reference max m of each row passes
+// from one warpgroup to the other once per tile through shared memory; it is
+// updated lazily (only when a tile's max exceeds it by more than 2^8), so
+// P <= 256.  When it moves, the factor 2^(m_old - m_new) travels with P and
+// the value CTA rescales O before the next P V product.
+//
+// Value CTA.  TMEM: O, all 512 columns.  Shared memory: a 3-stage ring of
+// 64-key kv tiles (eight 8 KB boxes) and two P slots (P 16 KB, the per-row
+// factor, and in slot 0 the final row sums).  Warps 0-3 check each tile's
+// factors (and rescale O when one moved), zero the tail rows of the last
+// tile's values, and release the P V product; warp 8 loads, warp 9 issues
+// the MMAs and hands P slots back; warps 0-7 run the epilogue.
+//
+// Every wait is bounded; a wait that runs out raises the device error word
+// and the thread takes its exit path.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -48,37 +59,56 @@ namespace mla {
 namespace sm100 {
 
 constexpr int kAttnThreads = 320;
-constexpr int kSoftmaxThreads = 256;   // warps 0-7
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kTileN = 64;     // keys per tile
-constexpr int kStages = 4;
-constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr int kTileN = 64;                 // keys per P tile (value CTA granule)
+constexpr int kTileQ = 128;                // keys per score tile
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kPrefetchTiles = 1;          // L2 prefetch distance of the score CTA, in score tiles
 
-struct AttnLayout {
-  static constexpr int kKvBox = kTileN * 128;           // 64 keys x 64 bf16 latent columns
-  static constexpr int kKv = 4 * kKvBox;                // this CTA's 256 latent columns
-  static constexpr int kPe = kTileN * 64;               // 64 keys x 32 bf16 rotary columns
-  static constexpr int kStage = kKv + kPe;              // 36 KB, a multiple of 1024
-  static constexpr int kQpe = 128 * 64;                 // 128 heads x 32 bf16
-  static constexpr int kP = 128 * kTileN * 2;           // 128 heads x 64 keys bf16 = 16 KB
-  static constexpr int kXchgSlot = 128 * kTileN * 2;    // 128 heads x 64 fp16 partial scores = 16 KB
-  // P buffer, outbox and the two inbox slots are contiguous (64 KB).  Before
-  // the first tile they are the landing zone of this CTA's q_abs half (4 boxes
-  // of 128 heads x 64 latent columns, 16 KB each) on its way into TMEM.
-  static constexpr int kOffQpe = kStages * kStage;
-  static constexpr int kOffP = kOffQpe + kQpe;
-  static constexpr int kOffOutbox = kOffP + kP;
-  static constexpr int kOffInbox = kOffOutbox + kXchgSlot;
-  static constexpr int kOffBars = kOffInbox + 2 * kXchgSlot;
-  static constexpr int kOffMisc = kOffBars + 256;      // per-row max of each half [2 slots][2][128], sums [2][128]
-  static constexpr int kBytes = kOffMisc + 4096;
-  static constexpr int kAlloc = kBytes + 1024;          // room to align the base to 1024
+// Score CTA shared memory.
+struct ScoreLayout {
+  static constexpr int kUnit = kTileQ * 128;               // 128 keys x 64 columns bf16 (one TMA box)
+  static constexpr int kUnits = 11;
+  static constexpr int kUnitsPerTile = 9;                  // 8 latent blocks + the rotary block
+  static constexpr int kOffQpe = kUnits * kUnit;           // q_pe: 128 heads x 64 bf16
+  static constexpr int kOffStaging = kOffQpe + 128 * 128;  // two P staging slots, laid out like the value CTA's
+  static constexpr int kSlot = 17408;                      // P 16 KB, factors 512 B, then 512 B of
+  static constexpr int kOffMInSlot = 16896;                //   reference-max hand-off for warpgroup (slot index)
+  static constexpr int kOffEndL = kOffStaging + 2 * kSlot; // warpgroup 1's row sums at the end [128]
+  static constexpr int kOffBars = kOffEndL + 512;
+  static constexpr int kBytes = kOffBars + 512;
+  // q_abs lands before the first tile in units 5..10 (boxes 0-5) and the staging slots (boxes 6-7)
+  static constexpr int kQUnit0 = 5;
 };
+
+// Value CTA shared memory.
+struct ValueLayout {
+  static constexpr int kKvBox = kTileN * 128;              // 64 keys x 64 latent columns bf16
+  static constexpr int kStage = 8 * kKvBox;                // 64 keys x 512 latent columns
+  static constexpr int kStages = 3;
+  static constexpr int kOffSlots = kStages * kStage;       // two P slots
+  static constexpr int kSlot = 17408;                      // 1024-aligned
+  static constexpr int kP = 128 * kTileN * 2;              // P: 128 heads x 64 keys bf16, 16 KB
+  static constexpr int kOffF = kP;                         // in a slot: the per-row factors, 512 B
+  static constexpr int kOffL = kOffSlots + kP + 512;       // in slot 0: the final row sums, 512 B
+  static constexpr int kOffBars = kOffSlots + 2 * kSlot;
+  static constexpr int kBytes = kOffBars + 512;
+};
+
+constexpr int kAttnSmem = ScoreLayout::kBytes > ValueLayout::kBytes ? ScoreLayout::kBytes : ValueLayout::kBytes;
+static_assert(kAttnSmem <= 232448, "attention shared memory above the per-CTA limit");
+static_assert(ScoreLayout::kOffQpe % 1024 == 0 && ScoreLayout::kOffStaging % 1024 == 0 &&
+                  ValueLayout::kOffSlots % 1024 == 0 && ValueLayout::kSlot % 1024 == 0,
+              "swizzled operands need 1024-byte alignment");
+static_assert(ScoreLayout::kSlot == ValueLayout::kSlot, "staging and P slots share one layout");
+static_assert(ValueLayout::kP + 1024 <= ValueLayout::kSlot, "P slot too small");
 
 struct AttnParams {
   const __nv_bfloat16* q_abs;   // [n_q, H, 512]
   const int* cu_q;              // [batch+1] for chunked prefill, nullptr for decode
   const int* cu_k;              // [batch+1]
+  const __nv_bfloat16* kv;      // [kv_rows, 512] (L2 prefetch)
+  const __nv_bfloat16* pe;      // [kv_rows, 64]
   int batch;
   int heads;
   int head_groups;              // heads / 128
@@ -86,87 +116,600 @@ struct AttnParams {
   int64_t kv_rows;
   int64_t n_q;
   float scale_log2;             // softmax_scale * log2(e)
-  __nv_bfloat16* o_lat;         // [n_q, H, 512], written when num_splits == 1
-  float* part_o;                // [splits, n_q, H, 512]
-  float* part_ml;               // [splits, n_q, H, 2] = (reference max in log2 units, sum)
+  __nv_bfloat16* o_lat;         // [n_q, H, 512]; plain stores only for units with no key
+  float* part_ml;               // [splits, n_q, H, 2] = (reference max in log2 units, row sum)
 };
 
-__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-__device__ __forceinline__ float2 f16x2_to_f2(uint32_t v) {
-  __half2 h = *reinterpret_cast<__half2*>(&v);
-  return __half22float2(h);
-}
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
-    latent_attn_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_pe,
-                       const __grid_constant__ CUtensorMap tmap_qpe, const __grid_constant__ CUtensorMap tmap_qabs,
-                       const AttnParams p) {
-  using L = AttnLayout;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qpe_s = smem + L::kOffQpe;
-  uint8_t* p_s = smem + L::kOffP;
-  uint8_t* xchg = smem + L::kOffP;      // q_abs landing zone = P + outbox + inbox
-  uint8_t* outbox = smem + L::kOffOutbox;
-  uint8_t* inbox = smem + L::kOffInbox;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBars);
-  // barrier slots, laid out from kStages so the ring depth can change safely
-  uint64_t* kv_full = bars;                      // [kStages] TMA tile landed
-  uint64_t* kv_empty = kv_full + kStages;        // [kStages] tile no longer read by the tensor core
-  uint64_t* s_full = kv_empty + kStages;         // [2]  QK product committed
-  uint64_t* s_free = s_full + 2;                 // [2]  softmax read S (256 arrivals)
-  uint64_t* p_ready = s_free + 2;                // [2]  P written (256 arrivals)
-  uint64_t* xchg_full = p_ready + 2;             // [2]  partner's partial scores landed in my inbox
-  uint64_t* xchg_free = xchg_full + 2;           // [2]  partner's inbox slot is free (8 arrivals from its warps)
-  uint64_t* outbox_ready = xchg_free + 2;        // [2]  all rows of my partial written (256 arrivals)
-  uint64_t* mx_bar = outbox_ready + 2;           // [2]  both halves published their tile max (256 arrivals)
-  uint64_t* o_done = mx_bar + 2;                 // one phase per P V product
-  uint64_t* o_final = o_done + 1;                // the last P V product finished
-  uint64_t* q_ready = o_final + 1;               // q_abs half stored in TMEM (256 arrivals)
-  uint64_t* q_full = q_ready + 1;                // q_abs half landed in the exchange area
-  uint64_t* qpe_full = q_full + 1;
-  uint64_t* mma_idle = qpe_full + 1;             // every MMA of this CTA finished
-  uint64_t* outbox_free = mma_idle + 1;          // the partner received my last copy (its MMA warp arrives)
-  uint64_t* l_bar = outbox_free + 1;             // both halves published their sums (256 arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(l_bar + 1);
-  static_assert(2 * kStages + 22 + 1 <= 256 / 8, "barrier area too small");   // 8-byte slots incl. the TMEM address
-  float* half_max = reinterpret_cast<float*>(smem + L::kOffMisc);          // [2][2][128]
-  float* half_sum = half_max + 512;                                        // [2][128]
+// A unit's query row, head group, split and key range [j_begin, j_end) within
+// its sequence (whose first cache row is k0); nt = number of 64-key P tiles.
+struct UnitRange {
+  int64_t row, k0, j_begin, j_end;
+  int hg, sp, nt;
+};
 
+__device__ __forceinline__ UnitRange unit_range(const AttnParams& p, int64_t unit) {
+  UnitRange u;
+  const int per_row = p.head_groups * p.num_splits;
+  u.row = unit / per_row;
+  u.hg = (int)((unit % per_row) / p.num_splits);
+  u.sp = (int)(unit % p.num_splits);
+  const int b = p.cu_q ? find_sequence(p.cu_q, p.batch, u.row) : (int)u.row;
+  u.k0 = min64(max64(0, __ldg(p.cu_k + b)), p.kv_rows);
+  const int64_t t = max64(0, min64((int64_t)__ldg(p.cu_k + b + 1), p.kv_rows) - u.k0);
+  int64_t visible = t;
+  if (p.cu_q) {
+    // query i of s new queries (aligned to the end of the cache) sees keys 0 .. t - s + i
+    const int64_t q0 = __ldg(p.cu_q + b);
+    const int64_t s = max64(0, (int64_t)__ldg(p.cu_q + b + 1) - q0);
+    visible = min64(t, max64(0, t - s + (u.row - q0) + 1));
+  }
+  // splits are whole score tiles
+  const int64_t per = ((visible + p.num_splits - 1) / p.num_splits + kTileQ - 1) / kTileQ * kTileQ;
+  u.j_begin = min64(visible, (int64_t)u.sp * per);
+  u.j_end = min64(visible, u.j_begin + per);
+  u.nt = (int)((u.j_end - u.j_begin + kTileN - 1) / kTileN);
+  return u;
+}
+
+// Barrier slots (8 bytes each) in the 512-byte barrier area of either role.
+namespace bar {
+// score CTA
+constexpr int kUFull = 0, kUEmpty = 13, kSFull = 26, kSFree = 28, kMBar = 30, kPFree = 32, kQFull = 34,
+              kQReady = 35, kEnd = 36, kScoreIdle = 37, kPSent = 38;
+// value CTA
+constexpr int kVFull = 0, kVEmpty = 3, kPFull = 6, kPvGo = 8, kPDone = 10, kOFinal = 12, kLFull = 13,
+              kValueIdle = 14;
+constexpr int kTmemSlot = 63;
+}  // namespace bar
+
+constexpr uint32_t kColQ = 0, kColS = 256;
+
+// ---------------------------------------------------------------- score CTA
+__device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const UnitRange& u, const AttnParams& p,
+                                           const CUtensorMap* tmap_kv, const CUtensorMap* tmap_pe,
+                                           const CUtensorMap* tmap_qpe, const CUtensorMap* tmap_qabs) {
+  using L = ScoreLayout;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBars);
+  uint64_t* u_full = bars + bar::kUFull;       // [13] ring unit landed
+  uint64_t* u_empty = bars + bar::kUEmpty;     // [13] ring unit read by the tensor core
+  uint64_t* s_full = bars + bar::kSFull;       // [2] QK product committed
+  uint64_t* s_free = bars + bar::kSFree;       // [2] S read out (128 arrivals)
+  uint64_t* m_bar = bars + bar::kMBar;         // [2] warpgroup g published the reference max of its tile (128)
+  uint64_t* p_free = bars + bar::kPFree;       // [2] the value CTA finished the P V product of this P slot
+  uint64_t* q_full = bars + bar::kQFull;       // q_abs and q_pe landed
+  uint64_t* q_ready = bars + bar::kQReady;     // q_abs in TMEM, its landing zone free (256 arrivals)
+  uint64_t* end_bar = bars + bar::kEnd;        // warpgroup 1 published its (l, m) (128)
+  uint64_t* p_sent = bars + bar::kPSent;       // [2] warpgroup g stored the P tiles of its score tile (4 warps)
+  uint64_t* idle = bars + bar::kScoreIdle;
   const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id();
-  const uint32_t rank = ptx::cluster_rank(), peer = rank ^ 1u;
+  const int ntp = u.nt;                        // 64-key P tiles
+  const int ntq = (ntp + 1) / 2;               // 128-key score tiles
+  const int nu = L::kUnitsPerTile * ntq;       // ring units
+  const int64_t key_base = u.k0 + u.j_begin;
+  const int head0 = u.hg * 128;
+  // where q_abs box b (latent columns 64b..) lands before the first tile
+  auto q_box = [&](int b) -> uint8_t* {
+    return b < 6 ? smem + (L::kQUnit0 + b) * L::kUnit : smem + L::kOffStaging + (b - 6) * L::kSlot;
+  };
+
+  if (warp == kProducerWarp) {
+    // ============================================================ producer
+    auto prefetch_tile = [&](int jj) {
+      const int64_t key = key_base + (int64_t)jj * kTileQ;
+      const int64_t rows = min64(kTileQ, p.kv_rows - key);
+      if (rows > 0) {
+        ptx::prefetch_l2(p.kv + key * 512, (uint32_t)(rows * 1024));
+        ptx::prefetch_l2(p.pe + key * 64, (uint32_t)(rows * 128));
+      }
+    };
+    int issued = 0;
+    if (ntp > 0) {
+      if (ptx::elect_one()) {
+        ptx::prefetch_tmap(tmap_kv);
+        ptx::prefetch_tmap(tmap_pe);
+        ptx::mbar_arrive_expect_tx(q_full, 8 * L::kUnit + 128 * 128);
+#pragma unroll
+        for (int b = 0; b < 8; ++b)
+          ptx::tma_load_2d(q_box(b), tmap_qabs, q_full, 64 * b, (int)(u.row * p.heads + head0));
+        ptx::tma_load_3d(smem + L::kOffQpe, tmap_qpe, q_full, 128, head0, (int)u.row);
+      }
+      __syncwarp();
+      for (int uu = 0; uu < nu; ++uu) {
+        const int slot = uu % L::kUnits, use = uu / L::kUnits;
+        const int jj = uu / L::kUnitsPerTile, cb = uu % L::kUnitsPerTile;
+        bool w = true;
+        if (uu >= L::kQUnit0 && uu < L::kUnits) w = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax);   // held q_abs
+        w = w && ptx::mbar_wait(&u_empty[slot], (use & 1) ^ 1, kErrTimeoutStageFree);
+        if (!__all_sync(0xffffffffu, w)) break;
+        if (ptx::elect_one()) {
+          const int key = (int)(key_base + (int64_t)jj * kTileQ);
+          ptx::mbar_arrive_expect_tx(&u_full[slot], L::kUnit);
+          if (cb < 8)
+            ptx::tma_load_2d(smem + slot * L::kUnit, tmap_kv, &u_full[slot], 64 * cb, key);
+          else
+            ptx::tma_load_2d(smem + slot * L::kUnit, tmap_pe, &u_full[slot], 0, key);
+          // once the ring is full, keep the next few tiles streaming into L2
+          // keep the score tile kPrefetchTiles ahead streaming into L2
+          if (kPrefetchTiles > 0 && cb == 0 && jj + kPrefetchTiles < ntq) prefetch_tile(jj + kPrefetchTiles);
+        }
+        __syncwarp();
+        issued = uu + 1;
+      }
+      // exit path: every copy this CTA started has landed before its shared memory goes away
+      for (int uu = (issued > L::kUnits ? issued - L::kUnits : 0); uu < issued; ++uu)
+        ptx::mbar_wait(&u_full[uu % L::kUnits], (uu / L::kUnits) & 1, kErrTimeoutDrain);
+      ptx::mbar_wait(q_full, 0, kErrTimeoutDrain);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ============================================================ MMA issuer
+    if (ntp > 0) {
+      constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, kTileQ, false, false);
+      bool ok = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, ok);
+      // K-major operands, 128-byte rows, 8-row groups 1024 bytes apart; the start
+      // address sits in the low bits, so byte offsets add directly (>> 4)
+      const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(smem), 16, 1024, ptx::kSwizzle128);
+      const uint64_t d_qpe = ptx::smem_desc(ptx::smem_u32(smem + L::kOffQpe), 16, 1024, ptx::kSwizzle128);
+      ptx::tc_fence_after();
+      // Each issue site has one fixed MMA form (the column-block loop is unrolled):
+      // a loop that can reach both the TMEM-A and the shared-memory-A form from one
+      // elected branch issued at a quarter of the tensor-core rate.
+      for (int jj = 0; ok && jj < ntq; ++jj) {
+        if (jj >= 2) {
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s_free[jj & 1], ((jj - 2) >> 1) & 1, kErrTimeoutSoftmax));
+          if (!ok) break;
+        }
+        const uint32_t scol = tmem + kColS + (uint32_t)(jj & 1) * kTileQ;
+#pragma unroll
+        for (int cb = 0; cb < L::kUnitsPerTile; ++cb) {
+          const int uu = L::kUnitsPerTile * jj + cb, slot = uu % L::kUnits;
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(&u_full[slot], (uu / L::kUnits) & 1, kErrTimeoutTmaFull));
+          if (!ok) break;
+          ptx::tc_fence_after();
+          const uint64_t d_b = d_ring + (uint32_t)((slot * L::kUnit) >> 4);
+          if (cb < 8) {
+            // latent block cb: A = q_abs columns 64cb.. in TMEM
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              if (ptx::elect_one())
+                ptx::mma_ts(scol, tmem + kColQ + 32 * cb + 8 * k, d_b + (uint32_t)((k * 32) >> 4), idesc,
+                            (cb | k) ? 1u : 0u);
+              __syncwarp();
+            }
+          } else {
+            // rotary block: A = q_pe in shared memory
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              if (ptx::elect_one())
+                ptx::mma_ss(scol, d_qpe + (uint32_t)((k * 32) >> 4), d_b + (uint32_t)((k * 32) >> 4), idesc, 1u);
+              __syncwarp();
+            }
+          }
+          if (ptx::elect_one()) {
+            ptx::mma_commit(&u_empty[slot]);
+            if (cb == 8) ptx::mma_commit(&s_full[jj & 1]);
+          }
+          __syncwarp();
+        }
+      }
+      // nothing of ours may still run in the tensor core when TMEM is freed
+      if (ptx::elect_one()) ptx::mma_commit(idle);
+      __syncwarp();
+      ptx::mbar_wait(idle, 0, kErrTimeoutDrain);
+    }
+    __syncwarp();
+  } else {
+    // ============================================================ softmax
+    const int g = (int)(warp >> 2);                 // warpgroup: score tiles jj with jj % 2 == g
+    const int qd = (int)(warp & 3);                 // TMEM lane quadrant
+    const int h = qd * 32 + (int)lane;              // head within the group = TMEM lane
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    const float sl2 = p.scale_log2;
+    // reference max published by warpgroup x for its latest tile: 128 floats in staging slot x's tail
+    auto m_slot = [&](int x) -> float* { return reinterpret_cast<float*>(smem + L::kOffStaging + x * L::kSlot + L::kOffMInSlot); };
+    float* end_l = reinterpret_cast<float*>(smem + L::kOffEndL);  // warpgroup 1's row sums at the end
+    bool ok = true;
+    float m_used = -INFINITY, l = 0.f;   // reference this warpgroup last used, and its row sum relative to it
+    if (ntp > 0) {
+      // q_abs row h, latent block b (columns 64b..) -> TMEM columns 32b.. (bf16 pairs); warpgroup g moves blocks 4g..4g+3
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(q_full, 0, kErrTimeoutTmaFull));
+      if (ok) {
+#pragma unroll 1
+        for (int b = 4 * g; b < 4 * g + 4; ++b) {
+          const uint8_t* src = q_box(b) + h * 128;
+          uint32_t r[32];
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 x = *reinterpret_cast<const uint4*>(src + ((v ^ (h & 7)) << 4));
+            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+          }
+          ptx::tmem_st32(tmem + lane_base + kColQ + 32 * b, r);
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+      }
+      ptx::mbar_arrive(q_ready);
+      const uint32_t v_base = ptx::map_peer(ptx::smem_u32(smem), 1);
+
+      for (int jj = g; ok && jj < ntq; jj += 2) {
+        const int sb = jj & 1;
+        bool w = ptx::mbar_wait(&s_full[sb], (jj >> 1) & 1, kErrTimeoutMma);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        ptx::tc_fence_after();
+        uint32_t s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t a[32];
+          ptx::tmem_ld32(tmem + lane_base + kColS + sb * kTileQ + 32 * c, a);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * c + i] = a[i];
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&s_free[sb]);                 // S buffer may take QK(jj+2)
+        const int n_valid = (int)min64(kTileQ, u.j_end - (u.j_begin + (int64_t)jj * kTileQ));
+        // row max of the raw scores over the valid keys (scale >= 0 commutes with max)
+        float mx;
+        {
+          float m8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i < n_valid) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(s[i]));
+          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          mx *= sl2;
+        }
+        // the reference after tile jj-1 comes from the other warpgroup
+        float m_prev = -INFINITY;
+        if (jj > 0) {
+          w = ptx::mbar_wait(&m_bar[g ^ 1], ((jj - 1) >> 1) & 1, kErrTimeoutSoftmax);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          m_prev = m_slot(g ^ 1)[h];
+        }
+        const float m_new = mx > m_prev + kRescaleThreshold ? mx : m_prev;
+        m_slot(g)[h] = m_new;
+        ptx::mbar_arrive(&m_bar[g]);
+        const float f = (jj == 0 || m_new == m_prev) ? 1.f : fast_exp2(m_prev - m_new);
+        if (m_used != m_new) {
+          l = m_used == -INFINITY ? 0.f : l * fast_exp2(m_used - m_new);
+          m_used = m_new;
+        }
+        // P tiles reach the value CTA's two slots strictly in order: the other warpgroup
+        // stored those of score tile jj-1 first.  (It hands over the reference max before
+        // its P, so without this a warpgroup could wait on a P slot barrier two phases
+        // ahead, which a parity wait cannot tell from the phase before.)
+        if (jj > 0) {
+          w = ptx::mbar_wait(&p_sent[g ^ 1], ((jj - 1) >> 1) & 1, kErrTimeoutSoftmax);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        }
+        // P = 2^(s * scale * log2(e) - m) as bf16, in two 64-key P tiles; keys past the end weigh exactly 0
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (kTileN * half >= n_valid) break;
+          const int t = 2 * jj + half, ps = t & 1;
+          if (t >= 2) {
+            w = ptx::mbar_wait<true>(&p_free[ps], ((t - 2) >> 1) & 1, kErrTimeoutPeer);
+            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          }
+          uint32_t pk[32];
+          float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int k = kTileN * half + 2 * i;
+            float e0 = fast_exp2(fmaf(__uint_as_float(s[k]), sl2, -m_new));
+            float e1 = fast_exp2(fmaf(__uint_as_float(s[k + 1]), sl2, -m_new));
+            if (k >= n_valid) e0 = 0.f;
+            if (k + 1 >= n_valid) e1 = 0.f;
+            ps0 += e0;
+            ps1 += e1;
+            pk[i] = ptx::pack_bf16x2(e0, e1);
+          }
+          l += ps0 + ps1;
+          // row h of the K-major P tile (128-byte swizzle) and the row's factor into staging slot ps,
+          // then this warp's 32 rows and factors to the value CTA's P slot ps (two bulk copies)
+          uint8_t* stg = smem + L::kOffStaging + ps * L::kSlot;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(stg + h * 128 + ((c ^ (h & 7)) << 4)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          reinterpret_cast<float*>(stg + ValueLayout::kOffF)[h] = half == 0 ? f : 1.f;
+          ptx::fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t dst = v_base + ValueLayout::kOffSlots + (uint32_t)ps * ValueLayout::kSlot;
+            const uint32_t vbar = v_base + ValueLayout::kOffBars + 8 * (bar::kPFull + ps);
+            ptx::bulk_copy_to_peer(dst + qd * 4096, ptx::smem_u32(stg) + qd * 4096, 4096, vbar);
+            ptx::bulk_copy_to_peer(dst + ValueLayout::kOffF + qd * 128, ptx::smem_u32(stg) + ValueLayout::kOffF + qd * 128,
+                                   128, vbar);
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) ptx::mbar_arrive(&p_sent[g]);
+      }
+      // the row's final (m, l): both warpgroups' sums taken to the last reference
+      // (warpgroup 1's last reference is the last one it published; it has none with one tile)
+      if (g == 1) {
+        end_l[h] = l;
+        ptx::mbar_arrive(end_bar);
+      } else if (ok) {
+        const bool w = ptx::mbar_wait(end_bar, 0, kErrTimeoutSoftmax);
+        if (__all_sync(0xffffffffu, w)) {
+          const float l1 = end_l[h], m1 = ntq > 1 ? m_slot(1)[h] : -INFINITY;
+          const float m_fin = fmaxf(m_used, m1);
+          const float lt = l * fast_exp2(m_used - m_fin) + (m1 == -INFINITY ? 0.f : l1 * fast_exp2(m1 - m_fin));
+          if (p.num_splits > 1) {
+            const int64_t slot = ((int64_t)u.sp * p.n_q + u.row) * p.heads + head0 + h;
+            reinterpret_cast<float2*>(p.part_ml)[slot] = make_float2(m_fin, lt);
+          }
+          ptx::st_async_b32(v_base + ValueLayout::kOffL + 4 * h, v_base + ValueLayout::kOffBars + 8 * bar::kLFull,
+                            __float_as_uint(lt));
+        }
+      }
+    } else if (p.num_splits > 1 && g == 0) {
+      // a split with no key contributes nothing to the merge
+      const int64_t slot = ((int64_t)u.sp * p.n_q + u.row) * p.heads + head0 + h;
+      reinterpret_cast<float2*>(p.part_ml)[slot] = make_float2(-INFINITY, 0.f);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- value CTA
+__device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const UnitRange& u, const AttnParams& p,
+                                           const CUtensorMap* tmap_kv, const CUtensorMap* tmap_out) {
+  using L = ValueLayout;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBars);
+  uint64_t* v_full = bars + bar::kVFull;      // [3] kv tile landed
+  uint64_t* v_empty = bars + bar::kVEmpty;    // [3] kv tile read by the tensor core
+  uint64_t* p_full = bars + bar::kPFull;      // [2] P and factors of a tile landed (bulk copies from the score CTA)
+  uint64_t* pv_go = bars + bar::kPvGo;        // [2] factors applied, tail cleared: P V may run (128 arrivals)
+  uint64_t* p_done = bars + bar::kPDone;      // [2] P V product of this slot finished
+  uint64_t* o_final = bars + bar::kOFinal;    // the last P V product finished
+  uint64_t* l_full = bars + bar::kLFull;      // the row sums landed
+  uint64_t* idle = bars + bar::kValueIdle;
+  const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id();
+  const int nt = u.nt;
+  const int64_t key_base = u.k0 + u.j_begin;
+
+  if (warp == kProducerWarp) {
+    // ============================================================ producer
+    int issued = 0;
+    if (nt > 0) {
+      if (ptx::elect_one()) ptx::prefetch_tmap(tmap_kv);
+      __syncwarp();
+      for (int j = 0; j < nt; ++j) {
+        const int st = j % L::kStages;
+        const bool w = ptx::mbar_wait(&v_empty[st], ((j / L::kStages) & 1) ^ 1, kErrTimeoutStageFree);
+        if (!__all_sync(0xffffffffu, w)) break;
+        if (ptx::elect_one()) {
+          const int key = (int)(key_base + (int64_t)j * kTileN);
+          ptx::mbar_arrive_expect_tx(&v_full[st], L::kStage);
+#pragma unroll
+          for (int bx = 0; bx < 8; ++bx)
+            ptx::tma_load_2d(smem + st * L::kStage + bx * L::kKvBox, tmap_kv, &v_full[st], 64 * bx, key);
+        }
+        __syncwarp();
+        issued = j + 1;
+      }
+      for (int j = (issued > L::kStages ? issued - L::kStages : 0); j < issued; ++j)
+        ptx::mbar_wait(&v_full[j % L::kStages], (j / L::kStages) & 1, kErrTimeoutDrain);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ============================================================ MMA issuer
+    // Two streams: P V of tile pv once its kv tile landed and its P was
+    // released, and handing P slot fw back to the score CTA once P V of tile
+    // fw finished (only for tiles the score CTA still waits on).
+    if (nt > 0) {
+      constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, 256, false, true);
+      const uint64_t d_p0 = ptx::smem_desc(ptx::smem_u32(smem + L::kOffSlots), 16, 1024, ptx::kSwizzle128);
+      const uint64_t d_v0 = ptx::smem_desc(ptx::smem_u32(smem), L::kKvBox, 1024, ptx::kSwizzle128);
+      const uint32_t score_free0 = ptx::map_peer(ptx::smem_u32(smem + ScoreLayout::kOffBars + 8 * bar::kPFree), 0);
+      bool ok = true;
+      int pv = 0, fw = 0;
+      uint64_t t_last = global_timer_ns();
+      while (ok && (pv < nt || fw < nt - 2)) {
+        bool progressed = false;
+        bool go = fw < nt - 2 && fw < pv && ptx::mbar_test(&p_done[fw & 1], (fw >> 1) & 1);
+        if (__shfl_sync(0xffffffffu, go, 0)) {
+          if (lane == 0) ptx::mbar_arrive_cluster_relaxed_addr(score_free0 + 8 * (fw & 1));
+          __syncwarp();
+          ++fw;
+          progressed = true;
+        }
+        go = pv < nt && ptx::mbar_test(&v_full[pv % L::kStages], (pv / L::kStages) & 1) &&
+             ptx::mbar_test(&pv_go[pv & 1], (pv >> 1) & 1);
+        if (__shfl_sync(0xffffffffu, go, 0)) {
+          ptx::tc_fence_after();
+          const uint32_t so = (uint32_t)((pv % L::kStages) * L::kStage) >> 4;
+          const uint32_t po = (uint32_t)((pv & 1) * L::kSlot) >> 4;
+#pragma unroll
+          for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int ks = 0; ks < kTileN / 16; ++ks) {
+              if (ptx::elect_one())
+                ptx::mma_ss(tmem + 256 * n, d_p0 + po + (uint32_t)((ks * 32) >> 4),
+                            d_v0 + so + (uint32_t)((n * 4 * L::kKvBox + ks * 2048) >> 4), idesc,
+                            (pv > 0 || ks > 0) ? 1u : 0u);
+              __syncwarp();
+            }
+          if (ptx::elect_one()) {
+            ptx::mma_commit(&v_empty[pv % L::kStages]);
+            ptx::mma_commit(&p_done[pv & 1]);
+            if (pv == nt - 1) ptx::mma_commit(o_final);
+          }
+          __syncwarp();
+          ++pv;
+          progressed = true;
+        }
+        if (progressed) {
+          t_last = global_timer_ns();
+        } else {
+          __nanosleep(20);
+          const bool late = global_timer_ns() - t_last > kWaitLimitNs;
+          if (__shfl_sync(0xffffffffu, late, 0)) {
+            if (lane == 0) raise_error(pv < nt ? kErrTimeoutPeer : kErrTimeoutMma);
+            ok = false;
+          }
+        }
+      }
+      if (ptx::elect_one()) ptx::mma_commit(idle);
+      __syncwarp();
+      ptx::mbar_wait(idle, 0, kErrTimeoutDrain);
+    }
+    __syncwarp();
+  } else {
+    // ============================================================ warps 0-7
+    const int qd = (int)(warp & 3);
+    const int h = qd * 32 + (int)lane;
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    bool ok = true;
+    if (nt > 0 && warp < 4) {
+      // per tile: apply the row factors to O (rare), clear the tail rows, release P V
+      if (threadIdx.x == 0) ptx::mbar_arrive_expect_tx(l_full, 512);
+      for (int j = 0; j < nt; ++j) {
+        const int s = j & 1;
+        if (threadIdx.x == 0) ptx::mbar_arrive_expect_tx(&p_full[s], L::kP + 512);   // 4 x (4 KB + 128 B)
+        bool w = ptx::mbar_wait<true>(&p_full[s], (j >> 1) & 1, kErrTimeoutPeer);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        const float f = reinterpret_cast<const float*>(smem + L::kOffSlots + s * L::kSlot + L::kOffF)[h];
+        if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
+          // O holds the products of tiles < j relative to the old reference: scale it
+          w = ptx::mbar_wait(&p_done[(j - 1) & 1], ((j - 1) >> 1) & 1, kErrTimeoutMma);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          ptx::tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tmem + lane_base + 32 * c, r);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+            ptx::tmem_st32(tmem + lane_base + 32 * c, r);
+          }
+          ptx::tmem_wait_st();
+        }
+        const int n_valid = (int)min64(kTileN, u.j_end - (u.j_begin + (int64_t)j * kTileN));
+        if (n_valid < kTileN) {
+          // keys past the end have P = 0, but 0 * NaN is NaN: clear their value rows
+          w = ptx::mbar_wait(&v_full[j % L::kStages], (j / L::kStages) & 1, kErrTimeoutTmaFull);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          uint8_t* st = smem + (j % L::kStages) * L::kStage;
+          const int rows = kTileN - n_valid;
+          for (int idx = (int)threadIdx.x; idx < 8 * rows * 8; idx += 128) {
+            const int bx = idx / (rows * 8), rem = idx % (rows * 8);
+            *reinterpret_cast<uint4*>(st + bx * L::kKvBox + (n_valid + rem / 8) * 128 + (rem % 8) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          ptx::fence_async_smem();
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&pv_go[s]);
+      }
+    }
+    // ---- epilogue: warp (qd, c) stores rows 32qd.. and latent columns 256c..256c+255 as bf16,
+    // either o_lat = O / l (one split) or the split's partial O (relative to its final reference)
+    const int c = (int)(warp >> 2);
+    if (nt == 0) {
+      if (p.num_splits == 1) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o_lat + (u.row * p.heads + u.hg * 128 + h) * 512 + 256 * c);
+        for (int v = 0; v < 32; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+      }
+    } else {
+      bool w = __all_sync(0xffffffffu, ok);
+      w = w && ptx::mbar_wait(o_final, 0, kErrTimeoutMma);
+      w = w && ptx::mbar_wait<true>(l_full, 0, kErrTimeoutPeer);   // also before exit: it writes here
+      if (__all_sync(0xffffffffu, w)) {
+        ptx::tc_fence_after();
+        uint8_t* stage = smem + warp * 16384;   // the kv ring is idle now: four 4 KB store boxes per warp
+        const float inv = p.num_splits > 1 ? 1.f : 1.f / reinterpret_cast<const float*>(smem + L::kOffL)[h];
+        const int64_t row0 = p.num_splits > 1 ? ((int64_t)u.sp * p.n_q + u.row) * p.heads : u.row * p.heads;
+        const int y = (int)(row0 + u.hg * 128 + 32 * qd);
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+          uint8_t* buf = stage + k * 4096;
+          uint32_t r[32], r2[32];
+          ptx::tmem_ld32(tmem + lane_base + 256 * c + 64 * k, r);
+          ptx::tmem_ld32(tmem + lane_base + 256 * c + 64 * k + 32, r2);
+          ptx::tmem_wait_ld();
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            pk[i] = ptx::pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+            pk[16 + i] = ptx::pack_bf16x2(__uint_as_float(r2[2 * i]) * inv, __uint_as_float(r2[2 * i + 1]) * inv);
+          }
+          // a 32-row x 128-byte box with 128-byte swizzle
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((v ^ (lane & 7)) << 4)) =
+                make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          ptx::fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_store_2d(tmap_out, buf, 256 * c + 64 * k, y);
+            ptx::bulk_commit_group();
+          }
+        }
+        if (lane == 0) ptx::bulk_wait_group_all();
+        __syncwarp();
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- the kernel
+// One cluster of two CTAs per work unit (query row, 128-head group, split).
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
+    latent_attn_kernel(const __grid_constant__ CUtensorMap tmap_kv_score, const __grid_constant__ CUtensorMap tmap_pe,
+                       const __grid_constant__ CUtensorMap tmap_qpe, const __grid_constant__ CUtensorMap tmap_kv_value,
+                       const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ CUtensorMap tmap_qabs,
+                       const AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t warp = ptx::warp_id();
+  const uint32_t rank = ptx::cluster_rank();
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (rank == 0 ? ScoreLayout::kOffBars : ValueLayout::kOffBars));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + bar::kTmemSlot);
+  // the swizzled tiles need a 1024-byte aligned base (both CTAs see the same alignment)
+  const bool aligned = (ptx::smem_u32(smem) & 1023u) == 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(&kv_full[s], 1);
-      ptx::mbar_init(&kv_empty[s], 1);
+    if (rank == 0) {
+      for (int s = 0; s < ScoreLayout::kUnits; ++s) {
+        ptx::mbar_init(&bars[bar::kUFull + s], 1);
+        ptx::mbar_init(&bars[bar::kUEmpty + s], 1);
+      }
+      for (int s = 0; s < 2; ++s) {
+        ptx::mbar_init(&bars[bar::kSFull + s], 1);
+        ptx::mbar_init(&bars[bar::kSFree + s], 128);
+        ptx::mbar_init(&bars[bar::kMBar + s], 128);
+        ptx::mbar_init(&bars[bar::kPFree + s], 1);
+        ptx::mbar_init(&bars[bar::kPSent + s], 4);
+      }
+      ptx::mbar_init(&bars[bar::kQFull], 1);
+      ptx::mbar_init(&bars[bar::kQReady], 256);
+      ptx::mbar_init(&bars[bar::kEnd], 128);
+      ptx::mbar_init(&bars[bar::kScoreIdle], 1);
+    } else {
+      for (int s = 0; s < ValueLayout::kStages; ++s) {
+        ptx::mbar_init(&bars[bar::kVFull + s], 1);
+        ptx::mbar_init(&bars[bar::kVEmpty + s], 1);
+      }
+      for (int s = 0; s < 2; ++s) {
+        ptx::mbar_init(&bars[bar::kPFull + s], 1);
+        ptx::mbar_init(&bars[bar::kPvGo + s], 128);
+        ptx::mbar_init(&bars[bar::kPDone + s], 1);
+      }
+      ptx::mbar_init(&bars[bar::kOFinal], 1);
+      ptx::mbar_init(&bars[bar::kLFull], 1);
+      ptx::mbar_init(&bars[bar::kValueIdle], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(&s_full[s], 1);
-      ptx::mbar_init(&s_free[s], kSoftmaxThreads);
-      ptx::mbar_init(&p_ready[s], kSoftmaxThreads);
-      ptx::mbar_init(&xchg_full[s], 1);
-      ptx::mbar_init(&xchg_free[s], kSoftmaxThreads / 32);
-      ptx::mbar_init(&outbox_ready[s], kSoftmaxThreads);
-      ptx::mbar_init(&mx_bar[s], kSoftmaxThreads);
-    }
-    ptx::mbar_init(l_bar, kSoftmaxThreads);
-    ptx::mbar_init(outbox_free, 1);
-    ptx::mbar_init(o_done, 1);
-    ptx::mbar_init(o_final, 1);
-    ptx::mbar_init(q_ready, kSoftmaxThreads);
-    ptx::mbar_init(q_full, 1);
-    ptx::mbar_init(qpe_full, 1);
-    ptx::mbar_init(mma_idle, 1);
     ptx::fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -182,456 +725,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
 
-  // ---- work unit: (query row, head group, split) -------------------------
-  const int64_t unit = blockIdx.x >> 1;
-  const int per_row = p.head_groups * p.num_splits;
-  const int64_t row = unit / per_row;
-  const int hg = (int)((unit % per_row) / p.num_splits);
-  const int sp = (int)(unit % p.num_splits);
-  const int b = p.cu_q ? find_sequence(p.cu_q, p.batch, row) : (int)row;
-  const int64_t k0 = min64(max64(0, __ldg(p.cu_k + b)), p.kv_rows);
-  const int64_t t = max64(0, min64((int64_t)__ldg(p.cu_k + b + 1), p.kv_rows) - k0);
-  int64_t visible = t;
-  if (p.cu_q) {
-    const int64_t q0 = __ldg(p.cu_q + b);
-    const int64_t s = max64(0, (int64_t)__ldg(p.cu_q + b + 1) - q0);
-    visible = min64(t, max64(0, t - s + (row - q0) + 1));
+  UnitRange u = unit_range(p, blockIdx.x >> 1);
+  if (!aligned) {
+    if (threadIdx.x == 0) raise_error(kErrBadSchedule);
+    u.nt = 0;
   }
-  const int64_t per = ((visible + p.num_splits - 1) / p.num_splits + kTileN - 1) / kTileN * kTileN;
-  const int64_t j_begin = min64(visible, (int64_t)sp * per);
-  const int64_t j_end = min64(visible, j_begin + per);
-  const int nt = (int)((j_end - j_begin + kTileN - 1) / kTileN);
-  const int head0 = hg * 128;
-
-
-  constexpr uint32_t kColO = 0, kColQ = 256, kColS = 384;
-
-  if (warp == kProducerWarp) {
-    // ================================================= TMA producer ======
-    // The whole warp runs the loop (waits are warp-wide); one elected lane issues.
-    int issued = 0;
-    if (ptx::elect_one()) {
-      ptx::prefetch_tmap(&tmap_kv);
-      ptx::prefetch_tmap(&tmap_pe);
-      if (nt > 0) {
-        ptx::mbar_arrive_expect_tx(q_full, 4 * L::kXchgSlot);
-#pragma unroll
-        for (int bx = 0; bx < 4; ++bx)
-          ptx::tma_load_2d(xchg + bx * L::kXchgSlot, &tmap_qabs, q_full, 256 * (int)rank + 64 * bx,
-                           (int)(row * p.heads + head0));
-        ptx::mbar_arrive_expect_tx(qpe_full, L::kQpe);
-        ptx::tma_load_3d(qpe_s, &tmap_qpe, qpe_full, 128 + 32 * (int)rank, head0, (int)row);
-      }
-    }
-    __syncwarp();
-    for (int j = 0; j < nt; ++j) {
-      const int s = j % kStages;
-      const bool w = ptx::mbar_wait(&kv_empty[s], ((j / kStages) & 1) ^ 1, kErrTimeoutStageFree);
-      if (!__all_sync(0xffffffffu, w)) break;
-      if (ptx::elect_one()) {
-        uint8_t* st = smem + s * L::kStage;
-        ptx::mbar_arrive_expect_tx(&kv_full[s], L::kStage);
-        const int key = (int)(k0 + j_begin + (int64_t)j * kTileN);
-#pragma unroll
-        for (int bx = 0; bx < 4; ++bx)
-          ptx::tma_load_2d(st + bx * L::kKvBox, &tmap_kv, &kv_full[s], 256 * (int)rank + 64 * bx, key);
-        ptx::tma_load_2d(st + L::kKv, &tmap_pe, &kv_full[s], 32 * (int)rank, key);
-      }
-      __syncwarp();
-      issued = j + 1;
-    }
-    // exit path: every copy this CTA started has landed before its smem goes away
-    for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-      ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, kErrTimeoutDrain);
-    if (nt > 0) {
-      ptx::mbar_wait(qpe_full, 0, kErrTimeoutDrain);
-      ptx::mbar_wait(q_full, 0, kErrTimeoutDrain);
-    }
-    __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ================================================= MMA issuer ========
-    // Two streams issued as their inputs arrive: QK(j) needs tile j and S
-    // buffer j&1 read out (tile j-2); PV(j) needs P(j).  QK runs ahead of PV,
-    // so the scores of the next tiles are ready while the softmax works.
-    // The whole warp runs the loop with warp-uniform decisions; one elected
-    // lane issues each MMA and commit.
-    if (nt > 0) {
-      constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(128, kTileN, false, false);
-      constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(128, 256, false, true);
-      bool ok = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax) && ptx::mbar_wait(qpe_full, 0, kErrTimeoutTmaFull);
-      ok = __all_sync(0xffffffffu, ok);
-      // descriptor bases; the start address sits in the low bits, so offsets add directly (>> 4)
-      const uint64_t d_stage0 = ptx::smem_desc(ptx::smem_u32(smem), 16, 1024, ptx::kSwizzle128);
-      const uint64_t d_pe0 = ptx::smem_desc(ptx::smem_u32(smem + L::kKv), 16, 512, ptx::kSwizzle64);
-      const uint64_t d_qpe = ptx::smem_desc(ptx::smem_u32(qpe_s), 16, 512, ptx::kSwizzle64);
-      const uint64_t d_p0 = ptx::smem_desc(ptx::smem_u32(p_s), 16, 1024, ptx::kSwizzle128);
-      const uint64_t d_v0 = ptx::smem_desc(ptx::smem_u32(smem), L::kKvBox, 1024, ptx::kSwizzle128);
-      int qk = 0, pv = 0, fw = 0;
-      uint64_t t_last = global_timer_ns();
-      ptx::tc_fence_after();
-      // Third stream: as soon as the partner's copy of tile fw has landed in my
-      // inbox, tell it (its single outbox may be refilled).  This must not wait
-      // for the softmax: the softmax sends tile j+1 before it finishes tile j.
-      while (ok && (pv < nt || fw < nt - 1)) {
-        bool progressed = false;
-        bool go_fw = fw < nt - 1 && ptx::mbar_test(&xchg_full[fw & 1], (fw >> 1) & 1);
-        if (__shfl_sync(0xffffffffu, go_fw, 0)) {
-          if (lane == 0) ptx::mbar_arrive_cluster_relaxed(outbox_free, peer);
-          __syncwarp();
-          ++fw;
-          progressed = true;
-        }
-        bool go = qk < nt && (qk < 2 || ptx::mbar_test(&s_free[qk & 1], ((qk - 2) >> 1) & 1)) &&
-                  ptx::mbar_test(&kv_full[qk % kStages], (qk / kStages) & 1);
-        if (__shfl_sync(0xffffffffu, go, 0)) {
-          ptx::tc_fence_after();
-          const uint32_t so = (uint32_t)((qk % kStages) * L::kStage) >> 4;
-          const uint32_t scol = tmem + kColS + (qk & 1) * kTileN;
-#pragma unroll
-          for (int ks = 0; ks < 16; ++ks) {
-            if (ptx::elect_one())
-              ptx::mma_ts(scol, tmem + kColQ + ks * 8,
-                          d_stage0 + so + (((ks >> 2) * L::kKvBox + (ks & 3) * 32) >> 4), idesc_qk,
-                          ks > 0 ? 1u : 0u);
-            __syncwarp();
-          }
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            if (ptx::elect_one()) ptx::mma_ss(scol, d_qpe + ((ks * 32) >> 4), d_pe0 + so + ((ks * 32) >> 4), idesc_qk, 1u);
-            __syncwarp();
-          }
-          if (ptx::elect_one()) ptx::mma_commit(&s_full[qk & 1]);
-          __syncwarp();
-          ++qk;
-          progressed = true;
-        }
-        go = pv < qk && ptx::mbar_test(&p_ready[pv & 1], (pv >> 1) & 1);
-        if (__shfl_sync(0xffffffffu, go, 0)) {
-          ptx::tc_fence_after();
-          const uint32_t so = (uint32_t)((pv % kStages) * L::kStage) >> 4;
-#pragma unroll
-          for (int ks = 0; ks < kTileN / 16; ++ks) {
-            if (ptx::elect_one())
-              ptx::mma_ss(tmem + kColO, d_p0 + ((ks * 32) >> 4), d_v0 + so + ((ks * 2048) >> 4), idesc_pv,
-                          (pv > 0 || ks > 0) ? 1u : 0u);
-            __syncwarp();
-          }
-          if (ptx::elect_one()) {
-            ptx::mma_commit(&kv_empty[pv % kStages]);
-            ptx::mma_commit(o_done);
-            if (pv == nt - 1) ptx::mma_commit(o_final);
-          }
-          __syncwarp();
-          ++pv;
-          progressed = true;
-        }
-        if (progressed) {
-          t_last = global_timer_ns();
-        } else {
-          __nanosleep(20);
-          bool late = global_timer_ns() - t_last > kWaitLimitNs;
-          if (__shfl_sync(0xffffffffu, late, 0)) {
-            if (lane == 0) raise_error(qk < nt ? kErrTimeoutTmaFull : kErrTimeoutSoftmax);
-            ok = false;
-          }
-        }
-      }
-      // nothing of ours may still be running in the tensor core when TMEM is freed
-      if (ptx::elect_one()) ptx::mma_commit(mma_idle);
-      __syncwarp();
-      ptx::mbar_wait(mma_idle, 0, kErrTimeoutDrain);
-    }
-    __syncwarp();
-  } else {
-    // ================================================= softmax (warps 0-7)
-    const int g = (int)(warp >> 2);                    // half: key columns 32g.. of a tile, O columns 128g..
-    const int h = (int)((warp & 3) * 32 + lane);       // head within the group = TMEM lane
-    const uint32_t lane_base = (warp & 3) * 32u << 16;
-    const int64_t head = head0 + h;
-    const uint32_t sw = (uint32_t)(h & 7);             // 128-byte swizzle phase of row h
-    bool ok = true;
-    float m_ref = -INFINITY, l = 0.f;                  // l: this half's share of the row sum
-    if (nt > 0) {
-      // this CTA's half of q_abs: exchange area (TMA, 128-byte swizzle) -> TMEM columns [256, 384)
-      bool w = ptx::mbar_wait(q_full, 0, kErrTimeoutTmaFull);
-      ok = __all_sync(0xffffffffu, w);
-      if (ok) {
-#pragma unroll 1
-        for (int c = 2 * g; c < 2 * g + 2; ++c) {
-          const uint8_t* src = xchg + c * L::kXchgSlot + h * 128;
-          uint32_t r[32];
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const uint4 x = *reinterpret_cast<const uint4*>(src + ((v ^ sw) << 4));
-            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
-          }
-          ptx::tmem_st32(tmem + lane_base + kColQ + c * 32, r);
-        }
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(q_ready);
-        // every softmax thread has read its part of the landing zone before any is reused
-        w = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax);
-        ok = __all_sync(0xffffffffu, w);
-      }
-      if (ok) {
-        // the inbox is free again: the partner may send into it
-        __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive_cluster_relaxed(&xchg_free[0], peer);
-          ptx::mbar_arrive_cluster_relaxed(&xchg_free[1], peer);
-        }
-      }
-
-      const uint32_t peer_inbox = ptx::map_peer(ptx::smem_u32(inbox), peer);
-      const uint32_t peer_full0 = ptx::map_peer(ptx::smem_u32(&xchg_full[0]), peer);
-      const uint32_t peer_full1 = ptx::map_peer(ptx::smem_u32(&xchg_full[1]), peer);
-      const float sl2 = p.scale_log2;
-
-      // Send: my 32 partial scores of tile j (TMEM -> fp16 -> outbox -> one bulk
-      // copy of the whole outbox into the partner's inbox); kept in `own`.
-      auto send = [&](int j, uint32_t (&own)[16]) -> bool {
-        const int slot = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        bool w = ptx::mbar_wait(&s_full[slot], par, kErrTimeoutMma);
-        if (!__all_sync(0xffffffffu, w)) return false;
-        ptx::tc_fence_after();
-        {
-          uint32_t a[32];
-          ptx::tmem_ld32(tmem + lane_base + kColS + slot * kTileN + 32 * g, a);
-          ptx::tmem_wait_ld();
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(&s_free[slot]);               // S buffer may take QK(j+2)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) own[i] = cvt_f16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
-        }
-        w = ptx::mbar_wait<true>(&xchg_free[slot], par, kErrTimeoutPeer);
-        // the outbox is free once the partner has received my previous copy
-        if (j >= 1) w = w && ptx::mbar_wait<true>(outbox_free, (j - 1) & 1, kErrTimeoutPeer);
-        if (!__all_sync(0xffffffffu, w)) return false;
-        uint8_t* dst = outbox + h * 128;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<uint4*>(dst + (((4 * g + k) ^ sw) << 4)) =
-              make_uint4(own[4 * k], own[4 * k + 1], own[4 * k + 2], own[4 * k + 3]);
-        ptx::fence_async_smem();
-        ptx::mbar_arrive(&outbox_ready[slot]);
-        if (threadIdx.x == 0) {
-          // every row is in the outbox (a bounded wait, unlike a named barrier) -> one bulk copy
-          if (ptx::mbar_wait(&outbox_ready[slot], par, kErrTimeoutSoftmax))
-            ptx::bulk_copy_to_peer(peer_inbox + slot * L::kXchgSlot, ptx::smem_u32(outbox), L::kXchgSlot,
-                                   slot ? peer_full1 : peer_full0);
-          ptx::mbar_arrive_expect_tx(&xchg_full[slot], L::kXchgSlot);
-        }
-        return true;
-      };
-
-      // Finish tile j: add the partner's partial, online softmax, P into shared memory.
-      auto finish = [&](int j, const uint32_t (&own)[16]) -> bool {
-        const int slot = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        bool w = ptx::mbar_wait<true>(&xchg_full[slot], par, kErrTimeoutPeer);
-        if (!__all_sync(0xffffffffu, w)) return false;
-        // raw scores: my fp16 partial + the partner's fp16 partial (packed fp16 adds)
-        uint32_t sum2[16];
-        {
-          const uint8_t* mine = inbox + slot * L::kXchgSlot + h * 128;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint4 v = *reinterpret_cast<const uint4*>(mine + (((4 * g + k) ^ sw) << 4));
-            const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __half2 a = *reinterpret_cast<const __half2*>(&own[4 * k + e]);
-              __half2 c = *reinterpret_cast<const __half2*>(&pv[e]);
-              __half2 r = __hadd2(a, c);
-              sum2[4 * k + e] = *reinterpret_cast<uint32_t*>(&r);
-            }
-          }
-        }
-        const int64_t key0 = j_begin + (int64_t)j * kTileN;
-        const int n_valid = (int)min64(kTileN, j_end - key0);
-        const int c0 = 32 * g;                           // first key column of this half
-        if (n_valid < kTileN) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            // keys past the end: -inf (fp16 0xFC00) in the masked half(s)
-            if (c0 + 2 * i >= n_valid) sum2[i] = 0xFC00FC00u;
-            else if (c0 + 2 * i + 1 >= n_valid) sum2[i] = (sum2[i] & 0x0000FFFFu) | 0xFC000000u;
-          }
-        }
-        float hm;
-        {
-          __half2 m4[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const __half2* v = reinterpret_cast<const __half2*>(&sum2[4 * i]);
-            m4[i] = __hmax2(__hmax2(v[0], v[1]), __hmax2(v[2], v[3]));
-          }
-          const __half2 m2 = __hmax2(__hmax2(m4[0], m4[1]), __hmax2(m4[2], m4[3]));
-          hm = fmaxf(__low2float(m2), __high2float(m2)) * sl2;   // scale >= 0
-        }
-        // the row max is the max of the two halves' maxima
-        half_max[(slot * 2 + g) * 128 + h] = hm;
-        ptx::mbar_arrive(&mx_bar[slot]);
-        w = ptx::mbar_wait(&mx_bar[slot], par, kErrTimeoutSoftmax);
-        if (!__all_sync(0xffffffffu, w)) return false;
-        const float mx = fmaxf(hm, half_max[(slot * 2 + (g ^ 1)) * 128 + h]);
-        // the P buffer and O are only touched once the P V product of tile j-1 is done
-        if (j >= 1) {
-          w = ptx::mbar_wait(o_done, (j - 1) & 1, kErrTimeoutMma);
-          if (!__all_sync(0xffffffffu, w)) return false;
-          ptx::tc_fence_after();
-        }
-        if (j == 0) {
-          m_ref = mx;
-        } else {
-          const bool grow = mx > m_ref + kRescaleThreshold;
-          // Both halves of a row see the same mx, so they agree on the rescale.
-          // TMEM loads/stores are warp-wide: the warp rescales together, lanes
-          // whose row max did not grow use factor 1.  Half g rescales O[:, 128g..].
-          if (__any_sync(0xffffffffu, grow)) {
-            const float f = grow ? fast_exp2(m_ref - mx) : 1.f;
-            l *= f;
-#pragma unroll 1
-            for (int c = 4 * g; c < 4 * g + 4; ++c) {
-              uint32_t r[32];
-              ptx::tmem_ld32(tmem + lane_base + kColO + c * 32, r);
-              ptx::tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-              ptx::tmem_st32(tmem + lane_base + kColO + c * 32, r);
-            }
-            ptx::tmem_wait_st();
-            if (grow) m_ref = mx;
-          }
-        }
-        // P = 2^(s*scale*log2e - m_ref) as bf16, keys 32g.. of row h of the K-major P tile (128-byte swizzle)
-        uint8_t* prow = p_s + h * 128;
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t q4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 xs = __half22float2(*reinterpret_cast<const __half2*>(&sum2[4 * k + e]));
-            float e0 = fast_exp2(fmaf(xs.x, sl2, -m_ref));
-            float e1 = fast_exp2(fmaf(xs.y, sl2, -m_ref));
-            if (n_valid < kTileN) {   // keys past the end weigh exactly 0 (also when scale is 0)
-              if (c0 + 8 * k + 2 * e >= n_valid) e0 = 0.f;
-              if (c0 + 8 * k + 2 * e + 1 >= n_valid) e1 = 0.f;
-            }
-            ps[e] += e0 + e1;
-            q4[e] = ptx::pack_bf16x2(e0, e1);
-          }
-          *reinterpret_cast<uint4*>(prow + (((4 * g + k) ^ sw) << 4)) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
-        }
-        l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-        if (n_valid < kTileN) {
-          // keys past the end get P = 0, but 0 * NaN is NaN: clear their latent rows
-          uint8_t* st = smem + (j % kStages) * L::kStage;
-          const int rows = kTileN - n_valid;
-          for (int idx = (int)threadIdx.x; idx < rows * 4 * 8; idx += kSoftmaxThreads) {
-            const int bx = idx / (rows * 8), rem = idx % (rows * 8);
-            *reinterpret_cast<uint4*>(st + bx * L::kKvBox + (n_valid + rem / 8) * 128 + (rem % 8) * 16) =
-                make_uint4(0, 0, 0, 0);
-          }
-        }
-        ptx::fence_async_smem();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&p_ready[slot]);
-        // my inbox slot is consumed: the partner may send tile j+2 into it
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_cluster_relaxed(&xchg_free[slot], peer);
-        return true;
-      };
-
-      uint32_t cur[16], nxt[16];
-      if (ok) ok = send(0, cur);
-      for (int j = 0; ok && j < nt; ++j) {
-        if (j + 1 < nt) {
-          ok = send(j + 1, nxt);
-          if (!ok) break;
-        }
-        ok = finish(j, cur);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) cur[i] = nxt[i];
-      }
-    }
-
-    // ---- epilogue ----------------------------------------------------------
-    // thread (g, h) writes latent columns 256*rank + 128g .. +127 of head h
-    const int64_t out_row = (row * p.heads + head) * 512 + 256 * rank + 128 * g;
-    if (nt == 0) {
-      if (p.num_splits == 1) {
-        uint4* dst = reinterpret_cast<uint4*>(p.o_lat + out_row);
-        for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
-      } else if (rank == 0 && g == 0) {
-        float* ml = p.part_ml + (((int64_t)sp * p.n_q + row) * p.heads + head) * 2;
-        ml[0] = -INFINITY;
-        ml[1] = 0.f;
-      }
-    } else if (ok) {
-      // the row sum is the sum of the two halves' sums
-      half_sum[g * 128 + h] = l;
-      ptx::mbar_arrive(l_bar);
-      bool w = ptx::mbar_wait(l_bar, 0, kErrTimeoutSoftmax) && ptx::mbar_wait(o_final, 0, kErrTimeoutMma);
-      if (__all_sync(0xffffffffu, w)) {
-        const float lsum = half_sum[h] + half_sum[128 + h];
-        ptx::tc_fence_after();
-        if (p.num_splits == 1) {
-          const float inv = 1.f / lsum;
-          uint4* dst = reinterpret_cast<uint4*>(p.o_lat + out_row);
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tmem + lane_base + kColO + (4 * g + c) * 32, r);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint32_t q4[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                q4[e] = ptx::pack_bf16x2(__uint_as_float(r[8 * v + 2 * e]) * inv,
-                                         __uint_as_float(r[8 * v + 2 * e + 1]) * inv);
-              dst[c * 4 + v] = make_uint4(q4[0], q4[1], q4[2], q4[3]);
-            }
-          }
-        } else {
-          const int64_t slot = ((int64_t)sp * p.n_q + row) * p.heads + head;
-          float4* dst = reinterpret_cast<float4*>(p.part_o + slot * 512 + 256 * rank + 128 * g);
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tmem + lane_base + kColO + (4 * g + c) * 32, r);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[c * 8 + v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                           __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-          }
-          if (rank == 0 && g == 0) {
-            p.part_ml[slot * 2] = m_ref;
-            p.part_ml[slot * 2 + 1] = lsum;
-          }
-        }
-      }
-    }
-  }
+  if (rank == 0)
+    score_role(smem, tmem, u, p, &tmap_kv_score, &tmap_pe, &tmap_qpe, &tmap_qabs);
+  else
+    value_role(smem, tmem, u, p, &tmap_kv_value, &tmap_out);
 
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, 512);
-  ptx::cluster_sync();   // the partner no longer writes into this CTA's shared memory
+  ptx::cluster_sync();   // neither CTA's shared memory goes away while the partner may still write into it
 }
 
-// Merge split partials: o = sum_s 2^{m_s - M} o_s / sum_s 2^{m_s - M} l_s, M = max_s m_s.
-// One block of 128 threads per (row, head); warp 0 turns the (m, l) pairs into
-// weights, then thread i accumulates columns 4i..4i+3 over the splits with
-// several loads in flight.  Splits with no key (m = -inf) get weight 0 and
-// their (unwritten) partial is never used.
+// Merge split partials: o = sum_s 2^{m_s - M} O_s / sum_s 2^{m_s - M} l_s, M = max_s m_s,
+// with O_s the bf16 partial of split s (relative to its reference m_s).
+// One block of 128 threads per (row, head); thread i owns columns 4i..4i+3.
+// Every thread starts loading its partial columns of (up to) the first 16
+// splits at once, while warp 0 turns the (m, l) pairs into weights, so the
+// two memory round trips overlap.  Splits with no key (m = -inf) get weight 0
+// and their (unwritten) partial is never used.
 constexpr int kMaxSplits = 256;
-__global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restrict__ part_o,
+constexpr int kMergeInFlight = 16;
+__global__ void __launch_bounds__(128) merge_splits_kernel(const __nv_bfloat16* __restrict__ part_o,
                                                            const float* __restrict__ part_ml, int num_splits,
                                                            int64_t n_q, int heads, __nv_bfloat16* __restrict__ o_lat) {
   __shared__ float s_w[kMaxSplits];
@@ -642,6 +761,12 @@ __global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restri
   const int head = blockIdx.y;
   const int64_t split_stride = n_q * heads;
   const int64_t base = row * heads + head;
+  const uint2* src = reinterpret_cast<const uint2*>(part_o + base * 512) + threadIdx.x;
+  const int64_t step = split_stride * 512 / 4;
+  uint2 v[kMergeInFlight];
+#pragma unroll
+  for (int s = 0; s < kMergeInFlight; ++s)
+    if (s < num_splits) v[s] = __ldcg(src + s * step);
   if (threadIdx.x < 32) {
     float M = -INFINITY;
     for (int s = threadIdx.x; s < num_splits; s += 32) M = fmaxf(M, part_ml[(s * split_stride + base) * 2]);
@@ -657,22 +782,23 @@ __global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restri
     if (threadIdx.x == 0) s_inv = L > 0.f ? 1.f / L : 0.f;
   }
   __syncthreads();
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float4* src = reinterpret_cast<const float4*>(part_o + base * 512) + threadIdx.x;
-  const int64_t step = split_stride * 512 / 4;
-#pragma unroll 8
-  for (int s = 0; s < num_splits; ++s) {
-    const float w = s_w[s];
-    const float4 v = src[s * step];
-    if (w != 0.f) {
-      acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
-    }
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  auto acc = [&](float w, uint2 x) {
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
+    a0 = fmaf(w, lo.x, a0); a1 = fmaf(w, lo.y, a1); a2 = fmaf(w, hi.x, a2); a3 = fmaf(w, hi.y, a3);
+  };
+#pragma unroll
+  for (int s = 0; s < kMergeInFlight; ++s)
+    if (s < num_splits && s_w[s] != 0.f) acc(s_w[s], v[s]);
+  for (int s = kMergeInFlight; s < num_splits; ++s) {
+    const uint2 x = __ldcg(src + s * step);
+    if (s_w[s] != 0.f) acc(s_w[s], x);
   }
   const float inv = s_inv;
   uint2 o;
-  o.x = ptx::pack_bf16x2(acc.x * inv, acc.y * inv);
-  o.y = ptx::pack_bf16x2(acc.z * inv, acc.w * inv);
+  o.x = ptx::pack_bf16x2(a0 * inv, a1 * inv);
+  o.y = ptx::pack_bf16x2(a2 * inv, a3 * inv);
   reinterpret_cast<uint2*>(o_lat + base * 512)[threadIdx.x] = o;
 }
 

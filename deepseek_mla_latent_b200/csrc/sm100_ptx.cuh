@@ -76,6 +76,10 @@ __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint64_t* bar, uint3
       "r"(rank)
       : "memory");
 }
+// The same, given the partner's barrier as a shared::cluster address (from map_peer).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed_addr(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -280,6 +284,52 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, ui
       "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
       "r"(src), "r"(bytes), "r"(bar)
       : "memory");
+}
+// 32-bit store into another CTA's shared memory; completion is counted in
+// bytes (4) on that CTA's mbarrier (both addresses from map_peer).
+__device__ __forceinline__ void st_async_b32(uint32_t remote_addr, uint32_t remote_bar, uint32_t v) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %2, [%1];" ::"r"(remote_addr),
+               "r"(remote_bar), "r"(v)
+               : "memory");
+}
+// Start pulling `bytes` (multiple of 16, 16-byte aligned address) of global
+// memory into L2; nothing waits for it.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+// TMA tensor store of one box from this CTA's shared memory (bulk async-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed bulk groups of this thread still read their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until every committed bulk group of this thread has completed (writes performed).
+__device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Plain stores into another CTA's shared memory (address from map_peer).
+__device__ __forceinline__ void st_cluster_v4(uint32_t remote_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(remote_addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_b32(uint32_t remote_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(remote_addr), "r"(v) : "memory");
+}
+// Order this thread's generic-proxy writes to cluster shared memory before
+// later async-proxy reads of it (a tensor-core operand in the receiving CTA).
+__device__ __forceinline__ void fence_async_smem_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+// Release-arrive on a barrier given as a shared::cluster address (from map_peer).
+__device__ __forceinline__ void mbar_arrive_cluster_addr(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
 // Make this thread's generic-proxy shared-memory writes visible to async-proxy readers (TMA, bulk copy, MMA).
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
