@@ -9,8 +9,10 @@ One step = the whole hot path on one batch: mla_absorb_q -> mla_attn_decode
 
 Prints one JSON line.  `value` is microseconds per step (lower is better),
 the max over ranks; with N > 1 every rank runs an independent replica (the
-path has no cross-GPU exchange).  L2 is flushed (a 256 MiB write) before every
-timed step, outside the timed events.  `--impl reference` times the fp64 CPU
+path has no cross-GPU exchange).  L2 is flushed before every timed step, outside
+the timed events: a 256 MiB write followed by a 256 MiB read, so
+each timed step starts with none of its inputs in L2 and no dirty lines left
+to write back.  `--impl reference` times the fp64 CPU
 oracle on the host cores instead, one (sequence, head) pair per step.
 """
 from __future__ import annotations
@@ -236,7 +238,15 @@ def main():
             "out": torch.empty((B, H, Dv), dtype=dt, device=dev),
             "ws": mla.workspace(d, B, B, max_k, 0, device=dev)}
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_read = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+    flush_sum = torch.empty((), dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        # evict every input (write a buffer larger than L2), then read another one so the
+        # dirty lines of that write are written back before the timed region starts
+        flush.zero_()
+        torch.sum(flush_read, dim=0, out=flush_sum)
 
     def step():
         # the whole hot path through the public calls: absorb -> attention (+ merge) -> output projection
@@ -248,7 +258,7 @@ def main():
         mla.attn_decode(d, bufs["q_abs"], q, kv, pe, cu_k, max_k, bufs["o_lat"], bufs["ws"])
 
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush_l2()
         step()
     mla.device_status()
 
@@ -267,9 +277,9 @@ def main():
 
     g_step, g_attn = capture(step), capture(attention_call)
     for _ in range(3):
-        flush.zero_()
+        flush_l2()
         g_step.replay()
-        flush.zero_()
+        flush_l2()
         g_attn.replay()
     mla.device_status()
 
@@ -293,7 +303,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
-        flush.zero_()                     # L2 flush, outside the timed events
+        flush_l2()                        # L2 flush, outside the timed events
         ev_s[i].record(stream)
         g_step.replay()
         ev_e[i].record(stream)
@@ -302,7 +312,7 @@ def main():
         dist.barrier()
     # the attention call alone (its kernel + split merge), for the roofline figure
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2()
         ev_as[i].record(stream)
         g_attn.replay()
         ev_ae[i].record(stream)
@@ -323,7 +333,7 @@ def main():
     e2e_s = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
     e2e_e = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
     for i in range(e2e_steps):
-        flush.zero_()
+        flush_l2()
         e2e_s[i].record(stream)
         q_dev.copy_(q_pinned, non_blocking=True)
         q_abs = mla.absorb_q(d, q_dev, wkv_b, bufs["q_abs"])
@@ -349,7 +359,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32", "data": "synthetic",
             "config": {"workload": w.name, "batch": B, "heads": H, "kv_lora_rank": C, "qk_rope": w.dims.qk_rope,
                        "seq_len_k": max_k, "queries_per_seq": 1, "parallelism": "replicas" if world > 1 else "single",
-                       "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+                       "l2": "flushed before every timed step (256 MiB write then 256 MiB read, outside the events)"},
             "tokens_per_s": world * B / (us_step / 1e6),
             "attn_kernel_us": mean_attn_ms * 1e3,
             "attn_cache_gbs": achieved_gbs,

@@ -187,7 +187,7 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   if (units == 0) return MLA_OK;
   if (2 * units >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
   if ((uint64_t)n_q * H * (uint64_t)splits >= (1ULL << 31)) return MLA_ERR_INVALID_ARG;
-  CUtensorMap tkv_s, tpe, tqpe, tkv_v, tout;
+  CUtensorMap tkv_s, tpe, tqpe, tkv_v;
   // kv_rows may be 0 (every sequence empty); the maps still need one row.
   const uint64_t rows = kv_rows > 0 ? (uint64_t)kv_rows : 1;
   const void* kv_base = kv_rows > 0 ? kv : q_abs;   // any valid 16-byte aligned address for an unused map
@@ -237,17 +237,10 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
     part_o = static_cast<__nv_bfloat16*>(ws);
     p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)splits * n_q * H * 512 * 2));
   }
-  {
-    // the epilogue's output, [rows, 512] bf16 in boxes of 64 columns x 32 rows: the split
-    // partials [splits * n_q * H, 512], or o_lat [n_q * H, 512] directly
-    const uint64_t d[2] = {512, (uint64_t)(splits > 1 ? splits : 1) * n_q * H}, st[1] = {1024};
-    const uint32_t b[2] = {64, 32};
-    if (!make_map(&tout, splits > 1 ? (void*)part_o : o_lat, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B))
-      return MLA_ERR_CUDA;
-  }
+  p.out = splits > 1 ? part_o : static_cast<__nv_bfloat16*>(o_lat);
   if (!set_smem(latent_attn_kernel, kAttnSmem)) return MLA_ERR_CUDA;
   mla_status_t st = launch(true, latent_attn_kernel, dim3((unsigned)(2 * units)), dim3(kAttnThreads), kAttnSmem,
-                           stream, tkv_s, tpe, tqpe, tkv_v, tout, tqa, p);
+                           stream, tkv_s, tpe, tqpe, tkv_v, tqa, p);
   if (st != MLA_OK || splits <= 1) return st;
   return launch(true, merge_splits_kernel, dim3((unsigned)n_q, H), dim3(128), 0, stream,
                 (const __nv_bfloat16*)part_o, (const float*)p.part_ml, splits, n_q, H,

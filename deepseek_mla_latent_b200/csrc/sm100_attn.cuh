@@ -19,9 +19,9 @@
 //     sent to the value CTA with one bulk copy per warp.
 //   value CTA (rank 1): O in TMEM, O += P V (8 tcgen05.mma with N = 256 per
 //     64 keys, A = P and B = the kv tile, both from shared memory), the rare O
-//     rescale, and the epilogue (TMA stores of O or of the split partial).
+//     rescale, and the epilogue (O or the split partial as bf16).
 //
-// The score CTA never waits for the value CTA except for a free P slot (two
+// The score CTA never waits for the value CTA except for a free P slot (four
 // slots), so the pair forms a pipeline instead of exchanging partial scores
 // every tile.  Each CTA streams its own copy of the kv rows: the score CTA
 // from HBM (it also prefetches its key range into L2), the value CTA a little
@@ -42,9 +42,10 @@
 // P <= 256.  When it moves, the factor 2^(m_old - m_new) travels with P and
 // the value CTA rescales O before the next P V product.
 //
-// Value CTA.  TMEM: O, all 512 columns.  Shared memory: a 3-stage ring of
-// 64-key kv tiles (eight 8 KB boxes) and two P slots (P 16 KB, the per-row
-// factor, and in slot 0 the final row sums).  Warps 0-3 check each tile's
+// Value CTA.  TMEM: O, all 512 columns.  Shared memory: a 2-stage ring of
+// 64-key kv tiles (eight 8 KB boxes; they hit L2, the score CTA read the rows
+// first) and four P slots (P 16 KB, the per-row factor, and in slot 0 the
+// final row sums).  Warps 0-3 check each tile's
 // factors (and rescale O when one moved), zero the tail rows of the last
 // tile's values, and release the P V product; warp 8 loads, warp 9 issues
 // the MMAs and hands P slots back; warps 0-7 run the epilogue.
@@ -85,13 +86,14 @@ struct ScoreLayout {
 struct ValueLayout {
   static constexpr int kKvBox = kTileN * 128;              // 64 keys x 64 latent columns bf16
   static constexpr int kStage = 8 * kKvBox;                // 64 keys x 512 latent columns
-  static constexpr int kStages = 3;
-  static constexpr int kOffSlots = kStages * kStage;       // two P slots
+  static constexpr int kStages = 2;
+  static constexpr int kPSlots = 4;
+  static constexpr int kOffSlots = kStages * kStage;       // P slots
   static constexpr int kSlot = 17408;                      // 1024-aligned
   static constexpr int kP = 128 * kTileN * 2;              // P: 128 heads x 64 keys bf16, 16 KB
   static constexpr int kOffF = kP;                         // in a slot: the per-row factors, 512 B
   static constexpr int kOffL = kOffSlots + kP + 512;       // in slot 0: the final row sums, 512 B
-  static constexpr int kOffBars = kOffSlots + 2 * kSlot;
+  static constexpr int kOffBars = kOffSlots + kPSlots * kSlot;
   static constexpr int kBytes = kOffBars + 512;
 };
 
@@ -116,7 +118,8 @@ struct AttnParams {
   int64_t kv_rows;
   int64_t n_q;
   float scale_log2;             // softmax_scale * log2(e)
-  __nv_bfloat16* o_lat;         // [n_q, H, 512]; plain stores only for units with no key
+  __nv_bfloat16* o_lat;         // [n_q, H, 512]
+  __nv_bfloat16* out;           // the epilogue's rows of 512: o_lat, or the split partials [splits * n_q * H, 512]
   float* part_ml;               // [splits, n_q, H, 2] = (reference max in log2 units, row sum)
 };
 
@@ -160,11 +163,11 @@ __device__ __forceinline__ UnitRange unit_range(const AttnParams& p, int64_t uni
 // Barrier slots (8 bytes each) in the 512-byte barrier area of either role.
 namespace bar {
 // score CTA
-constexpr int kUFull = 0, kUEmpty = 13, kSFull = 26, kSFree = 28, kMBar = 30, kPFree = 32, kQFull = 34,
-              kQReady = 35, kEnd = 36, kScoreIdle = 37, kPSent = 38;
+constexpr int kUFull = 0, kUEmpty = 11, kSFull = 22, kSFree = 24, kMBar = 26, kPFree = 28, kQFull = 32,
+              kQReady = 33, kEnd = 34, kScoreIdle = 35, kPSent = 36, kStgFree = 38;
 // value CTA
-constexpr int kVFull = 0, kVEmpty = 3, kPFull = 6, kPvGo = 8, kPDone = 10, kOFinal = 12, kLFull = 13,
-              kValueIdle = 14;
+constexpr int kVFull = 0, kVEmpty = 2, kPFull = 4, kPvGo = 8, kPDone = 12, kOFinal = 16, kLFull = 17,
+              kValueIdle = 18;
 constexpr int kTmemSlot = 63;
 }  // namespace bar
 
@@ -181,7 +184,8 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
   uint64_t* s_full = bars + bar::kSFull;       // [2] QK product committed
   uint64_t* s_free = bars + bar::kSFree;       // [2] S read out (128 arrivals)
   uint64_t* m_bar = bars + bar::kMBar;         // [2] warpgroup g published the reference max of its tile (128)
-  uint64_t* p_free = bars + bar::kPFree;       // [2] the value CTA finished the P V product of this P slot
+  uint64_t* p_free = bars + bar::kPFree;       // [4] the value CTA finished the P V product of this P slot
+  uint64_t* stg_free = bars + bar::kStgFree;   // [2] the P tile in this staging slot landed in the value CTA
   uint64_t* q_full = bars + bar::kQFull;       // q_abs and q_pe landed
   uint64_t* q_ready = bars + bar::kQReady;     // q_abs in TMEM, its landing zone free (256 arrivals)
   uint64_t* end_bar = bars + bar::kEnd;        // warpgroup 1 published its (l, m) (128)
@@ -234,7 +238,6 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
             ptx::tma_load_2d(smem + slot * L::kUnit, tmap_kv, &u_full[slot], 64 * cb, key);
           else
             ptx::tma_load_2d(smem + slot * L::kUnit, tmap_pe, &u_full[slot], 0, key);
-          // once the ring is full, keep the next few tiles streaming into L2
           // keep the score tile kPrefetchTiles ahead streaming into L2
           if (kPrefetchTiles > 0 && cb == 0 && jj + kPrefetchTiles < ntq) prefetch_tile(jj + kPrefetchTiles);
         }
@@ -319,6 +322,7 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
     float m_used = -INFINITY, l = 0.f;   // reference this warpgroup last used, and its row sum relative to it
     if (ntp > 0) {
       // q_abs row h, latent block b (columns 64b..) -> TMEM columns 32b.. (bf16 pairs); warpgroup g moves blocks 4g..4g+3
+      const uint32_t v_base = ptx::map_peer(ptx::smem_u32(smem), 1);
       ok = __all_sync(0xffffffffu, ptx::mbar_wait(q_full, 0, kErrTimeoutTmaFull));
       if (ok) {
 #pragma unroll 1
@@ -336,7 +340,6 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
         ptx::tc_fence_before();
       }
       ptx::mbar_arrive(q_ready);
-      const uint32_t v_base = ptx::map_peer(ptx::smem_u32(smem), 1);
 
       for (int jj = g; ok && jj < ntq; jj += 2) {
         const int sb = jj & 1;
@@ -345,13 +348,11 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
         ptx::tc_fence_after();
         uint32_t s[128];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t a[32];
-          ptx::tmem_ld32(tmem + lane_base + kColS + sb * kTileQ + 32 * c, a);
-          ptx::tmem_wait_ld();
+        for (int c = 0; c < 4; ++c)
+          ptx::tmem_ld32(tmem + lane_base + kColS + sb * kTileQ + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
+        ptx::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) s[32 * c + i] = a[i];
-        }
+        for (int c = 0; c < 4; ++c) ptx::reg_fence32(&s[32 * c]);
         ptx::tc_fence_before();
         ptx::mbar_arrive(&s_free[sb]);                 // S buffer may take QK(jj+2)
         const int n_valid = (int)min64(kTileQ, u.j_end - (u.j_begin + (int64_t)jj * kTileQ));
@@ -382,23 +383,11 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
           l = m_used == -INFINITY ? 0.f : l * fast_exp2(m_used - m_new);
           m_used = m_new;
         }
-        // P tiles reach the value CTA's two slots strictly in order: the other warpgroup
-        // stored those of score tile jj-1 first.  (It hands over the reference max before
-        // its P, so without this a warpgroup could wait on a P slot barrier two phases
-        // ahead, which a parity wait cannot tell from the phase before.)
-        if (jj > 0) {
-          w = ptx::mbar_wait(&p_sent[g ^ 1], ((jj - 1) >> 1) & 1, kErrTimeoutSoftmax);
-          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        }
         // P = 2^(s * scale * log2(e) - m) as bf16, in two 64-key P tiles; keys past the end weigh exactly 0
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (kTileN * half >= n_valid) break;
-          const int t = 2 * jj + half, ps = t & 1;
-          if (t >= 2) {
-            w = ptx::mbar_wait<true>(&p_free[ps], ((t - 2) >> 1) & 1, kErrTimeoutPeer);
-            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-          }
+          const int t = 2 * jj + half, ps = t & 1, vs = t & 3;
           uint32_t pk[32];
           float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
@@ -413,6 +402,16 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
             pk[i] = ptx::pack_bf16x2(e0, e1);
           }
           l += ps0 + ps1;
+          // P tiles reach the value CTA's slots strictly in order: the other warpgroup stored
+          // those of score tile jj-1 first.  (It hands over the reference max before its P, so
+          // without this a warpgroup could wait on a P slot barrier two phases ahead, which a
+          // parity wait cannot tell from the phase before.)  Then staging slot ps is free once
+          // P tile t-2 landed in the value CTA, and its P slot vs once P V of tile t-4 finished.
+          w = true;
+          if (half == 0 && jj > 0) w = ptx::mbar_wait(&p_sent[g ^ 1], ((jj - 1) >> 1) & 1, kErrTimeoutSoftmax);
+          if (t >= 2) w = w && ptx::mbar_wait<true>(&stg_free[ps], ((t - 2) >> 1) & 1, kErrTimeoutPeer);
+          if (t >= 4) w = w && ptx::mbar_wait<true>(&p_free[vs], ((t - 4) >> 2) & 1, kErrTimeoutPeer);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           // row h of the K-major P tile (128-byte swizzle) and the row's factor into staging slot ps,
           // then this warp's 32 rows and factors to the value CTA's P slot ps (two bulk copies)
           uint8_t* stg = smem + L::kOffStaging + ps * L::kSlot;
@@ -424,8 +423,8 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
           ptx::fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            const uint32_t dst = v_base + ValueLayout::kOffSlots + (uint32_t)ps * ValueLayout::kSlot;
-            const uint32_t vbar = v_base + ValueLayout::kOffBars + 8 * (bar::kPFull + ps);
+            const uint32_t dst = v_base + ValueLayout::kOffSlots + (uint32_t)vs * ValueLayout::kSlot;
+            const uint32_t vbar = v_base + ValueLayout::kOffBars + 8 * (bar::kPFull + vs);
             ptx::bulk_copy_to_peer(dst + qd * 4096, ptx::smem_u32(stg) + qd * 4096, 4096, vbar);
             ptx::bulk_copy_to_peer(dst + ValueLayout::kOffF + qd * 128, ptx::smem_u32(stg) + ValueLayout::kOffF + qd * 128,
                                    128, vbar);
@@ -463,14 +462,14 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
 
 // ---------------------------------------------------------------- value CTA
 __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const UnitRange& u, const AttnParams& p,
-                                           const CUtensorMap* tmap_kv, const CUtensorMap* tmap_out) {
+                                           const CUtensorMap* tmap_kv) {
   using L = ValueLayout;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBars);
-  uint64_t* v_full = bars + bar::kVFull;      // [3] kv tile landed
-  uint64_t* v_empty = bars + bar::kVEmpty;    // [3] kv tile read by the tensor core
-  uint64_t* p_full = bars + bar::kPFull;      // [2] P and factors of a tile landed (bulk copies from the score CTA)
-  uint64_t* pv_go = bars + bar::kPvGo;        // [2] factors applied, tail cleared: P V may run (128 arrivals)
-  uint64_t* p_done = bars + bar::kPDone;      // [2] P V product of this slot finished
+  uint64_t* v_full = bars + bar::kVFull;      // [2] kv tile landed
+  uint64_t* v_empty = bars + bar::kVEmpty;    // [2] kv tile read by the tensor core
+  uint64_t* p_full = bars + bar::kPFull;      // [4] P and factors of a tile landed (bulk copies from the score CTA)
+  uint64_t* pv_go = bars + bar::kPvGo;        // [4] factors applied, tail cleared: P V may run (128 arrivals)
+  uint64_t* p_done = bars + bar::kPDone;      // [4] P V product of this slot finished
   uint64_t* o_final = bars + bar::kOFinal;    // the last P V product finished
   uint64_t* l_full = bars + bar::kLFull;      // the row sums landed
   uint64_t* idle = bars + bar::kValueIdle;
@@ -484,7 +483,10 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
     if (nt > 0) {
       if (ptx::elect_one()) ptx::prefetch_tmap(tmap_kv);
       __syncwarp();
-      for (int j = 0; j < nt; ++j) {
+      // The first P tile arrives several microseconds in; loading values before then would only
+      // add to the start-up burst on HBM (these rows reach L2 through the score CTA meanwhile).
+      bool w0 = ptx::mbar_wait<true>(&p_full[0], 0, kErrTimeoutPeer);
+      for (int j = 0; w0 && j < nt; ++j) {
         const int st = j % L::kStages;
         const bool w = ptx::mbar_wait(&v_empty[st], ((j / L::kStages) & 1) ^ 1, kErrTimeoutStageFree);
         if (!__all_sync(0xffffffffu, w)) break;
@@ -512,24 +514,25 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
       const uint64_t d_p0 = ptx::smem_desc(ptx::smem_u32(smem + L::kOffSlots), 16, 1024, ptx::kSwizzle128);
       const uint64_t d_v0 = ptx::smem_desc(ptx::smem_u32(smem), L::kKvBox, 1024, ptx::kSwizzle128);
       const uint32_t score_free0 = ptx::map_peer(ptx::smem_u32(smem + ScoreLayout::kOffBars + 8 * bar::kPFree), 0);
+      constexpr int kS = L::kPSlots;
       bool ok = true;
       int pv = 0, fw = 0;
       uint64_t t_last = global_timer_ns();
-      while (ok && (pv < nt || fw < nt - 2)) {
+      while (ok && (pv < nt || fw < nt - kS)) {
         bool progressed = false;
-        bool go = fw < nt - 2 && fw < pv && ptx::mbar_test(&p_done[fw & 1], (fw >> 1) & 1);
+        bool go = fw < nt - kS && fw < pv && ptx::mbar_test(&p_done[fw % kS], (fw / kS) & 1);
         if (__shfl_sync(0xffffffffu, go, 0)) {
-          if (lane == 0) ptx::mbar_arrive_cluster_relaxed_addr(score_free0 + 8 * (fw & 1));
+          if (lane == 0) ptx::mbar_arrive_cluster_relaxed_addr(score_free0 + 8 * (fw % kS));
           __syncwarp();
           ++fw;
           progressed = true;
         }
         go = pv < nt && ptx::mbar_test(&v_full[pv % L::kStages], (pv / L::kStages) & 1) &&
-             ptx::mbar_test(&pv_go[pv & 1], (pv >> 1) & 1);
+             ptx::mbar_test(&pv_go[pv % kS], (pv / kS) & 1);
         if (__shfl_sync(0xffffffffu, go, 0)) {
           ptx::tc_fence_after();
           const uint32_t so = (uint32_t)((pv % L::kStages) * L::kStage) >> 4;
-          const uint32_t po = (uint32_t)((pv & 1) * L::kSlot) >> 4;
+          const uint32_t po = (uint32_t)((pv % kS) * L::kSlot) >> 4;
 #pragma unroll
           for (int n = 0; n < 2; ++n)
 #pragma unroll
@@ -542,7 +545,7 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
             }
           if (ptx::elect_one()) {
             ptx::mma_commit(&v_empty[pv % L::kStages]);
-            ptx::mma_commit(&p_done[pv & 1]);
+            ptx::mma_commit(&p_done[pv % kS]);
             if (pv == nt - 1) ptx::mma_commit(o_final);
           }
           __syncwarp();
@@ -574,15 +577,19 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
     if (nt > 0 && warp < 4) {
       // per tile: apply the row factors to O (rare), clear the tail rows, release P V
       if (threadIdx.x == 0) ptx::mbar_arrive_expect_tx(l_full, 512);
+      constexpr int kS = L::kPSlots;
+      const uint32_t score_stg0 = ptx::map_peer(ptx::smem_u32(smem + ScoreLayout::kOffBars + 8 * bar::kStgFree), 0);
       for (int j = 0; j < nt; ++j) {
-        const int s = j & 1;
+        const int s = j % kS;
         if (threadIdx.x == 0) ptx::mbar_arrive_expect_tx(&p_full[s], L::kP + 512);   // 4 x (4 KB + 128 B)
-        bool w = ptx::mbar_wait<true>(&p_full[s], (j >> 1) & 1, kErrTimeoutPeer);
+        bool w = ptx::mbar_wait<true>(&p_full[s], (j / kS) & 1, kErrTimeoutPeer);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        // the score CTA may refill the staging slot this tile came from (only tiles it still waits on)
+        if (threadIdx.x == 0 && j < nt - 2) ptx::mbar_arrive_cluster_relaxed_addr(score_stg0 + 8 * (j & 1));
         const float f = reinterpret_cast<const float*>(smem + L::kOffSlots + s * L::kSlot + L::kOffF)[h];
         if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
           // O holds the products of tiles < j relative to the old reference: scale it
-          w = ptx::mbar_wait(&p_done[(j - 1) & 1], ((j - 1) >> 1) & 1, kErrTimeoutMma);
+          w = ptx::mbar_wait(&p_done[(j - 1) % kS], ((j - 1) / kS) & 1, kErrTimeoutMma);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           ptx::tc_fence_after();
 #pragma unroll 1
@@ -628,37 +635,44 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
       w = w && ptx::mbar_wait<true>(l_full, 0, kErrTimeoutPeer);   // also before exit: it writes here
       if (__all_sync(0xffffffffu, w)) {
         ptx::tc_fence_after();
-        uint8_t* stage = smem + warp * 16384;   // the kv ring is idle now: four 4 KB store boxes per warp
+        uint8_t* buf = smem + warp * 8192;   // the kv ring is idle now: two 32-row x 128-byte tiles per warp
         const float inv = p.num_splits > 1 ? 1.f : 1.f / reinterpret_cast<const float*>(smem + L::kOffL)[h];
-        const int64_t row0 = p.num_splits > 1 ? ((int64_t)u.sp * p.n_q + u.row) * p.heads : u.row * p.heads;
-        const int y = (int)(row0 + u.hg * 128 + 32 * qd);
+        const int64_t row0 = (p.num_splits > 1 ? ((int64_t)u.sp * p.n_q + u.row) * p.heads : u.row * p.heads) +
+                             u.hg * 128 + 32 * qd;
 #pragma unroll 1
-        for (int k = 0; k < 4; ++k) {
-          uint8_t* buf = stage + k * 4096;
-          uint32_t r[32], r2[32];
-          ptx::tmem_ld32(tmem + lane_base + 256 * c + 64 * k, r);
-          ptx::tmem_ld32(tmem + lane_base + 256 * c + 64 * k + 32, r2);
+        for (int kk = 0; kk < 2; ++kk) {
+          // 128 columns per TMEM round trip (the loads' latency is the epilogue's cost)
+          uint32_t r[128];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            ptx::tmem_ld32(tmem + lane_base + 256 * c + 128 * kk + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * i]));
           ptx::tmem_wait_ld();
-          uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            pk[i] = ptx::pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-            pk[16 + i] = ptx::pack_bf16x2(__uint_as_float(r2[2 * i]) * inv, __uint_as_float(r2[2 * i + 1]) * inv);
-          }
-          // a 32-row x 128-byte box with 128-byte swizzle
+          for (int i = 0; i < 4; ++i) ptx::reg_fence32(&r[32 * i]);
+          __syncwarp();   // the previous pieces were read out of buf
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            *reinterpret_cast<uint4*>(buf + lane * 128 + ((v ^ (lane & 7)) << 4)) =
-                make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-          ptx::fence_async_smem();
+          for (int k2 = 0; k2 < 2; ++k2)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const uint32_t* x = &r[64 * k2 + 8 * v];
+              *reinterpret_cast<uint4*>(buf + k2 * 4096 + lane * 128 + ((v ^ (lane & 7)) << 4)) =
+                  make_uint4(ptx::pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
+                             ptx::pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
+                             ptx::pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
+                             ptx::pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
+            }
           __syncwarp();
-          if (lane == 0) {
-            ptx::tma_store_2d(tmap_out, buf, 256 * c + 64 * k, y);
-            ptx::bulk_commit_group();
-          }
+          // transposed read-back: each store instruction writes four whole 128-byte row pieces
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int rr = 4 * i + (int)(lane >> 3), ch = (int)(lane & 7);
+              const uint4 x = *reinterpret_cast<const uint4*>(buf + k2 * 4096 + rr * 128 + ((ch ^ (rr & 7)) << 4));
+              *reinterpret_cast<uint4*>(p.out + (row0 + rr) * 512 + 256 * c + 128 * kk + 64 * k2 + 8 * ch) = x;
+            }
         }
-        if (lane == 0) ptx::bulk_wait_group_all();
-        __syncwarp();
+
       }
     }
   }
@@ -669,8 +683,7 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tmap_kv_score, const __grid_constant__ CUtensorMap tmap_pe,
                        const __grid_constant__ CUtensorMap tmap_qpe, const __grid_constant__ CUtensorMap tmap_kv_value,
-                       const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ CUtensorMap tmap_qabs,
-                       const AttnParams p) {
+                       const __grid_constant__ CUtensorMap tmap_qabs, const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t warp = ptx::warp_id();
   const uint32_t rank = ptx::cluster_rank();
@@ -689,9 +702,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         ptx::mbar_init(&bars[bar::kSFull + s], 1);
         ptx::mbar_init(&bars[bar::kSFree + s], 128);
         ptx::mbar_init(&bars[bar::kMBar + s], 128);
-        ptx::mbar_init(&bars[bar::kPFree + s], 1);
         ptx::mbar_init(&bars[bar::kPSent + s], 4);
+        ptx::mbar_init(&bars[bar::kStgFree + s], 1);
       }
+      for (int s = 0; s < ValueLayout::kPSlots; ++s) ptx::mbar_init(&bars[bar::kPFree + s], 1);
       ptx::mbar_init(&bars[bar::kQFull], 1);
       ptx::mbar_init(&bars[bar::kQReady], 256);
       ptx::mbar_init(&bars[bar::kEnd], 128);
@@ -701,7 +715,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         ptx::mbar_init(&bars[bar::kVFull + s], 1);
         ptx::mbar_init(&bars[bar::kVEmpty + s], 1);
       }
-      for (int s = 0; s < 2; ++s) {
+      for (int s = 0; s < ValueLayout::kPSlots; ++s) {
         ptx::mbar_init(&bars[bar::kPFull + s], 1);
         ptx::mbar_init(&bars[bar::kPvGo + s], 128);
         ptx::mbar_init(&bars[bar::kPDone + s], 1);
@@ -733,7 +747,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   if (rank == 0)
     score_role(smem, tmem, u, p, &tmap_kv_score, &tmap_pe, &tmap_qpe, &tmap_qabs);
   else
-    value_role(smem, tmem, u, p, &tmap_kv_value, &tmap_out);
+    value_role(smem, tmem, u, p, &tmap_kv_value);
 
   ptx::tc_fence_before();
   __syncthreads();

@@ -331,6 +331,21 @@ __device__ __forceinline__ void fence_async_smem_cluster() {
 __device__ __forceinline__ void mbar_arrive_cluster_addr(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
+// 16-byte load from another CTA's shared memory (address from map_peer).
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t remote_addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(remote_addr) : "memory");
+  return v;
+}
+// Pin 32 registers filled by tcgen05.ld: the compiler must not read them before the
+// tcgen05.wait::ld that precedes this (it emits no instruction).
+__device__ __forceinline__ void reg_fence32(uint32_t* r) {
+  asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+               "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+               "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+               "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
 // Make this thread's generic-proxy shared-memory writes visible to async-proxy readers (TMA, bulk copy, MMA).
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // Named barrier over `count` threads (id 0 is __syncthreads).
