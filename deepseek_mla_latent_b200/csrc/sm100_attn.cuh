@@ -346,25 +346,33 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
         bool w = ptx::mbar_wait(&s_full[sb], (jj >> 1) & 1, kErrTimeoutMma);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         ptx::tc_fence_after();
-        uint32_t s[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          ptx::tmem_ld32(tmem + lane_base + kColS + sb * kTileQ + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::reg_fence32(&s[32 * c]);
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&s_free[sb]);                 // S buffer may take QK(jj+2)
+        const uint32_t s_col = tmem + lane_base + kColS + sb * kTileQ;
         const int n_valid = (int)min64(kTileQ, u.j_end - (u.j_begin + (int64_t)jj * kTileQ));
-        // row max of the raw scores over the valid keys (scale >= 0 commutes with max)
+        // row max of the raw scores over the valid keys (scale >= 0 commutes with max); S stays in
+        // TMEM and is read 64 columns at a time, here and again for the exponentials, so few
+        // registers are live and the exponentials of a row can be issued back to back
         float mx;
         {
           float m8[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
+#pragma unroll 1
+          for (int c2 = 0; c2 < 2; ++c2) {
+            uint32_t a[64];
+            ptx::tmem_ld32(s_col + 64 * c2, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+            ptx::tmem_ld32(s_col + 64 * c2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+            ptx::tmem_wait_ld();
+            ptx::reg_fence32(&a[0]);
+            ptx::reg_fence32(&a[32]);
+            if (n_valid >= 64 * (c2 + 1)) {
 #pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i < n_valid) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(s[i]));
+              for (int i = 0; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(a[i]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 64; ++i)
+                if (64 * c2 + i < n_valid) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(a[i]));
+            }
+          }
           mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
           mx *= sl2;
         }
@@ -390,16 +398,40 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
           const int t = 2 * jj + half, ps = t & 1, vs = t & 3;
           uint32_t pk[32];
           float ps0 = 0.f, ps1 = 0.f;
+          {
+            uint32_t a[64];
+            ptx::tmem_ld32(s_col + kTileN * half, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+            ptx::tmem_ld32(s_col + kTileN * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+            ptx::tmem_wait_ld();
+            ptx::reg_fence32(&a[0]);
+            ptx::reg_fence32(&a[32]);
+            if (half == 1 || kTileN >= n_valid) {
+              // the last read of this S buffer: QK(jj+2) may overwrite it
+              ptx::tc_fence_before();
+              ptx::mbar_arrive(&s_free[sb]);
+            }
+            if (kTileN * (half + 1) <= n_valid) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int k = kTileN * half + 2 * i;
-            float e0 = fast_exp2(fmaf(__uint_as_float(s[k]), sl2, -m_new));
-            float e1 = fast_exp2(fmaf(__uint_as_float(s[k + 1]), sl2, -m_new));
-            if (k >= n_valid) e0 = 0.f;
-            if (k + 1 >= n_valid) e1 = 0.f;
-            ps0 += e0;
-            ps1 += e1;
-            pk[i] = ptx::pack_bf16x2(e0, e1);
+              for (int i = 0; i < 32; ++i) {
+                const float e0 = fast_exp2(fmaf(__uint_as_float(a[2 * i]), sl2, -m_new));
+                const float e1 = fast_exp2(fmaf(__uint_as_float(a[2 * i + 1]), sl2, -m_new));
+                ps0 += e0;
+                ps1 += e1;
+                pk[i] = ptx::pack_bf16x2(e0, e1);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int k = kTileN * half + 2 * i;
+                float e0 = fast_exp2(fmaf(__uint_as_float(a[2 * i]), sl2, -m_new));
+                float e1 = fast_exp2(fmaf(__uint_as_float(a[2 * i + 1]), sl2, -m_new));
+                if (k >= n_valid) e0 = 0.f;
+                if (k + 1 >= n_valid) e1 = 0.f;
+                ps0 += e0;
+                ps1 += e1;
+                pk[i] = ptx::pack_bf16x2(e0, e1);
+              }
+            }
           }
           l += ps0 + ps1;
           // P tiles reach the value CTA's slots strictly in order: the other warpgroup stored
@@ -461,6 +493,47 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
 }
 
 // ---------------------------------------------------------------- value CTA
+// Value CTA epilogue of one warp: rows 32qd.. and latent columns 256c..256c+255 of O (TMEM), scaled
+// by inv and stored as bf16 rows of 512 at out_rows (row 0 = this warp's first row), through a
+// 32-row x 128-byte shared-memory transpose (buf, 8 KB) so that each store instruction writes four
+// whole 128-byte row pieces.
+__device__ __forceinline__ void store_o_rows(uint8_t* buf, uint32_t t_base, uint32_t lane, float inv,
+                                             __nv_bfloat16* out_rows) {
+#pragma unroll 1
+  for (int kk = 0; kk < 2; ++kk) {
+    // 128 columns per TMEM round trip
+    uint32_t r[128];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      ptx::tmem_ld32(t_base + 128 * kk + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * i]));
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ptx::reg_fence32(&r[32 * i]);
+    __syncwarp();   // the previous pieces were read out of buf
+#pragma unroll
+    for (int k2 = 0; k2 < 2; ++k2)
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const uint32_t* x = &r[64 * k2 + 8 * v];
+        *reinterpret_cast<uint4*>(buf + k2 * 4096 + lane * 128 + ((v ^ (lane & 7)) << 4)) =
+            make_uint4(ptx::pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
+                       ptx::pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
+                       ptx::pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
+                       ptx::pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
+      }
+    __syncwarp();
+#pragma unroll
+    for (int k2 = 0; k2 < 2; ++k2)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = 4 * i + (int)(lane >> 3), ch = (int)(lane & 7);
+        const uint4 x = *reinterpret_cast<const uint4*>(buf + k2 * 4096 + rr * 128 + ((ch ^ (rr & 7)) << 4));
+        *reinterpret_cast<uint4*>(out_rows + (int64_t)rr * 512 + 128 * kk + 64 * k2 + 8 * ch) = x;
+      }
+  }
+}
+
+
 __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const UnitRange& u, const AttnParams& p,
                                            const CUtensorMap* tmap_kv) {
   using L = ValueLayout;
@@ -624,6 +697,7 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
     // ---- epilogue: warp (qd, c) stores rows 32qd.. and latent columns 256c..256c+255 as bf16,
     // either o_lat = O / l (one split) or the split's partial O (relative to its final reference)
     const int c = (int)(warp >> 2);
+
     if (nt == 0) {
       if (p.num_splits == 1) {
         uint4* dst = reinterpret_cast<uint4*>(p.o_lat + (u.row * p.heads + u.hg * 128 + h) * 512 + 256 * c);
@@ -635,43 +709,10 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
       w = w && ptx::mbar_wait<true>(l_full, 0, kErrTimeoutPeer);   // also before exit: it writes here
       if (__all_sync(0xffffffffu, w)) {
         ptx::tc_fence_after();
-        uint8_t* buf = smem + warp * 8192;   // the kv ring is idle now: two 32-row x 128-byte tiles per warp
         const float inv = p.num_splits > 1 ? 1.f : 1.f / reinterpret_cast<const float*>(smem + L::kOffL)[h];
         const int64_t row0 = (p.num_splits > 1 ? ((int64_t)u.sp * p.n_q + u.row) * p.heads : u.row * p.heads) +
                              u.hg * 128 + 32 * qd;
-#pragma unroll 1
-        for (int kk = 0; kk < 2; ++kk) {
-          // 128 columns per TMEM round trip (the loads' latency is the epilogue's cost)
-          uint32_t r[128];
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            ptx::tmem_ld32(tmem + lane_base + 256 * c + 128 * kk + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * i]));
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 4; ++i) ptx::reg_fence32(&r[32 * i]);
-          __syncwarp();   // the previous pieces were read out of buf
-#pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2)
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const uint32_t* x = &r[64 * k2 + 8 * v];
-              *reinterpret_cast<uint4*>(buf + k2 * 4096 + lane * 128 + ((v ^ (lane & 7)) << 4)) =
-                  make_uint4(ptx::pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
-                             ptx::pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
-                             ptx::pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
-                             ptx::pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
-            }
-          __syncwarp();
-          // transposed read-back: each store instruction writes four whole 128-byte row pieces
-#pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int rr = 4 * i + (int)(lane >> 3), ch = (int)(lane & 7);
-              const uint4 x = *reinterpret_cast<const uint4*>(buf + k2 * 4096 + rr * 128 + ((ch ^ (rr & 7)) << 4));
-              *reinterpret_cast<uint4*>(p.out + (row0 + rr) * 512 + 256 * c + 128 * kk + 64 * k2 + 8 * ch) = x;
-            }
-        }
+        store_o_rows(smem + warp * 8192, tmem + lane_base + 256 * c, lane, inv, p.out + row0 * 512 + 256 * c);
 
       }
     }
