@@ -238,9 +238,17 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
     p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)splits * n_q * H * 512 * 2));
   }
   p.out = splits > 1 ? part_o : static_cast<__nv_bfloat16*>(o_lat);
+  CUtensorMap tout;
+  {
+    // the epilogue's output rows (o_lat, or the bf16 split partials) as [rows, 512]: boxes of
+    // 64 latent columns x 32 heads
+    const uint64_t d[2] = {512, (uint64_t)(splits > 1 ? splits : 1) * n_q * H}, st[1] = {1024};
+    const uint32_t b[2] = {64, 32};
+    if (!make_map(&tout, p.out, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
   if (!set_smem(latent_attn_kernel, kAttnSmem)) return MLA_ERR_CUDA;
   mla_status_t st = launch(true, latent_attn_kernel, dim3((unsigned)(2 * units)), dim3(kAttnThreads), kAttnSmem,
-                           stream, tkv_s, tpe, tqpe, tkv_v, tqa, p);
+                           stream, tkv_s, tpe, tqpe, tkv_v, tqa, tout, p);
   if (st != MLA_OK || splits <= 1) return st;
   return launch(true, merge_splits_kernel, dim3((unsigned)n_q, H), dim3(128), 0, stream,
                 (const __nv_bfloat16*)part_o, (const float*)p.part_ml, splits, n_q, H,

@@ -493,49 +493,45 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
 }
 
 // ---------------------------------------------------------------- value CTA
-// Value CTA epilogue of one warp: rows 32qd.. and latent columns 256c..256c+255 of O (TMEM), scaled
-// by inv and stored as bf16 rows of 512 at out_rows (row 0 = this warp's first row), through a
-// 32-row x 128-byte shared-memory transpose (buf, 8 KB) so that each store instruction writes four
-// whole 128-byte row pieces.
-__device__ __forceinline__ void store_o_rows(uint8_t* buf, uint32_t t_base, uint32_t lane, float inv,
-                                             __nv_bfloat16* out_rows) {
+// Value CTA epilogue of one warp: rows 32qd.. (TMEM lanes) and latent columns 256c..256c+255 of O,
+// scaled by inv, as bf16. Each 64-column piece goes through a 32-row x 128-byte box in shared
+// memory (buf, 16 KB, 1024-byte aligned, 128-byte swizzle: conflict-free row writes) and leaves
+// through the tensor memory accelerator at (x0 + 64 i, y0) of the output map. Returns once the
+// boxes have been read out of shared memory.
+__device__ __forceinline__ void store_o_tma(uint8_t* buf, uint32_t t_base, uint32_t lane, float inv,
+                                            const CUtensorMap* tmap_out, int32_t x0, int32_t y0) {
 #pragma unroll 1
-  for (int kk = 0; kk < 2; ++kk) {
-    // 128 columns per TMEM round trip
-    uint32_t r[128];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      ptx::tmem_ld32(t_base + 128 * kk + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * i]));
+  for (int bx = 0; bx < 4; ++bx) {   // one box: two 32-column TMEM loads, one wait
+    uint32_t r[64];
+    ptx::tmem_ld32(t_base + 64 * bx, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    ptx::tmem_ld32(t_base + 64 * bx + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
     ptx::tmem_wait_ld();
+    ptx::reg_fence32(&r[0]);
+    ptx::reg_fence32(&r[32]);
+    uint8_t* box = buf + bx * 4096;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) ptx::reg_fence32(&r[32 * i]);
-    __syncwarp();   // the previous pieces were read out of buf
-#pragma unroll
-    for (int k2 = 0; k2 < 2; ++k2)
-#pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        const uint32_t* x = &r[64 * k2 + 8 * v];
-        *reinterpret_cast<uint4*>(buf + k2 * 4096 + lane * 128 + ((v ^ (lane & 7)) << 4)) =
-            make_uint4(ptx::pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
-                       ptx::pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
-                       ptx::pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
-                       ptx::pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
-      }
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t* x = &r[8 * j];
+      *reinterpret_cast<uint4*>(box + lane * 128 + (((uint32_t)j ^ (lane & 7u)) << 4)) =
+          make_uint4(ptx::pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
+                     ptx::pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
+                     ptx::pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
+                     ptx::pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
+    }
+    ptx::fence_async_smem();
     __syncwarp();
-#pragma unroll
-    for (int k2 = 0; k2 < 2; ++k2)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int rr = 4 * i + (int)(lane >> 3), ch = (int)(lane & 7);
-        const uint4 x = *reinterpret_cast<const uint4*>(buf + k2 * 4096 + rr * 128 + ((ch ^ (rr & 7)) << 4));
-        *reinterpret_cast<uint4*>(out_rows + (int64_t)rr * 512 + 128 * kk + 64 * k2 + 8 * ch) = x;
-      }
+    if (lane == 0) {
+      ptx::tma_store_2d(tmap_out, box, x0 + 64 * bx, y0);
+      ptx::bulk_commit_group();
+    }
   }
+  if (lane == 0) ptx::bulk_wait_read_all();
+  __syncwarp();
 }
 
 
 __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const UnitRange& u, const AttnParams& p,
-                                           const CUtensorMap* tmap_kv) {
+                                           const CUtensorMap* tmap_kv, const CUtensorMap* tmap_out) {
   using L = ValueLayout;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBars);
   uint64_t* v_full = bars + bar::kVFull;      // [2] kv tile landed
@@ -554,7 +550,10 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
     // ============================================================ producer
     int issued = 0;
     if (nt > 0) {
-      if (ptx::elect_one()) ptx::prefetch_tmap(tmap_kv);
+      if (ptx::elect_one()) {
+        ptx::prefetch_tmap(tmap_kv);
+        ptx::prefetch_tmap(tmap_out);
+      }
       __syncwarp();
       // The first P tile arrives several microseconds in; loading values before then would only
       // add to the start-up burst on HBM (these rows reach L2 through the score CTA meanwhile).
@@ -712,7 +711,8 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
         const float inv = p.num_splits > 1 ? 1.f : 1.f / reinterpret_cast<const float*>(smem + L::kOffL)[h];
         const int64_t row0 = (p.num_splits > 1 ? ((int64_t)u.sp * p.n_q + u.row) * p.heads : u.row * p.heads) +
                              u.hg * 128 + 32 * qd;
-        store_o_rows(smem + warp * 8192, tmem + lane_base + 256 * c, lane, inv, p.out + row0 * 512 + 256 * c);
+        // the value stages are idle once the last P V product finished: 16 KB of boxes per warp
+        store_o_tma(smem + warp * 16384, tmem + lane_base + 256 * c, lane, inv, tmap_out, 256 * c, (int32_t)row0);
 
       }
     }
@@ -724,7 +724,8 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tmap_kv_score, const __grid_constant__ CUtensorMap tmap_pe,
                        const __grid_constant__ CUtensorMap tmap_qpe, const __grid_constant__ CUtensorMap tmap_kv_value,
-                       const __grid_constant__ CUtensorMap tmap_qabs, const AttnParams p) {
+                       const __grid_constant__ CUtensorMap tmap_qabs, const __grid_constant__ CUtensorMap tmap_out,
+                       const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t warp = ptx::warp_id();
   const uint32_t rank = ptx::cluster_rank();
@@ -788,7 +789,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   if (rank == 0)
     score_role(smem, tmem, u, p, &tmap_kv_score, &tmap_pe, &tmap_qpe, &tmap_qabs);
   else
-    value_role(smem, tmem, u, p, &tmap_kv_value);
+    value_role(smem, tmem, u, p, &tmap_kv_value, &tmap_out);
 
   ptx::tc_fence_before();
   __syncthreads();
