@@ -9,11 +9,13 @@ One step = the whole hot path on one batch: mla_absorb_q -> mla_attn_decode
 
 Prints one JSON line.  `value` is microseconds per step (lower is better),
 the max over ranks; with N > 1 every rank runs an independent replica (the
-path has no cross-GPU exchange).  L2 is flushed before every timed step, outside
-the timed events: a 256 MiB write followed by a 256 MiB read, so
-each timed step starts with none of its inputs in L2 and no dirty lines left
-to write back.  `--impl reference` times the fp64 CPU
-oracle on the host cores instead, one (sequence, head) pair per step.
+path has no cross-GPU exchange).  Inputs are larger than L2: every per-step
+input (q, kv and pe caches, wkv_b) exists in several copies, step i uses copy
+i mod copies, and between two uses of one copy the other copies move more than
+twice the L2 size, so each step reads its inputs from HBM.  The K timed steps
+run back to back (CUDA-graph replays of the public calls) between two CUDA
+events.  `--impl reference` times the fp64 CPU oracle on the host cores
+instead, one (sequence, head) pair per step.
 """
 from __future__ import annotations
 
@@ -38,7 +40,8 @@ UNIT = "us/step"
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 KV_BYTES_PER_TOKEN = (512 + 64) * 2            # latent + rotary key, bf16
 FLOP_PER_TOKEN_PER_HEAD = 2 * (576 + 512)      # score and value products
-L2_FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 << 20                           # B200 L2
+ROTATE_MIN_BYTES = 2 * L2_BYTES                # traffic between two uses of one input copy
 
 
 def parse_args():
@@ -228,38 +231,32 @@ def main():
     w = wl.workload(args.workload)
     d = mla.dims_from(w.dims)
     dt = torch.bfloat16 if w.dims.dtype == "bf16" else torch.float32
-    T = lambda a: torch.from_numpy(a).to(device=dev, dtype=dt)
-    q, kv, pe, wkv_b = T(w.q), T(w.kv), T(w.pe), T(w.wkv_b)
-    cu_k = torch.from_numpy(w.cu_seqlens_k).to(dev)
     B, H, C, Dv = w.batch, w.dims.heads, w.dims.kv_lora_rank, w.dims.v_head
     max_k = max(w.seqlens_k)
+    cu_k = torch.from_numpy(w.cu_seqlens_k).to(dev)
+    host = [torch.from_numpy(a).to(dtype=dt) for a in (w.q, w.kv, w.pe, w.wkv_b)]
+    per_copy = sum(t.numel() * t.element_size() for t in host)
+    copies = min(16, max(2, math.ceil(ROTATE_MIN_BYTES / per_copy) + 1))
+    inputs = [[t.to(dev) for t in host] for _ in range(copies)]   # (q, kv, pe, wkv_b) per copy
     bufs = {"q_abs": torch.empty((B, H, C), dtype=dt, device=dev),
             "o_lat": torch.empty((B, H, C), dtype=dt, device=dev),
             "out": torch.empty((B, H, Dv), dtype=dt, device=dev),
             "ws": mla.workspace(d, B, B, max_k, 0, device=dev)}
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    flush_read = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
-    flush_sum = torch.empty((), dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream()
 
-    def flush_l2():
-        # evict every input (write a buffer larger than L2), then read another one so the
-        # dirty lines of that write are written back before the timed region starts
-        flush.zero_()
-        torch.sum(flush_read, dim=0, out=flush_sum)
-
-    def step():
+    def step(k):
         # the whole hot path through the public calls: absorb -> attention (+ merge) -> output projection
+        q, kv, pe, wkv_b = inputs[k]
         q_abs = mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
         o_lat = mla.attn_decode(d, q_abs, q, kv, pe, cu_k, max_k, bufs["o_lat"], bufs["ws"])
         return mla.out_proj(d, o_lat, wkv_b, bufs["out"])
 
-    def attention_call():
+    def attention_call(k):
+        q, kv, pe, _ = inputs[k]
         mla.attn_decode(d, bufs["q_abs"], q, kv, pe, cu_k, max_k, bufs["o_lat"], bufs["ws"])
 
-    for _ in range(max(3, args.warmup)):
-        flush_l2()
-        step()
+    for i in range(max(3, args.warmup)):
+        step(i % copies)
     mla.device_status()
 
     # The timed steps replay CUDA graphs captured from the same calls, so host-side
@@ -275,19 +272,12 @@ def main():
             fn()
         return graph
 
-    g_step, g_attn = capture(step), capture(attention_call)
-    for _ in range(3):
-        flush_l2()
-        g_step.replay()
-        flush_l2()
-        g_attn.replay()
+    g_step = [capture(lambda k=k: step(k)) for k in range(copies)]
+    g_attn = [capture(lambda k=k: attention_call(k)) for k in range(copies)]
+    for i in range(max(3, args.warmup)):
+        g_step[i % copies].replay()
+        g_attn[i % copies].replay()
     mla.device_status()
-
-    n_ev = args.steps
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-    ev_as = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-    ev_ae = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
 
     sampler = None
     if rank == 0:
@@ -299,50 +289,50 @@ def main():
         sampler = ClockSampler(gpu_id)
         sampler.start()
         time.sleep(0.3)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush_l2()                        # L2 flush, outside the timed events
-        ev_s[i].record(stream)
-        g_step.replay()
-        ev_e[i].record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+
+    def timed(graphs, n):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            graphs[i % copies].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return e0.elapsed_time(e1)
+
+    total_ms = timed(g_step, args.steps)
     # the attention call alone (its kernel + split merge), for the roofline figure
-    for i in range(args.steps):
-        flush_l2()
-        ev_as[i].record(stream)
-        g_attn.replay()
-        ev_ae[i].record(stream)
-    torch.cuda.synchronize()
+    attn_total_ms = timed(g_attn, args.steps)
     clocks = sampler.stop() if sampler else None
     mla.device_status()
-
-    step_ms = [s.elapsed_time(e) for s, e in zip(ev_s, ev_e)]
-    attn_ms = [s.elapsed_time(e) for s, e in zip(ev_as, ev_ae)]
-    total_ms, mean_attn_ms = reduce_max([sum(step_ms), sum(attn_ms) / len(attn_ms)], dev)
+    total_ms, attn_total_ms = reduce_max([total_ms, attn_total_ms], dev)
     us_step = total_ms / args.steps * 1e3
+    mean_attn_ms = attn_total_ms / args.steps
 
-    # End to end through the same public calls: pinned host q -> device, step, out -> pinned host.
+    # End to end through the same public calls: pinned host q -> device, step, out -> pinned host,
+    # the K steps back to back between two events, inputs rotating over the same copies.
     q_pinned = torch.from_numpy(w.q).to(dt).pin_memory()
     out_pinned = torch.empty((B, H, Dv), dtype=dt).pin_memory()
-    q_dev = torch.empty_like(q)
     e2e_steps = min(args.steps, 500)
-    e2e_s = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
-    e2e_e = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
-    for i in range(e2e_steps):
-        flush_l2()
-        e2e_s[i].record(stream)
-        q_dev.copy_(q_pinned, non_blocking=True)
-        q_abs = mla.absorb_q(d, q_dev, wkv_b, bufs["q_abs"])
-        o_lat = mla.attn_decode(d, q_abs, q_dev, kv, pe, cu_k, max_k, bufs["o_lat"], bufs["ws"])
-        out = mla.out_proj(d, o_lat, wkv_b, bufs["out"])
-        out_pinned.copy_(out, non_blocking=True)
-        e2e_e[i].record(stream)
+    for i in range(3):
+        inputs[i % copies][0].copy_(q_pinned, non_blocking=True)
+        out_pinned.copy_(step(i % copies), non_blocking=True)
     torch.cuda.synchronize()
-    e2e_ms, = reduce_max([sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))], dev)
+    if world > 1:
+        dist.barrier()
+    e2e_s, e2e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_s.record(stream)
+    for i in range(e2e_steps):
+        k = i % copies
+        inputs[k][0].copy_(q_pinned, non_blocking=True)
+        out_pinned.copy_(step(k), non_blocking=True)
+    e2e_e.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms, = reduce_max([e2e_s.elapsed_time(e2e_e)], dev)
     e2e_us = e2e_ms / e2e_steps * 1e3
 
     if rank == 0:
@@ -359,7 +349,8 @@ def main():
             "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32", "data": "synthetic",
             "config": {"workload": w.name, "batch": B, "heads": H, "kv_lora_rank": C, "qk_rope": w.dims.qk_rope,
                        "seq_len_k": max_k, "queries_per_seq": 1, "parallelism": "replicas" if world > 1 else "single",
-                       "l2": "flushed before every timed step (256 MiB write then 256 MiB read, outside the events)"},
+                       "l2": f"inputs larger than L2: {copies} rotating copies of q, kv, pe and wkv_b "
+                             f"({copies * per_copy / 2**20:.0f} MiB), steps back to back between two events"},
             "tokens_per_s": world * B / (us_step / 1e6),
             "attn_kernel_us": mean_attn_ms * 1e3,
             "attn_cache_gbs": achieved_gbs,
