@@ -195,9 +195,12 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   {
     const uint64_t d[2] = {512, rows}, st[1] = {1024};
     const uint32_t bs[2] = {64, (uint32_t)kTileQ};    // score CTA: 64 latent columns x 128 keys
-    const uint32_t bv[2] = {64, (uint32_t)kTileN};    // value CTA: 64 latent columns x 64 keys
     if (!make_map(&tkv_s, kv_base, 2, d, st, bs, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-    if (!make_map(&tkv_v, kv_base, 2, d, st, bv, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    // value CTA: the cache as [8 latent blocks][rows][64 columns] (block stride 128 bytes), so one
+    // copy brings a whole 64-key tile as eight 64-column blocks
+    const uint64_t d3[3] = {64, rows, 8}, st3[2] = {1024, 128};
+    const uint32_t bv[3] = {64, (uint32_t)kTileN, 8};
+    if (!make_map(&tkv_v, kv_base, 3, d3, st3, bv, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
   {
     const uint64_t d[2] = {64, rows}, st[1] = {128};
@@ -240,17 +243,19 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   p.out = splits > 1 ? part_o : static_cast<__nv_bfloat16*>(o_lat);
   CUtensorMap tout;
   {
-    // the epilogue's output rows (o_lat, or the bf16 split partials) as [rows, 512]: boxes of
-    // 64 latent columns x 32 heads
-    const uint64_t d[2] = {512, (uint64_t)(splits > 1 ? splits : 1) * n_q * H}, st[1] = {1024};
-    const uint32_t b[2] = {64, 32};
-    if (!make_map(&tout, p.out, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    // the epilogue's output rows (o_lat, or the bf16 split partials) as [8 latent blocks][rows][64]:
+    // boxes of 4 blocks x 32 heads x 64 columns (a warp's quarter of the rows, half of the columns)
+    const uint64_t d[3] = {64, (uint64_t)(splits > 1 ? splits : 1) * n_q * H, 8}, st[2] = {1024, 128};
+    const uint32_t b[3] = {64, 32, 4};
+    if (!make_map(&tout, p.out, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
   if (!set_smem(latent_attn_kernel, kAttnSmem)) return MLA_ERR_CUDA;
   mla_status_t st = launch(true, latent_attn_kernel, dim3((unsigned)(2 * units)), dim3(kAttnThreads), kAttnSmem,
                            stream, tkv_s, tpe, tqpe, tkv_v, tqa, tout, p);
   if (st != MLA_OK || splits <= 1) return st;
-  return launch(true, merge_splits_kernel, dim3((unsigned)n_q, H), dim3(128), 0, stream,
+  const int64_t pairs_per_block = kMergeThreads / 64;   // two warps per (row, head)
+  const int64_t merge_blocks = (n_q * H + pairs_per_block - 1) / pairs_per_block;
+  return launch(true, merge_splits_kernel, dim3((unsigned)merge_blocks), dim3(kMergeThreads), 0, stream,
                 (const __nv_bfloat16*)part_o, (const float*)p.part_ml, splits, n_q, H,
                 static_cast<__nv_bfloat16*>(o_lat));
 }

@@ -494,12 +494,12 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
 
 // ---------------------------------------------------------------- value CTA
 // Value CTA epilogue of one warp: rows 32qd.. (TMEM lanes) and latent columns 256c..256c+255 of O,
-// scaled by inv, as bf16. Each 64-column piece goes through a 32-row x 128-byte box in shared
-// memory (buf, 16 KB, 1024-byte aligned, 128-byte swizzle: conflict-free row writes) and leaves
-// through the tensor memory accelerator at (x0 + 64 i, y0) of the output map. Returns once the
-// boxes have been read out of shared memory.
+// scaled by inv, as bf16. The four 64-column pieces fill four 32-row x 128-byte boxes in shared
+// memory (buf, 16 KB, 1024-byte aligned, 128-byte swizzle: conflict-free row writes) that leave
+// in one tensor store at (0, y0, z0) of the output map, whose third axis steps through 64-column
+// blocks. Returns once the boxes have been read out of shared memory.
 __device__ __forceinline__ void store_o_tma(uint8_t* buf, uint32_t t_base, uint32_t lane, float inv,
-                                            const CUtensorMap* tmap_out, int32_t x0, int32_t y0) {
+                                            const CUtensorMap* tmap_out, int32_t y0, int32_t z0) {
 #pragma unroll 1
   for (int bx = 0; bx < 4; ++bx) {   // one box: two 32-column TMEM loads, one wait
     uint32_t r[64];
@@ -518,14 +518,14 @@ __device__ __forceinline__ void store_o_tma(uint8_t* buf, uint32_t t_base, uint3
                      ptx::pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
                      ptx::pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
     }
-    ptx::fence_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      ptx::tma_store_2d(tmap_out, box, x0 + 64 * bx, y0);
-      ptx::bulk_commit_group();
-    }
   }
-  if (lane == 0) ptx::bulk_wait_read_all();
+  ptx::fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    ptx::tma_store_3d(tmap_out, buf, 0, y0, z0);
+    ptx::bulk_commit_group();
+    ptx::bulk_wait_read_all();
+  }
   __syncwarp();
 }
 
@@ -565,9 +565,9 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
         if (ptx::elect_one()) {
           const int key = (int)(key_base + (int64_t)j * kTileN);
           ptx::mbar_arrive_expect_tx(&v_full[st], L::kStage);
-#pragma unroll
-          for (int bx = 0; bx < 8; ++bx)
-            ptx::tma_load_2d(smem + st * L::kStage + bx * L::kKvBox, tmap_kv, &v_full[st], 64 * bx, key);
+          // one copy for the whole tile: eight 64-column blocks of 64 keys (the map's third axis
+          // steps through the latent blocks), laid out block after block
+          ptx::tma_load_3d(smem + st * L::kStage, tmap_kv, &v_full[st], 0, key, 0);
         }
         __syncwarp();
         issued = j + 1;
@@ -712,7 +712,7 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
         const int64_t row0 = (p.num_splits > 1 ? ((int64_t)u.sp * p.n_q + u.row) * p.heads : u.row * p.heads) +
                              u.hg * 128 + 32 * qd;
         // the value stages are idle once the last P V product finished: 16 KB of boxes per warp
-        store_o_tma(smem + warp * 16384, tmem + lane_base + 256 * c, lane, inv, tmap_out, 256 * c, (int32_t)row0);
+        store_o_tma(smem + warp * 16384, tmem + lane_base + 256 * c, lane, inv, tmap_out, (int32_t)row0, 4 * c);
 
       }
     }
@@ -799,63 +799,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
 
 // Merge split partials: o = sum_s 2^{m_s - M} O_s / sum_s 2^{m_s - M} l_s, M = max_s m_s,
 // with O_s the bf16 partial of split s (relative to its reference m_s).
-// One block of 128 threads per (row, head); thread i owns columns 4i..4i+3.
-// Every thread starts loading its partial columns of (up to) the first 16
-// splits at once, while warp 0 turns the (m, l) pairs into weights, so the
-// two memory round trips overlap.  Splits with no key (m = -inf) get weight 0
-// and their (unwritten) partial is never used.
-constexpr int kMaxSplits = 256;
+// Two warps per (row, head), four per block; lane i of warp k owns columns
+// 256k + 8i .. +7.  A lane starts loading its columns of (up to) the first
+// kMergeInFlight splits, then reads the (m, l) pair of split `lane` (one round
+// trip; weights reach the other lanes by shuffle), so the two memory round trips
+// overlap.  The kernel needs no shared memory: its blocks can be resident beside
+// the attention CTAs and start as soon as the attention grid completes.  Splits
+// with no key (m = -inf) get weight 0 and their (unwritten) partial is never used.
 constexpr int kMergeInFlight = 16;
-__global__ void __launch_bounds__(128) merge_splits_kernel(const __nv_bfloat16* __restrict__ part_o,
-                                                           const float* __restrict__ part_ml, int num_splits,
-                                                           int64_t n_q, int heads, __nv_bfloat16* __restrict__ o_lat) {
-  __shared__ float s_w[kMaxSplits];
-  __shared__ float s_inv;
+constexpr int kMergeThreads = 128;
+
+__device__ __forceinline__ void merge_acc(float (&a)[8], float w, const uint4& x) {
+  const uint32_t u[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[i]));
+    a[2 * i] = fmaf(w, f.x, a[2 * i]);
+    a[2 * i + 1] = fmaf(w, f.y, a[2 * i + 1]);
+  }
+}
+
+__global__ void __launch_bounds__(kMergeThreads) merge_splits_kernel(const __nv_bfloat16* __restrict__ part_o,
+                                                                 const float* __restrict__ part_ml, int num_splits,
+                                                                 int64_t n_q, int heads,
+                                                                 __nv_bfloat16* __restrict__ o_lat) {
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
-  const int64_t row = blockIdx.x;
-  const int head = blockIdx.y;
+  const int64_t warp_g = (int64_t)blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5);
+  const int64_t pair = warp_g >> 1;
+  if (pair >= n_q * heads) return;   // warp-uniform
+  const int lane = (int)(threadIdx.x & 31);
   const int64_t split_stride = n_q * heads;
-  const int64_t base = row * heads + head;
-  const uint2* src = reinterpret_cast<const uint2*>(part_o + base * 512) + threadIdx.x;
-  const int64_t step = split_stride * 512 / 4;
-  uint2 v[kMergeInFlight];
+  const uint4* src = reinterpret_cast<const uint4*>(part_o + pair * 512) + 32 * (warp_g & 1) + lane;
+  const int64_t step = split_stride * 512 / 8;   // one split further, in 16-byte units
+  uint4 v[kMergeInFlight];
 #pragma unroll
   for (int s = 0; s < kMergeInFlight; ++s)
     if (s < num_splits) v[s] = __ldcg(src + s * step);
-  if (threadIdx.x < 32) {
-    float M = -INFINITY;
-    for (int s = threadIdx.x; s < num_splits; s += 32) M = fmaxf(M, part_ml[(s * split_stride + base) * 2]);
-    M = warp_max(M);
-    float L = 0.f;
-    for (int s = threadIdx.x; s < num_splits; s += 32) {
-      const float ms = part_ml[(s * split_stride + base) * 2];
-      const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
-      s_w[s] = w;
-      L += w * part_ml[(s * split_stride + base) * 2 + 1];
-    }
-    L = warp_sum(L);
-    if (threadIdx.x == 0) s_inv = L > 0.f ? 1.f / L : 0.f;
+  const float2* ml = reinterpret_cast<const float2*>(part_ml) + pair;
+  const float2 mine = lane < num_splits ? __ldcg(ml + lane * split_stride) : make_float2(-INFINITY, 0.f);
+  float M = mine.x;
+  for (int s = lane + 32; s < num_splits; s += 32) M = fmaxf(M, __ldcg(ml + s * split_stride).x);
+  M = warp_max(M);
+  const float w_lane = mine.x == -INFINITY ? 0.f : exp2f(mine.x - M);   // the weight of split `lane`
+  float L = w_lane * mine.y;
+  for (int s = lane + 32; s < num_splits; s += 32) {
+    const float2 x = __ldcg(ml + s * split_stride);
+    if (x.x != -INFINITY) L += exp2f(x.x - M) * x.y;
   }
-  __syncthreads();
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  auto acc = [&](float w, uint2 x) {
-    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
-    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
-    a0 = fmaf(w, lo.x, a0); a1 = fmaf(w, lo.y, a1); a2 = fmaf(w, hi.x, a2); a3 = fmaf(w, hi.y, a3);
-  };
+  L = warp_sum(L);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = 0.f;
 #pragma unroll
   for (int s = 0; s < kMergeInFlight; ++s)
-    if (s < num_splits && s_w[s] != 0.f) acc(s_w[s], v[s]);
+    if (s < num_splits) {
+      const float w = __shfl_sync(0xffffffffu, w_lane, s);
+      if (w != 0.f) merge_acc(a, w, v[s]);
+    }
   for (int s = kMergeInFlight; s < num_splits; ++s) {
-    const uint2 x = __ldcg(src + s * step);
-    if (s_w[s] != 0.f) acc(s_w[s], x);
+    const float w = __shfl_sync(0xffffffffu, w_lane, s & 31);
+    const float2 x = __ldcg(ml + s * split_stride);   // splits >= 32: not in a lane's register
+    const float ws = s < 32 ? w : (x.x == -INFINITY ? 0.f : exp2f(x.x - M));
+    if (ws != 0.f) merge_acc(a, ws, __ldcg(src + s * step));
   }
-  const float inv = s_inv;
-  uint2 o;
-  o.x = ptx::pack_bf16x2(a0 * inv, a1 * inv);
-  o.y = ptx::pack_bf16x2(a2 * inv, a3 * inv);
-  reinterpret_cast<uint2*>(o_lat + base * 512)[threadIdx.x] = o;
+  uint4 o;
+  o.x = ptx::pack_bf16x2(a[0] * inv, a[1] * inv);
+  o.y = ptx::pack_bf16x2(a[2] * inv, a[3] * inv);
+  o.z = ptx::pack_bf16x2(a[4] * inv, a[5] * inv);
+  o.w = ptx::pack_bf16x2(a[6] * inv, a[7] * inv);
+  reinterpret_cast<uint4*>(o_lat + pair * 512)[32 * (warp_g & 1) + lane] = o;
 }
 
 }  // namespace sm100
