@@ -193,12 +193,12 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   const void* kv_base = kv_rows > 0 ? kv : q_abs;   // any valid 16-byte aligned address for an unused map
   const void* pe_base = kv_rows > 0 ? pe : q_abs;
   {
-    const uint64_t d[2] = {512, rows}, st[1] = {1024};
-    const uint32_t bs[2] = {64, (uint32_t)kTileQ};    // score CTA: 64 latent columns x 128 keys
-    if (!make_map(&tkv_s, kv_base, 2, d, st, bs, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-    // value CTA: the cache as [8 latent blocks][rows][64 columns] (block stride 128 bytes), so one
-    // copy brings a whole 64-key tile as eight 64-column blocks
+    // the cache as [8 latent blocks][rows][64 columns] (block stride 128 bytes): the score CTA
+    // copies two 64-column blocks of 128 keys at a time, the value CTA a whole 64-key tile
+    // (eight blocks) at a time
     const uint64_t d3[3] = {64, rows, 8}, st3[2] = {1024, 128};
+    const uint32_t bs[3] = {64, (uint32_t)kTileQ, 2};
+    if (!make_map(&tkv_s, kv_base, 3, d3, st3, bs, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     const uint32_t bv[3] = {64, (uint32_t)kTileN, 8};
     if (!make_map(&tkv_v, kv_base, 3, d3, st3, bv, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
@@ -215,17 +215,16 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   }
   CUtensorMap tqa;
   {
-    // q_abs viewed as [n_q * H, 512]: boxes of 64 latent columns x 128 heads
-    const uint64_t d[2] = {512, (uint64_t)n_q * H}, st[1] = {1024};
-    const uint32_t b[2] = {64, 128};
-    if (!make_map(&tqa, q_abs, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    // q_abs viewed as [8 latent blocks][n_q * H rows][64 columns] (block stride 128 bytes): one box
+    // is a unit's 128 heads, all eight 64-column blocks (128 KB)
+    const uint64_t d[3] = {64, (uint64_t)n_q * H, 8}, st[2] = {1024, 128};
+    const uint32_t b[3] = {64, 128, 8};
+    if (!make_map(&tqa, q_abs, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
   AttnParams p;
   p.q_abs = static_cast<const __nv_bfloat16*>(q_abs);
   p.cu_q = cu_q;
   p.cu_k = cu_k;
-  p.kv = static_cast<const __nv_bfloat16*>(kv);
-  p.pe = static_cast<const __nv_bfloat16*>(pe);
   p.batch = batch;
   p.heads = H;
   p.head_groups = H / 128;
@@ -244,9 +243,9 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   CUtensorMap tout;
   {
     // the epilogue's output rows (o_lat, or the bf16 split partials) as [8 latent blocks][rows][64]:
-    // boxes of 4 blocks x 32 heads x 64 columns (a warp's quarter of the rows, half of the columns)
+    // boxes of 32 heads x 64 columns (an epilogue warp writes four of them)
     const uint64_t d[3] = {64, (uint64_t)(splits > 1 ? splits : 1) * n_q * H, 8}, st[2] = {1024, 128};
-    const uint32_t b[3] = {64, 32, 4};
+    const uint32_t b[3] = {64, 32, 1};
     if (!make_map(&tout, p.out, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
   if (!set_smem(latent_attn_kernel, kAttnSmem)) return MLA_ERR_CUDA;

@@ -29,12 +29,15 @@
 // elected lane issuing, a 128 x 64 x 16 MMA takes 48 cycles where 32 would be
 // full rate, while N >= 128 runs at full rate.
 //
-// Score CTA.  TMEM: [0,256) q_abs (bf16 pairs; it lands by TMA in ring units
-// 5-10 and the staging slots and the softmax threads move it into TMEM), two S buffers of 128 columns at 256 and 384.  Shared
-// memory: a ring of eleven 16 KB units, a unit being one 64-column block of
-// 128 keys (eight latent blocks and the rotary block make a score tile) with
-// 128-byte swizzle, q_pe (128 heads x 64, the A operand of the rotary
-// products) and two P staging slots.  Warps 0-3 and 4-7 are two softmax warpgroups that take
+// Score CTA.  TMEM: [0,256) q_abs (bf16 pairs; it lands by TMA in latent
+// slots 1-4 and the softmax threads move it into TMEM), two S buffers of 128
+// columns at 256 and 384.  Shared memory (128-byte swizzle throughout): a ring
+// of five 32 KB latent slots (two 64-column blocks of 128 keys, one TMA copy
+// each; four make the latent part of a score tile), two 16 KB rotary slots
+// (the 64 rotary columns of 128 keys), q_pe (128 heads x 64, the A operand of
+// the rotary products) and one P staging slot.  A copy costs the TMA engine a
+// fixed overhead besides its bytes, so fewer, larger copies per tile raise the
+// rate at which one SM can pull keys.  Warps 0-3 and 4-7 are two softmax warpgroups that take
 // alternate score tiles (thread = head row, all 128 keys); warp 8 loads,
 // warp 9 issues the MMAs.  The running reference max m of each row passes
 // from one warpgroup to the other once per tile through shared memory; it is
@@ -64,22 +67,23 @@ constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kTileN = 64;                 // keys per P tile (value CTA granule)
 constexpr int kTileQ = 128;                // keys per score tile
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kPrefetchTiles = 1;          // L2 prefetch distance of the score CTA, in score tiles
 
 // Score CTA shared memory.
 struct ScoreLayout {
-  static constexpr int kUnit = kTileQ * 128;               // 128 keys x 64 columns bf16 (one TMA box)
-  static constexpr int kUnits = 11;
-  static constexpr int kUnitsPerTile = 9;                  // 8 latent blocks + the rotary block
-  static constexpr int kOffQpe = kUnits * kUnit;           // q_pe: 128 heads x 64 bf16
-  static constexpr int kOffStaging = kOffQpe + 128 * 128;  // two P staging slots, laid out like the value CTA's
-  static constexpr int kSlot = 17408;                      // P 16 KB, factors 512 B, then 512 B of
-  static constexpr int kOffMInSlot = 16896;                //   reference-max hand-off for warpgroup (slot index)
-  static constexpr int kOffEndL = kOffStaging + 2 * kSlot; // warpgroup 1's row sums at the end [128]
+  static constexpr int kBlock = kTileQ * 128;              // 128 keys x 64 columns bf16 (16 KB)
+  static constexpr int kLat = 2 * kBlock;                  // latent slot: two 64-column blocks (one TMA copy)
+  static constexpr int kLatSlots = 5;
+  static constexpr int kLatPerTile = 4;
+  static constexpr int kPeSlots = 2;
+  static constexpr int kOffPe = kLatSlots * kLat;          // rotary slots, 16 KB each
+  static constexpr int kOffQpe = kOffPe + kPeSlots * kBlock;  // q_pe: 128 heads x 64 bf16
+  static constexpr int kOffStaging = kOffQpe + 128 * 128;  // the P staging slot, laid out like the value CTA's
+  static constexpr int kSlot = 17408;                      // P 16 KB, factors 512 B
+  static constexpr int kOffM = kOffStaging + kSlot;        // reference max published by warpgroup g: [2][128]
+  static constexpr int kOffEndL = kOffM + 1024;            // warpgroup 1's row sums at the end [128]
   static constexpr int kOffBars = kOffEndL + 512;
   static constexpr int kBytes = kOffBars + 512;
-  // q_abs lands before the first tile in units 5..10 (boxes 0-5) and the staging slots (boxes 6-7)
-  static constexpr int kQUnit0 = 5;
+  static constexpr int kOffQ = kLat;                       // q_abs lands in latent slots 1-4 (128 KB)
 };
 
 // Value CTA shared memory.
@@ -99,7 +103,7 @@ struct ValueLayout {
 
 constexpr int kAttnSmem = ScoreLayout::kBytes > ValueLayout::kBytes ? ScoreLayout::kBytes : ValueLayout::kBytes;
 static_assert(kAttnSmem <= 232448, "attention shared memory above the per-CTA limit");
-static_assert(ScoreLayout::kOffQpe % 1024 == 0 && ScoreLayout::kOffStaging % 1024 == 0 &&
+static_assert(ScoreLayout::kOffPe % 1024 == 0 && ScoreLayout::kOffQpe % 1024 == 0 && ScoreLayout::kOffStaging % 1024 == 0 &&
                   ValueLayout::kOffSlots % 1024 == 0 && ValueLayout::kSlot % 1024 == 0,
               "swizzled operands need 1024-byte alignment");
 static_assert(ScoreLayout::kSlot == ValueLayout::kSlot, "staging and P slots share one layout");
@@ -109,8 +113,6 @@ struct AttnParams {
   const __nv_bfloat16* q_abs;   // [n_q, H, 512]
   const int* cu_q;              // [batch+1] for chunked prefill, nullptr for decode
   const int* cu_k;              // [batch+1]
-  const __nv_bfloat16* kv;      // [kv_rows, 512] (L2 prefetch)
-  const __nv_bfloat16* pe;      // [kv_rows, 64]
   int batch;
   int heads;
   int head_groups;              // heads / 128
@@ -163,8 +165,8 @@ __device__ __forceinline__ UnitRange unit_range(const AttnParams& p, int64_t uni
 // Barrier slots (8 bytes each) in the 512-byte barrier area of either role.
 namespace bar {
 // score CTA
-constexpr int kUFull = 0, kUEmpty = 11, kSFull = 22, kSFree = 24, kMBar = 26, kPFree = 28, kQFull = 32,
-              kQReady = 33, kEnd = 34, kScoreIdle = 35, kPSent = 36, kStgFree = 38;
+constexpr int kUFull = 0, kUEmpty = 5, kPeFull = 10, kPeEmpty = 12, kSFull = 22, kSFree = 24, kMBar = 26,
+              kPFree = 28, kQFull = 32, kQReady = 33, kEnd = 34, kScoreIdle = 35, kPSent = 36;
 // value CTA
 constexpr int kVFull = 0, kVEmpty = 2, kPFull = 4, kPvGo = 8, kPDone = 12, kOFinal = 16, kLFull = 17,
               kValueIdle = 18;
@@ -179,13 +181,14 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
                                            const CUtensorMap* tmap_qpe, const CUtensorMap* tmap_qabs) {
   using L = ScoreLayout;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBars);
-  uint64_t* u_full = bars + bar::kUFull;       // [13] ring unit landed
-  uint64_t* u_empty = bars + bar::kUEmpty;     // [13] ring unit read by the tensor core
+  uint64_t* u_full = bars + bar::kUFull;       // [5] latent slot landed
+  uint64_t* u_empty = bars + bar::kUEmpty;     // [5] latent slot read by the tensor core
+  uint64_t* pe_full = bars + bar::kPeFull;     // [2] rotary slot landed
+  uint64_t* pe_empty = bars + bar::kPeEmpty;   // [2] rotary slot read by the tensor core
   uint64_t* s_full = bars + bar::kSFull;       // [2] QK product committed
   uint64_t* s_free = bars + bar::kSFree;       // [2] S read out (128 arrivals)
   uint64_t* m_bar = bars + bar::kMBar;         // [2] warpgroup g published the reference max of its tile (128)
   uint64_t* p_free = bars + bar::kPFree;       // [4] the value CTA finished the P V product of this P slot
-  uint64_t* stg_free = bars + bar::kStgFree;   // [2] the P tile in this staging slot landed in the value CTA
   uint64_t* q_full = bars + bar::kQFull;       // q_abs and q_pe landed
   uint64_t* q_ready = bars + bar::kQReady;     // q_abs in TMEM, its landing zone free (256 arrivals)
   uint64_t* end_bar = bars + bar::kEnd;        // warpgroup 1 published its (l, m) (128)
@@ -194,59 +197,56 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
   const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id();
   const int ntp = u.nt;                        // 64-key P tiles
   const int ntq = (ntp + 1) / 2;               // 128-key score tiles
-  const int nu = L::kUnitsPerTile * ntq;       // ring units
   const int64_t key_base = u.k0 + u.j_begin;
   const int head0 = u.hg * 128;
-  // where q_abs box b (latent columns 64b..) lands before the first tile
-  auto q_box = [&](int b) -> uint8_t* {
-    return b < 6 ? smem + (L::kQUnit0 + b) * L::kUnit : smem + L::kOffStaging + (b - 6) * L::kSlot;
-  };
 
   if (warp == kProducerWarp) {
     // ============================================================ producer
-    auto prefetch_tile = [&](int jj) {
-      const int64_t key = key_base + (int64_t)jj * kTileQ;
-      const int64_t rows = min64(kTileQ, p.kv_rows - key);
-      if (rows > 0) {
-        ptx::prefetch_l2(p.kv + key * 512, (uint32_t)(rows * 1024));
-        ptx::prefetch_l2(p.pe + key * 64, (uint32_t)(rows * 128));
-      }
-    };
-    int issued = 0;
+    int lat_issued = 0, pe_issued = 0;
     if (ntp > 0) {
       if (ptx::elect_one()) {
         ptx::prefetch_tmap(tmap_kv);
         ptx::prefetch_tmap(tmap_pe);
-        ptx::mbar_arrive_expect_tx(q_full, 8 * L::kUnit + 128 * 128);
-#pragma unroll
-        for (int b = 0; b < 8; ++b)
-          ptx::tma_load_2d(q_box(b), tmap_qabs, q_full, 64 * b, (int)(u.row * p.heads + head0));
+        // q_abs (eight 64-column blocks of 128 heads, one copy) into latent slots 1-4, and q_pe
+        ptx::mbar_arrive_expect_tx(q_full, 128 * 1024 + 128 * 128);
+        ptx::tma_load_3d(smem + L::kOffQ, tmap_qabs, q_full, 0, (int)(u.row * p.heads + head0), 0);
         ptx::tma_load_3d(smem + L::kOffQpe, tmap_qpe, q_full, 128, head0, (int)u.row);
       }
       __syncwarp();
-      for (int uu = 0; uu < nu; ++uu) {
-        const int slot = uu % L::kUnits, use = uu / L::kUnits;
-        const int jj = uu / L::kUnitsPerTile, cb = uu % L::kUnitsPerTile;
-        bool w = true;
-        if (uu >= L::kQUnit0 && uu < L::kUnits) w = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax);   // held q_abs
-        w = w && ptx::mbar_wait(&u_empty[slot], (use & 1) ^ 1, kErrTimeoutStageFree);
+      bool ok = true;
+      for (int jj = 0; ok && jj < ntq; ++jj) {
+        const int key = (int)(key_base + (int64_t)jj * kTileQ);
+        // the rotary block of the tile
+        const int ps = jj % L::kPeSlots;
+        bool w = ptx::mbar_wait(&pe_empty[ps], ((jj / L::kPeSlots) & 1) ^ 1, kErrTimeoutStageFree);
         if (!__all_sync(0xffffffffu, w)) break;
         if (ptx::elect_one()) {
-          const int key = (int)(key_base + (int64_t)jj * kTileQ);
-          ptx::mbar_arrive_expect_tx(&u_full[slot], L::kUnit);
-          if (cb < 8)
-            ptx::tma_load_2d(smem + slot * L::kUnit, tmap_kv, &u_full[slot], 64 * cb, key);
-          else
-            ptx::tma_load_2d(smem + slot * L::kUnit, tmap_pe, &u_full[slot], 0, key);
-          // keep the score tile kPrefetchTiles ahead streaming into L2
-          if (kPrefetchTiles > 0 && cb == 0 && jj + kPrefetchTiles < ntq) prefetch_tile(jj + kPrefetchTiles);
+          ptx::mbar_arrive_expect_tx(&pe_full[ps], L::kBlock);
+          ptx::tma_load_2d(smem + L::kOffPe + ps * L::kBlock, tmap_pe, &pe_full[ps], 0, key);
         }
         __syncwarp();
-        issued = uu + 1;
+        pe_issued = jj + 1;
+        // the latent blocks, two per copy
+#pragma unroll 1
+        for (int k = 0; k < L::kLatPerTile; ++k) {
+          const int li = L::kLatPerTile * jj + k, slot = li % L::kLatSlots, use = li / L::kLatSlots;
+          w = true;
+          if (use == 0 && slot >= 1) w = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax);   // held q_abs
+          w = w && ptx::mbar_wait(&u_empty[slot], (use & 1) ^ 1, kErrTimeoutStageFree);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          if (ptx::elect_one()) {
+            ptx::mbar_arrive_expect_tx(&u_full[slot], L::kLat);
+            ptx::tma_load_3d(smem + slot * L::kLat, tmap_kv, &u_full[slot], 0, key, 2 * k);
+          }
+          __syncwarp();
+          lat_issued = li + 1;
+        }
       }
       // exit path: every copy this CTA started has landed before its shared memory goes away
-      for (int uu = (issued > L::kUnits ? issued - L::kUnits : 0); uu < issued; ++uu)
-        ptx::mbar_wait(&u_full[uu % L::kUnits], (uu / L::kUnits) & 1, kErrTimeoutDrain);
+      for (int li = (lat_issued > L::kLatSlots ? lat_issued - L::kLatSlots : 0); li < lat_issued; ++li)
+        ptx::mbar_wait(&u_full[li % L::kLatSlots], (li / L::kLatSlots) & 1, kErrTimeoutDrain);
+      for (int jj = (pe_issued > L::kPeSlots ? pe_issued - L::kPeSlots : 0); jj < pe_issued; ++jj)
+        ptx::mbar_wait(&pe_full[jj % L::kPeSlots], (jj / L::kPeSlots) & 1, kErrTimeoutDrain);
       ptx::mbar_wait(q_full, 0, kErrTimeoutDrain);
     }
     __syncwarp();
@@ -261,7 +261,7 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
       const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(smem), 16, 1024, ptx::kSwizzle128);
       const uint64_t d_qpe = ptx::smem_desc(ptx::smem_u32(smem + L::kOffQpe), 16, 1024, ptx::kSwizzle128);
       ptx::tc_fence_after();
-      // Each issue site has one fixed MMA form (the column-block loop is unrolled):
+      // Each issue site has one fixed MMA form (the block loops are unrolled):
       // a loop that can reach both the TMEM-A and the shared-memory-A form from one
       // elected branch issued at a quarter of the tensor-core rate.
       for (int jj = 0; ok && jj < ntq; ++jj) {
@@ -270,34 +270,44 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
           if (!ok) break;
         }
         const uint32_t scol = tmem + kColS + (uint32_t)(jj & 1) * kTileQ;
-#pragma unroll
-        for (int cb = 0; cb < L::kUnitsPerTile; ++cb) {
-          const int uu = L::kUnitsPerTile * jj + cb, slot = uu % L::kUnits;
-          ok = __all_sync(0xffffffffu, ptx::mbar_wait(&u_full[slot], (uu / L::kUnits) & 1, kErrTimeoutTmaFull));
+        // rotary block first (it starts the accumulation): A = q_pe in shared memory
+        {
+          const int ps = jj % L::kPeSlots;
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(&pe_full[ps], (jj / L::kPeSlots) & 1, kErrTimeoutTmaFull));
           if (!ok) break;
           ptx::tc_fence_after();
-          const uint64_t d_b = d_ring + (uint32_t)((slot * L::kUnit) >> 4);
-          if (cb < 8) {
-            // latent block cb: A = q_abs columns 64cb.. in TMEM
+          const uint64_t d_b = d_ring + (uint32_t)((L::kOffPe + ps * L::kBlock) >> 4);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              if (ptx::elect_one())
-                ptx::mma_ts(scol, tmem + kColQ + 32 * cb + 8 * k, d_b + (uint32_t)((k * 32) >> 4), idesc,
-                            (cb | k) ? 1u : 0u);
-              __syncwarp();
-            }
-          } else {
-            // rotary block: A = q_pe in shared memory
+          for (int k = 0; k < 4; ++k) {
+            if (ptx::elect_one())
+              ptx::mma_ss(scol, d_qpe + (uint32_t)((k * 32) >> 4), d_b + (uint32_t)((k * 32) >> 4), idesc,
+                          k > 0 ? 1u : 0u);
+            __syncwarp();
+          }
+          if (ptx::elect_one()) ptx::mma_commit(&pe_empty[ps]);
+          __syncwarp();
+        }
+        // latent blocks: A = q_abs columns 64b.. in TMEM
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < L::kLatPerTile; ++k) {
+          const int li = L::kLatPerTile * jj + k, slot = li % L::kLatSlots;
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(&u_full[slot], (li / L::kLatSlots) & 1, kErrTimeoutTmaFull));
+          if (!ok) break;
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+            const int b = 2 * k + bb;
+            const uint64_t d_b = d_ring + (uint32_t)((slot * L::kLat + bb * L::kBlock) >> 4);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
               if (ptx::elect_one())
-                ptx::mma_ss(scol, d_qpe + (uint32_t)((k * 32) >> 4), d_b + (uint32_t)((k * 32) >> 4), idesc, 1u);
+                ptx::mma_ts(scol, tmem + kColQ + 32 * b + 8 * ks, d_b + (uint32_t)((ks * 32) >> 4), idesc, 1u);
               __syncwarp();
             }
           }
           if (ptx::elect_one()) {
             ptx::mma_commit(&u_empty[slot]);
-            if (cb == 8) ptx::mma_commit(&s_full[jj & 1]);
+            if (k == L::kLatPerTile - 1) ptx::mma_commit(&s_full[jj & 1]);
           }
           __syncwarp();
         }
@@ -316,7 +326,7 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
     const float sl2 = p.scale_log2;
     // reference max published by warpgroup x for its latest tile: 128 floats in staging slot x's tail
-    auto m_slot = [&](int x) -> float* { return reinterpret_cast<float*>(smem + L::kOffStaging + x * L::kSlot + L::kOffMInSlot); };
+    auto m_slot = [&](int x) -> float* { return reinterpret_cast<float*>(smem + L::kOffM + x * 512); };
     float* end_l = reinterpret_cast<float*>(smem + L::kOffEndL);  // warpgroup 1's row sums at the end
     bool ok = true;
     float m_used = -INFINITY, l = 0.f;   // reference this warpgroup last used, and its row sum relative to it
@@ -327,7 +337,7 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
       if (ok) {
 #pragma unroll 1
         for (int b = 4 * g; b < 4 * g + 4; ++b) {
-          const uint8_t* src = q_box(b) + h * 128;
+          const uint8_t* src = smem + L::kOffQ + b * L::kBlock + h * 128;
           uint32_t r[32];
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
@@ -391,66 +401,70 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
           l = m_used == -INFINITY ? 0.f : l * fast_exp2(m_used - m_new);
           m_used = m_new;
         }
-        // P = 2^(s * scale * log2(e) - m) as bf16, in two 64-key P tiles; keys past the end weigh exactly 0
+        // P = 2^(s * scale * log2(e) - m) as bf16, in two 64-key P tiles; keys past the end weigh
+        // exactly 0.  Both P tiles are computed before the wait for the other warpgroup's P: only
+        // the staging writes and copies are ordered between warpgroups, not the exponentials.
+        const int nh = n_valid > kTileN ? 2 : 1;
+        uint32_t pk[2][32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          if (kTileN * half >= n_valid) break;
-          const int t = 2 * jj + half, ps = t & 1, vs = t & 3;
-          uint32_t pk[32];
+          if (half >= nh) break;
           float ps0 = 0.f, ps1 = 0.f;
-          {
-            uint32_t a[64];
-            ptx::tmem_ld32(s_col + kTileN * half, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-            ptx::tmem_ld32(s_col + kTileN * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-            ptx::tmem_wait_ld();
-            ptx::reg_fence32(&a[0]);
-            ptx::reg_fence32(&a[32]);
-            if (half == 1 || kTileN >= n_valid) {
-              // the last read of this S buffer: QK(jj+2) may overwrite it
-              ptx::tc_fence_before();
-              ptx::mbar_arrive(&s_free[sb]);
+          uint32_t a[64];
+          ptx::tmem_ld32(s_col + kTileN * half, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+          ptx::tmem_ld32(s_col + kTileN * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+          ptx::tmem_wait_ld();
+          ptx::reg_fence32(&a[0]);
+          ptx::reg_fence32(&a[32]);
+          if (half == nh - 1) {
+            // the last read of this S buffer: QK(jj+2) may overwrite it
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&s_free[sb]);
+          }
+          if (kTileN * (half + 1) <= n_valid) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float e0 = fast_exp2(fmaf(__uint_as_float(a[2 * i]), sl2, -m_new));
+              const float e1 = fast_exp2(fmaf(__uint_as_float(a[2 * i + 1]), sl2, -m_new));
+              ps0 += e0;
+              ps1 += e1;
+              pk[half][i] = ptx::pack_bf16x2(e0, e1);
             }
-            if (kTileN * (half + 1) <= n_valid) {
+          } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float e0 = fast_exp2(fmaf(__uint_as_float(a[2 * i]), sl2, -m_new));
-                const float e1 = fast_exp2(fmaf(__uint_as_float(a[2 * i + 1]), sl2, -m_new));
-                ps0 += e0;
-                ps1 += e1;
-                pk[i] = ptx::pack_bf16x2(e0, e1);
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int k = kTileN * half + 2 * i;
-                float e0 = fast_exp2(fmaf(__uint_as_float(a[2 * i]), sl2, -m_new));
-                float e1 = fast_exp2(fmaf(__uint_as_float(a[2 * i + 1]), sl2, -m_new));
-                if (k >= n_valid) e0 = 0.f;
-                if (k + 1 >= n_valid) e1 = 0.f;
-                ps0 += e0;
-                ps1 += e1;
-                pk[i] = ptx::pack_bf16x2(e0, e1);
-              }
+            for (int i = 0; i < 32; ++i) {
+              const int k = kTileN * half + 2 * i;
+              float e0 = fast_exp2(fmaf(__uint_as_float(a[2 * i]), sl2, -m_new));
+              float e1 = fast_exp2(fmaf(__uint_as_float(a[2 * i + 1]), sl2, -m_new));
+              if (k >= n_valid) e0 = 0.f;
+              if (k + 1 >= n_valid) e1 = 0.f;
+              ps0 += e0;
+              ps1 += e1;
+              pk[half][i] = ptx::pack_bf16x2(e0, e1);
             }
           }
           l += ps0 + ps1;
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (half >= nh) break;
+          const int t = 2 * jj + half, vs = t & 3;
           // P tiles reach the value CTA's slots strictly in order: the other warpgroup stored
-          // those of score tile jj-1 first.  (It hands over the reference max before its P, so
-          // without this a warpgroup could wait on a P slot barrier two phases ahead, which a
-          // parity wait cannot tell from the phase before.)  Then staging slot ps is free once
-          // P tile t-2 landed in the value CTA, and its P slot vs once P V of tile t-4 finished.
+          // those of score tile jj-1 first (and its copies have read the staging slot).  (It hands
+          // over the reference max before its P, so without this a warpgroup could wait on a P slot
+          // barrier two phases ahead, which a parity wait cannot tell from the phase before.)  The
+          // value CTA's P slot vs is free once P V of tile t-4 finished.
           w = true;
           if (half == 0 && jj > 0) w = ptx::mbar_wait(&p_sent[g ^ 1], ((jj - 1) >> 1) & 1, kErrTimeoutSoftmax);
-          if (t >= 2) w = w && ptx::mbar_wait<true>(&stg_free[ps], ((t - 2) >> 1) & 1, kErrTimeoutPeer);
           if (t >= 4) w = w && ptx::mbar_wait<true>(&p_free[vs], ((t - 4) >> 2) & 1, kErrTimeoutPeer);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-          // row h of the K-major P tile (128-byte swizzle) and the row's factor into staging slot ps,
-          // then this warp's 32 rows and factors to the value CTA's P slot ps (two bulk copies)
-          uint8_t* stg = smem + L::kOffStaging + ps * L::kSlot;
+          // row h of the K-major P tile (128-byte swizzle) and the row's factor into the staging slot,
+          // then this warp's 32 rows and factors to the value CTA's P slot vs (two bulk copies)
+          uint8_t* stg = smem + L::kOffStaging;
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             *reinterpret_cast<uint4*>(stg + h * 128 + ((c ^ (h & 7)) << 4)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                make_uint4(pk[half][4 * c], pk[half][4 * c + 1], pk[half][4 * c + 2], pk[half][4 * c + 3]);
           reinterpret_cast<float*>(stg + ValueLayout::kOffF)[h] = half == 0 ? f : 1.f;
           ptx::fence_async_smem();
           __syncwarp();
@@ -460,7 +474,12 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
             ptx::bulk_copy_to_peer(dst + qd * 4096, ptx::smem_u32(stg) + qd * 4096, 4096, vbar);
             ptx::bulk_copy_to_peer(dst + ValueLayout::kOffF + qd * 128, ptx::smem_u32(stg) + ValueLayout::kOffF + qd * 128,
                                    128, vbar);
+            ptx::bulk_commit_group();
+            // these rows of the staging slot are written again (the next half, or the other
+            // warpgroup's next tile) only after the copies have read them
+            ptx::bulk_wait_read_all();
           }
+          __syncwarp();
         }
         if (!ok) break;
         if (lane == 0) ptx::mbar_arrive(&p_sent[g]);
@@ -494,41 +513,47 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
 
 // ---------------------------------------------------------------- value CTA
 // Value CTA epilogue of one warp: rows 32qd.. (TMEM lanes) and latent columns 256c..256c+255 of O,
-// scaled by inv, as bf16. The four 64-column pieces fill four 32-row x 128-byte boxes in shared
-// memory (buf, 16 KB, 1024-byte aligned, 128-byte swizzle: conflict-free row writes) that leave
-// in one tensor store at (0, y0, z0) of the output map, whose third axis steps through 64-column
-// blocks. Returns once the boxes have been read out of shared memory.
+// scaled by inv, as bf16. TMEM is read 128 columns per round trip; each 64-column piece fills a
+// 32-row x 128-byte box in shared memory (buf, 16 KB, 1024-byte aligned, 128-byte swizzle:
+// conflict-free row writes) that leaves in its own tensor store at (0, y0, z0 + box) of the output
+// map (whose third axis steps through 64-column blocks); the stores of the first two boxes overlap
+// the second TMEM round trip. Returns once the boxes have been read out.
 __device__ __forceinline__ void store_o_tma(uint8_t* buf, uint32_t t_base, uint32_t lane, float inv,
                                             const CUtensorMap* tmap_out, int32_t y0, int32_t z0) {
 #pragma unroll 1
-  for (int bx = 0; bx < 4; ++bx) {   // one box: two 32-column TMEM loads, one wait
-    uint32_t r[64];
-    ptx::tmem_ld32(t_base + 64 * bx, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-    ptx::tmem_ld32(t_base + 64 * bx + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-    ptx::tmem_wait_ld();
-    ptx::reg_fence32(&r[0]);
-    ptx::reg_fence32(&r[32]);
-    uint8_t* box = buf + bx * 4096;
+  for (int pr = 0; pr < 2; ++pr) {
+    uint32_t r[128];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t* x = &r[8 * j];
-      *reinterpret_cast<uint4*>(box + lane * 128 + (((uint32_t)j ^ (lane & 7u)) << 4)) =
-          make_uint4(ptx::pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
-                     ptx::pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
-                     ptx::pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
-                     ptx::pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
+    for (int i = 0; i < 4; ++i)
+      ptx::tmem_ld32(t_base + 128 * pr + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * i]));
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ptx::reg_fence32(&r[32 * i]);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      uint8_t* box = buf + (2 * pr + k) * 4096;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t* x = &r[64 * k + 8 * j];
+        *reinterpret_cast<uint4*>(box + lane * 128 + (((uint32_t)j ^ (lane & 7u)) << 4)) =
+            make_uint4(ptx::pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
+                       ptx::pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
+                       ptx::pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
+                       ptx::pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
+      }
     }
+    ptx::fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      ptx::tma_store_3d(tmap_out, buf + (2 * pr) * 4096, 0, y0, z0 + 2 * pr);
+      ptx::tma_store_3d(tmap_out, buf + (2 * pr + 1) * 4096, 0, y0, z0 + 2 * pr + 1);
+      ptx::bulk_commit_group();
+    }
+    __syncwarp();
   }
-  ptx::fence_async_smem();
-  __syncwarp();
-  if (lane == 0) {
-    ptx::tma_store_3d(tmap_out, buf, 0, y0, z0);
-    ptx::bulk_commit_group();
-    ptx::bulk_wait_read_all();
-  }
+  if (lane == 0) ptx::bulk_wait_read_all();
   __syncwarp();
 }
-
 
 __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const UnitRange& u, const AttnParams& p,
                                            const CUtensorMap* tmap_kv, const CUtensorMap* tmap_out) {
@@ -650,14 +675,11 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
       // per tile: apply the row factors to O (rare), clear the tail rows, release P V
       if (threadIdx.x == 0) ptx::mbar_arrive_expect_tx(l_full, 512);
       constexpr int kS = L::kPSlots;
-      const uint32_t score_stg0 = ptx::map_peer(ptx::smem_u32(smem + ScoreLayout::kOffBars + 8 * bar::kStgFree), 0);
       for (int j = 0; j < nt; ++j) {
         const int s = j % kS;
         if (threadIdx.x == 0) ptx::mbar_arrive_expect_tx(&p_full[s], L::kP + 512);   // 4 x (4 KB + 128 B)
         bool w = ptx::mbar_wait<true>(&p_full[s], (j / kS) & 1, kErrTimeoutPeer);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        // the score CTA may refill the staging slot this tile came from (only tiles it still waits on)
-        if (threadIdx.x == 0 && j < nt - 2) ptx::mbar_arrive_cluster_relaxed_addr(score_stg0 + 8 * (j & 1));
         const float f = reinterpret_cast<const float*>(smem + L::kOffSlots + s * L::kSlot + L::kOffF)[h];
         if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
           // O holds the products of tiles < j relative to the old reference: scale it
@@ -736,16 +758,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
 
   if (threadIdx.x == 0) {
     if (rank == 0) {
-      for (int s = 0; s < ScoreLayout::kUnits; ++s) {
+      for (int s = 0; s < ScoreLayout::kLatSlots; ++s) {
         ptx::mbar_init(&bars[bar::kUFull + s], 1);
         ptx::mbar_init(&bars[bar::kUEmpty + s], 1);
+      }
+      for (int s = 0; s < ScoreLayout::kPeSlots; ++s) {
+        ptx::mbar_init(&bars[bar::kPeFull + s], 1);
+        ptx::mbar_init(&bars[bar::kPeEmpty + s], 1);
       }
       for (int s = 0; s < 2; ++s) {
         ptx::mbar_init(&bars[bar::kSFull + s], 1);
         ptx::mbar_init(&bars[bar::kSFree + s], 128);
         ptx::mbar_init(&bars[bar::kMBar + s], 128);
         ptx::mbar_init(&bars[bar::kPSent + s], 4);
-        ptx::mbar_init(&bars[bar::kStgFree + s], 1);
       }
       for (int s = 0; s < ValueLayout::kPSlots; ++s) ptx::mbar_init(&bars[bar::kPFree + s], 1);
       ptx::mbar_init(&bars[bar::kQFull], 1);
@@ -823,8 +848,10 @@ __global__ void __launch_bounds__(kMergeThreads) merge_splits_kernel(const __nv_
                                                                  const float* __restrict__ part_ml, int num_splits,
                                                                  int64_t n_q, int heads,
                                                                  __nv_bfloat16* __restrict__ o_lat) {
-  ptx::griddep_wait();
+  // the next kernel may launch now: its set-up (and, for the output projection, its weight
+  // stream) overlaps this kernel, and it waits for this grid before reading o_lat
   ptx::griddep_launch_dependents();
+  ptx::griddep_wait();
   const int64_t warp_g = (int64_t)blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5);
   const int64_t pair = warp_g >> 1;
   if (pair >= n_q * heads) return;   // warp-uniform

@@ -69,7 +69,30 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
-  // set-up above touches no global memory; inputs may come from the previous kernel
+
+  // weight chunk i into stage s; the stage's barrier expects the weight and the activation bytes
+  auto load_w = [&](int i, int s) {
+    uint8_t* a = smem + s * L::kStage;
+    ptx::mbar_arrive_expect_tx(&full[s], L::kA + N_TILE * kProjBoxK * 2);
+    if (A_MN) {
+      // two 64(c) x 64(d) boxes: M elements 0..63 and 64..127 of this tile
+      const int c0 = m_tile * 128, row = w_row_base + h * w_rows_per_head + i * kProjBoxK;
+      ptx::tma_load_2d(a, &tmap_w, &full[s], c0, row);
+      ptx::tma_load_2d(a + L::kA / 2, &tmap_w, &full[s], c0 + 64, row);
+    } else {
+      // one 64(c) x 128(d) box: K elements i*64.., all 128 M rows
+      ptx::tma_load_2d(a, &tmap_w, &full[s], i * kProjBoxK, w_row_base + h * w_rows_per_head);
+    }
+  };
+  // The weights are never written by the kernels that may run before this one in the stream, so
+  // the first stages' weight copies start before the dependency wait and overlap the previous
+  // kernel's tail; the activations (the previous kernel's output) are read only after it.
+  const int early = warp == 0 ? (k_chunks < STAGES ? k_chunks : STAGES) : 0;
+  if (warp == 0) {
+    if (ptx::elect_one())
+      for (int i = 0; i < early; ++i) load_w(i, i);
+    __syncwarp();
+  }
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
 
@@ -78,23 +101,14 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(
     // producer: the whole warp loops, one elected lane issues
     for (int i = 0; i < k_chunks; ++i) {
       const int s = i % STAGES;
-      const bool w = ptx::mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, kErrTimeoutStageFree);
-      if (!__all_sync(0xffffffffu, w)) break;
-      if (ptx::elect_one()) {
-        uint8_t* a = smem + s * L::kStage;
-        uint8_t* b = a + L::kA;
-        ptx::mbar_arrive_expect_tx(&full[s], L::kA + N_TILE * kProjBoxK * 2);
-        if (A_MN) {
-          // two 64(c) x 64(d) boxes: M elements 0..63 and 64..127 of this tile
-          const int c0 = m_tile * 128, row = w_row_base + h * w_rows_per_head + i * kProjBoxK;
-          ptx::tma_load_2d(a, &tmap_w, &full[s], c0, row);
-          ptx::tma_load_2d(a + L::kA / 2, &tmap_w, &full[s], c0 + 64, row);
-        } else {
-          // one 64(c) x 128(d) box: K elements i*64.., all 128 M rows
-          ptx::tma_load_2d(a, &tmap_w, &full[s], i * kProjBoxK, w_row_base + h * w_rows_per_head);
-        }
-        ptx::tma_load_3d(b, &tmap_x, &full[s], i * kProjBoxK, h, n_tile * N_TILE);
+      if (i >= early) {
+        const bool w = ptx::mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, kErrTimeoutStageFree);
+        if (!__all_sync(0xffffffffu, w)) break;
+        if (ptx::elect_one()) load_w(i, s);
+        __syncwarp();
       }
+      if (ptx::elect_one())
+        ptx::tma_load_3d(smem + s * L::kStage + L::kA, &tmap_x, &full[s], i * kProjBoxK, h, n_tile * N_TILE);
       __syncwarp();
       issued = i + 1;
     }

@@ -284,13 +284,6 @@ __device__ __forceinline__ void st_async_b32(uint32_t remote_addr, uint32_t remo
                "r"(remote_bar), "r"(v)
                : "memory");
 }
-// Start pulling `bytes` (multiple of 16, 16-byte aligned address) of global
-// memory into L2; nothing waits for it.
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-               : "memory");
-}
-
 // Pin 32 registers filled by tcgen05.ld: the compiler must not read them before the
 // tcgen05.wait::ld that precedes this (it emits no instruction).
 __device__ __forceinline__ void reg_fence32(uint32_t* r) {

@@ -189,7 +189,12 @@ MLA_API mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* 
 
 /* Output projection: out[n,h,d] = sum_c o_lat[n,h,c] * wkv_b[h*(Dn+Dv)+Dn+d, c].
  * ("Absorb Path Execution", the last einsum, with the tail rows of wkv_b.)
- *   o_lat [n_rows, H, C] contiguous; out [n_rows, H, Dv] contiguous, written. */
+ *   o_lat [n_rows, H, C] contiguous; out [n_rows, H, Dv] contiguous, written.
+ * The tensor-core kernel may start while the previous kernel on the stream is
+ * still finishing (programmatic dependent launch, when that kernel allows it,
+ * as this library's attention calls do) and reads wkv_b before waiting for it:
+ * wkv_b must not be written by a kernel that allows its successor to start
+ * early.  o_lat is read only after the previous kernel has completed. */
 MLA_API mla_status_t mla_out_proj(const mla_dims_t* dims, const void* o_lat, const void* wkv_b, void* out,
                           int64_t n_rows, cudaStream_t stream);
 
