@@ -241,15 +241,16 @@ def main():
     bufs = {"q_abs": torch.empty((B, H, C), dtype=dt, device=dev),
             "o_lat": torch.empty((B, H, C), dtype=dt, device=dev),
             "out": torch.empty((B, H, Dv), dtype=dt, device=dev),
-            "ws": mla.workspace(d, B, B, max_k, 0, device=dev)}
+            "ws": mla.workspace(d, B, B, max_k, 0, device=dev),
+            "ws_out": mla.decode_out_workspace(d, B, max_k, 0, device=dev)}
     stream = torch.cuda.current_stream()
 
     def step(k):
-        # the whole hot path through the public calls: absorb -> attention (+ merge) -> output projection
+        # the whole hot path through the public calls: absorb, then attention (+ merge) and the
+        # output projection in one call (mla_attn_decode_out)
         q, kv, pe, wkv_b = inputs[k]
         q_abs = mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
-        o_lat = mla.attn_decode(d, q_abs, q, kv, pe, cu_k, max_k, bufs["o_lat"], bufs["ws"])
-        return mla.out_proj(d, o_lat, wkv_b, bufs["out"])
+        return mla.attn_decode_out(d, q_abs, q, kv, pe, cu_k, max_k, wkv_b, bufs["out"], bufs["ws_out"])
 
     def attention_call(k):
         q, kv, pe, _ = inputs[k]
@@ -365,9 +366,9 @@ def main():
             "kernel_family": mla.kernel_family(d),
             "kernel_source_hash": kernel_source_hash(),
         }
-        # absorb_q + attention + (merge when split) + out_proj, each one launch of ours
+        # absorb_q + attention + output projection (with the split merge fused in), one launch each
         splits = mla.decode_num_splits(d, B, max_k, 0)
-        line["gpu_launches"] = args.steps * (3 + (1 if splits > 1 else 0))
+        line["gpu_launches"] = args.steps * 3
         line["config"]["num_splits"] = splits
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_oracle(w, args.cpu_seconds)

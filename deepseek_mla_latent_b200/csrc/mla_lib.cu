@@ -286,6 +286,56 @@ mla_status_t mla_attn_decode_static_scratch(const mla_dims_t* dims, const void* 
                          stream);
 }
 
+size_t mla_decode_out_workspace_size(const mla_dims_t* dims, int32_t batch, int64_t max_seqlen_k,
+                                     int32_t num_splits) {
+  Geo g;
+  if (!dims || !geo_of(dims, &g) || batch < 0 || max_seqlen_k < 0 || num_splits < 0 || num_splits > 256) return 0;
+  const int splits = resolve_splits(g, batch, batch, max_seqlen_k, num_splits, true);
+  const size_t o_lat_bytes = align256((size_t)batch * g.H * g.C * (g.bf16 ? 2 : 4));
+  return o_lat_bytes + workspace_bytes_for(g, batch, batch, max_seqlen_k, splits, true);
+}
+
+mla_status_t mla_attn_decode_out(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
+                                 const void* kv_cache, const void* pe_cache, int64_t kv_rows,
+                                 const int32_t* cu_seqlens_k, int32_t batch, int64_t max_seqlen_k,
+                                 const void* wkv_b, void* out, void* workspace, size_t workspace_bytes,
+                                 int32_t num_splits, cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (batch < 0 || max_seqlen_k < 0 || kv_rows < 0 || num_splits < 0 || num_splits > 256 ||
+      q_row_stride < (int64_t)g.H * (g.Dn + g.R))
+    return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!q_abs || !q || !cu_seqlens_k || !wkv_b || !out || !aligned16(q_abs) || !aligned16(q) ||
+      !aligned16(wkv_b) || !aligned16(out))
+    return MLA_ERR_INVALID_ARG;
+  if (kv_rows > 0 && (!kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
+    return MLA_ERR_INVALID_ARG;
+  const size_t need = mla_decode_out_workspace_size(dims, batch, max_seqlen_k, num_splits);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return MLA_ERR_WORKSPACE;
+  // o_lat first, then the attention call's own workspace
+  const size_t o_lat_bytes = align256((size_t)batch * g.H * g.C * (g.bf16 ? 2 : 4));
+  void* o_lat = workspace;
+  void* ws = static_cast<char*>(workspace) + o_lat_bytes;
+  const size_t ws_bytes = workspace_bytes - o_lat_bytes;
+  if (g.family == 1) {
+    if ((q_row_stride * 2) % 16 != 0) return MLA_ERR_INVALID_ARG;
+    const int splits = resolve_splits(g, batch, batch, max_seqlen_k, num_splits, true);
+    // with splits the merge runs inside the projection kernel and o_lat is never written
+    mla_status_t st = mla::sm100::attention(q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, nullptr,
+                                            cu_seqlens_k, batch, batch, g.H, splits, g.scale, o_lat, ws, stream,
+                                            /*merge=*/splits <= 1);
+    if (st != MLA_OK) return st;
+    if (splits > 1) return mla::sm100::merge_out_proj(ws, splits, batch, g.H, wkv_b, out, stream);
+    return mla::sm100::out_proj(o_lat, wkv_b, out, batch, g.H, stream);
+  }
+  mla_status_t st = mla_attn_decode(dims, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_k, batch,
+                                    max_seqlen_k, o_lat, ws, ws_bytes, num_splits, stream);
+  if (st != MLA_OK) return st;
+  return mla_out_proj(dims, o_lat, wkv_b, out, batch, stream);
+}
+
 mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
                                     const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch,
                                     int64_t n_q_rows, int64_t max_seqlen_q, int64_t max_seqlen_k,

@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "mla.h"
 #include "sm100_attn.cuh"
+#include "sm100_merge_proj.cuh"
 #include "sm100_proj.cuh"
 
 namespace mla {
@@ -179,9 +180,17 @@ inline size_t workspace_bytes(int H, int64_t n_q, int splits) {
   return align256((size_t)splits * n_q * H * 512 * 2) + align256((size_t)splits * n_q * H * 2 * sizeof(float));
 }
 
+// Split partials in the workspace: bf16 O [splits, n_q, H, 512], then fp32 (m, l) [splits, n_q, H, 2].
+inline size_t partial_ml_offset(int H, int64_t n_q, int splits) {
+  return align256((size_t)splits * n_q * H * 512 * 2);
+}
+
+// merge = false (split runs only): leave the partials in the workspace for merge_out_proj
+// instead of merging them into o_lat.
 inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_stride, const void* kv, const void* pe,
                               int64_t kv_rows, const int32_t* cu_q, const int32_t* cu_k, int batch, int64_t n_q,
-                              int H, int splits, float scale, void* o_lat, void* ws, cudaStream_t stream) {
+                              int H, int splits, float scale, void* o_lat, void* ws, cudaStream_t stream,
+                              bool merge = true) {
   if (kv_rows >= (1LL << 31) || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
   const int64_t units = n_q * (H / 128) * splits;
   if (units == 0) return MLA_OK;
@@ -234,10 +243,11 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_lat = static_cast<__nv_bfloat16*>(o_lat);
   p.part_ml = nullptr;
+
   __nv_bfloat16* part_o = nullptr;
   if (splits > 1) {
     part_o = static_cast<__nv_bfloat16*>(ws);
-    p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)splits * n_q * H * 512 * 2));
+    p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + partial_ml_offset(H, n_q, splits));
   }
   p.out = splits > 1 ? part_o : static_cast<__nv_bfloat16*>(o_lat);
   CUtensorMap tout;
@@ -251,12 +261,30 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   if (!set_smem(latent_attn_kernel, kAttnSmem)) return MLA_ERR_CUDA;
   mla_status_t st = launch(true, latent_attn_kernel, dim3((unsigned)(2 * units)), dim3(kAttnThreads), kAttnSmem,
                            stream, tkv_s, tpe, tqpe, tkv_v, tqa, tout, p);
-  if (st != MLA_OK || splits <= 1) return st;
+  if (st != MLA_OK || splits <= 1 || !merge) return st;
   const int64_t pairs_per_block = kMergeThreads / 64;   // two warps per (row, head)
   const int64_t merge_blocks = (n_q * H + pairs_per_block - 1) / pairs_per_block;
   return launch(true, merge_splits_kernel, dim3((unsigned)merge_blocks), dim3(kMergeThreads), 0, stream,
                 (const __nv_bfloat16*)part_o, (const float*)p.part_ml, splits, n_q, H,
                 static_cast<__nv_bfloat16*>(o_lat));
+}
+
+// The output projection of a split decode with the split merge fused in: out [n_q, H, 128] from the
+// partials an attention(..., merge = false) call left in ws.
+inline mla_status_t merge_out_proj(const void* ws, int splits, int64_t n_q, int H, const void* wkv_b, void* out,
+                                   cudaStream_t stream) {
+  if (splits < 2 || splits > kMpMaxSplits || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  CUtensorMap tw;
+  const uint64_t wd[2] = {512, (uint64_t)H * 256}, wst[1] = {1024};
+  const uint32_t wb[2] = {64, 128};  // 64 latent columns x 128 value rows (K-major A)
+  if (!make_map(&tw, wkv_b, 2, wd, wst, wb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  constexpr size_t smem = merge_proj_smem_bytes();
+  if (!set_smem(merge_proj_kernel, smem)) return MLA_ERR_CUDA;
+  const auto* part_o = static_cast<const __nv_bfloat16*>(ws);
+  const auto* part_ml = reinterpret_cast<const float*>(static_cast<const char*>(ws) + partial_ml_offset(H, n_q, splits));
+  return launch(true, merge_proj_kernel, dim3((unsigned)H, (unsigned)((n_q + kMpRows - 1) / kMpRows)),
+                dim3(kMergeProjThreads), smem, stream, tw, part_o, part_ml, splits, (int)n_q, H,
+                static_cast<__nv_bfloat16*>(out));
 }
 
 }  // namespace sm100

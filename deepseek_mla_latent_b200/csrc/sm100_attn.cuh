@@ -844,6 +844,29 @@ __device__ __forceinline__ void merge_acc(float (&a)[8], float w, const uint4& x
   }
 }
 
+// The merge weights of one (row, head) as a warp computes them: lane s < 32 returns the weight
+// 2^(m_s - M) of split s (0 for a split with no key); M = max_s m_s and inv = 1 / sum_s w_s l_s
+// (0 when no split saw a key).  ml points at the (m, l) pair of split 0, split_stride pairs apart.
+// Both consumers of the partials (merge_splits_kernel, merge_proj_kernel) use this, so they
+// produce bit-identical o_lat rows.
+__device__ __forceinline__ float merge_weights(const float2* ml, int64_t split_stride, int num_splits, int lane,
+                                               float& M_out, float& inv_out) {
+  const float2 mine = lane < num_splits ? __ldcg(ml + lane * split_stride) : make_float2(-INFINITY, 0.f);
+  float M = mine.x;
+  for (int s = lane + 32; s < num_splits; s += 32) M = fmaxf(M, __ldcg(ml + s * split_stride).x);
+  M = warp_max(M);
+  const float w_lane = mine.x == -INFINITY ? 0.f : exp2f(mine.x - M);
+  float L = w_lane * mine.y;
+  for (int s = lane + 32; s < num_splits; s += 32) {
+    const float2 x = __ldcg(ml + s * split_stride);
+    if (x.x != -INFINITY) L += exp2f(x.x - M) * x.y;
+  }
+  L = warp_sum(L);
+  M_out = M;
+  inv_out = L > 0.f ? 1.f / L : 0.f;
+  return w_lane;
+}
+
 __global__ void __launch_bounds__(kMergeThreads) merge_splits_kernel(const __nv_bfloat16* __restrict__ part_o,
                                                                  const float* __restrict__ part_ml, int num_splits,
                                                                  int64_t n_q, int heads,
@@ -864,18 +887,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_splits_kernel(const __nv_
   for (int s = 0; s < kMergeInFlight; ++s)
     if (s < num_splits) v[s] = __ldcg(src + s * step);
   const float2* ml = reinterpret_cast<const float2*>(part_ml) + pair;
-  const float2 mine = lane < num_splits ? __ldcg(ml + lane * split_stride) : make_float2(-INFINITY, 0.f);
-  float M = mine.x;
-  for (int s = lane + 32; s < num_splits; s += 32) M = fmaxf(M, __ldcg(ml + s * split_stride).x);
-  M = warp_max(M);
-  const float w_lane = mine.x == -INFINITY ? 0.f : exp2f(mine.x - M);   // the weight of split `lane`
-  float L = w_lane * mine.y;
-  for (int s = lane + 32; s < num_splits; s += 32) {
-    const float2 x = __ldcg(ml + s * split_stride);
-    if (x.x != -INFINITY) L += exp2f(x.x - M) * x.y;
-  }
-  L = warp_sum(L);
-  const float inv = L > 0.f ? 1.f / L : 0.f;
+  float M, inv;
+  const float w_lane = merge_weights(ml, split_stride, num_splits, lane, M, inv);   // the weight of split `lane`
   float a[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) a[i] = 0.f;

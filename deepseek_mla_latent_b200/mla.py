@@ -109,6 +109,41 @@ def attn_decode(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, kv: torch.Tens
     return o_lat
 
 
+def decode_out_workspace(d: MlaDims, batch: int, max_seqlen_k: int, num_splits: int = 0,
+                         device="cuda") -> torch.Tensor:
+    nbytes = int(LIB.mla_decode_out_workspace_size(ctypes.byref(d), batch, max_seqlen_k, num_splits))
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def attn_decode_out(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, kv: torch.Tensor, pe: torch.Tensor,
+                    cu_seqlens_k: torch.Tensor, max_seqlen_k: int, wkv_b: torch.Tensor,
+                    out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, num_splits: int = 0,
+                    stream=None) -> torch.Tensor:
+    """Decode attention and the output projection in one call (mla_attn_decode_out)."""
+    dt = _dtype(d)
+    batch = cu_seqlens_k.numel() - 1
+    H, C, R = d.num_heads, d.kv_lora_rank, d.qk_rope_head_dim
+    rs = _q_row_stride(q, d)
+    _need(q_abs, "q_abs", dt, (batch, H, C))
+    _need(q, "q", dt, contiguous=False)
+    _need(kv, "kv", dt)
+    _need(pe, "pe", dt)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    _need(wkv_b, "wkv_b", dt, (H * (d.qk_nope_head_dim + d.v_head_dim), C))
+    if kv.dim() != 2 or kv.shape[1] != C or pe.dim() != 2 or pe.shape[1] != R or pe.shape[0] != kv.shape[0]:
+        raise ValueError("kv must be [T, C] and pe [T, R]")
+    if out is None:
+        out = torch.empty((batch, H, d.v_head_dim), dtype=dt, device=q_abs.device)
+    _need(out, "out", dt, (batch, H, d.v_head_dim))
+    if ws is None:
+        ws = decode_out_workspace(d, batch, max_seqlen_k, num_splits, device=q_abs.device)
+    _check(LIB.mla_attn_decode_out(ctypes.byref(d), _ptr(q_abs), _ptr(q), rs, _ptr(kv), _ptr(pe), kv.shape[0],
+                                   _ptr(cu_seqlens_k), batch, int(max_seqlen_k), _ptr(wkv_b), _ptr(out), _ptr(ws),
+                                   ws.numel(), num_splits, _stream(stream)),
+           "mla_attn_decode_out")
+    return out
+
+
 def attn_prefill_chunk(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
                        cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int, kv: torch.Tensor,
                        pe: torch.Tensor, o_lat: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
@@ -164,14 +199,15 @@ def device_status(stream=None) -> int:
 def decode_step(d: MlaDims, q: torch.Tensor, wkv_b: torch.Tensor, kv: torch.Tensor, pe: torch.Tensor,
                 cu_seqlens_k: torch.Tensor, max_seqlen_k: int, num_splits: int = 0, bufs: Optional[dict] = None,
                 stream=None) -> torch.Tensor:
-    """The whole absorb decode path: mla_absorb_q -> mla_attn_decode -> mla_out_proj.
+    """The whole absorb decode path: mla_absorb_q -> mla_attn_decode_out (attention, then the
+    output projection, with the projection's weights staged into L2 during the attention tail).
 
-    ``bufs`` may hold preallocated "q_abs", "o_lat", "out", "ws" tensors."""
+    ``bufs`` may hold preallocated "q_abs", "out" and "ws_out" (mla_decode_out_workspace_size
+    bytes) tensors."""
     bufs = bufs or {}
     q_abs = absorb_q(d, q, wkv_b, bufs.get("q_abs"), stream)
-    o_lat = attn_decode(d, q_abs, q, kv, pe, cu_seqlens_k, max_seqlen_k, bufs.get("o_lat"), bufs.get("ws"),
-                        num_splits, stream)
-    return out_proj(d, o_lat, wkv_b, bufs.get("out"), stream)
+    return attn_decode_out(d, q_abs, q, kv, pe, cu_seqlens_k, max_seqlen_k, wkv_b, bufs.get("out"),
+                           bufs.get("ws_out"), num_splits, stream)
 
 
 def prefill_step(d: MlaDims, q: torch.Tensor, wkv_b: torch.Tensor, kv: torch.Tensor, pe: torch.Tensor,

@@ -140,6 +140,30 @@ MLA_API mla_status_t mla_attn_decode(const mla_dims_t* dims, const void* q_abs, 
                              void* o_lat, void* workspace, size_t workspace_bytes,
                              int32_t num_splits, cudaStream_t stream);
 
+/* Bytes of workspace mla_attn_decode_out needs (num_splits as there; 0 = automatic). */
+MLA_API size_t mla_decode_out_workspace_size(const mla_dims_t* dims, int32_t batch, int64_t max_seqlen_k,
+                                             int32_t num_splits);
+
+/* Decode attention followed by the output projection in one call:
+ *   out[b,h,d] = sum_c o_lat[b,h,c] * wkv_b[h*(Dn+Dv)+Dn+d, c]
+ * with o_lat as mla_attn_decode computes it ("Absorb Path Execution": the
+ * score and latent value einsums, then the last einsum).  Arguments as in
+ * mla_attn_decode, except:
+ *   wkv_b      [H*(Dn+Dv), C], the same matrix mla_absorb_q and mla_out_proj take.
+ *   out        [batch, H, Dv] contiguous, written.
+ *   workspace  at least mla_decode_out_workspace_size(dims, batch, max_seqlen_k,
+ *              num_splits) bytes, 16-byte aligned; o_lat lives there and is not
+ *              returned.  Contents on entry are ignored.
+ * The result equals mla_attn_decode followed by mla_out_proj, bit for bit.
+ * On the tensor-core path with more than one split, the split merge runs
+ * inside the projection kernel: o_lat never goes to memory and one kernel
+ * launch is saved.  The wkv_b rule of mla_out_proj applies. */
+MLA_API mla_status_t mla_attn_decode_out(const mla_dims_t* dims, const void* q_abs, const void* q,
+                                         int64_t q_row_stride, const void* kv_cache, const void* pe_cache,
+                                         int64_t kv_rows, const int32_t* cu_seqlens_k, int32_t batch,
+                                         int64_t max_seqlen_k, const void* wkv_b, void* out, void* workspace,
+                                         size_t workspace_bytes, int32_t num_splits, cudaStream_t stream);
+
 /* Size of the device scratch array behind mla_attn_decode_static_scratch. */
 #define MLA_STATIC_SCRATCH_BYTES (32u << 20)
 

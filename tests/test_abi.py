@@ -102,3 +102,18 @@ def test_workspace_is_checked(lib):
     assert L.mla_workspace_size(ctypes.byref(d), 2, 2, 1 << 16, 1) == 0
     v3 = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
     assert L.mla_workspace_size(ctypes.byref(v3), 8, 8, 4096, 0) >= 0
+
+
+def test_decode_out_host_checks(lib):
+    L = lib.LIB
+    d = lib.make_dims(8, 64, 32, 16, 32, "f32", 0.1)
+    need = L.mla_decode_out_workspace_size(ctypes.byref(d), 2, 1 << 16, 4)
+    # o_lat [2, 8, 64] fp32 plus the split partials of the attention call
+    assert need >= 2 * 8 * 64 * 4 + L.mla_workspace_size(ctypes.byref(d), 2, 2, 1 << 16, 4)
+    args = lambda ws, wsb, wkv_b=A: (ctypes.byref(d), A, A, 384, A, A, 1 << 17, A, 2, 1 << 16, wkv_b, A, ws, wsb, 4, None)
+    assert L.mla_attn_decode_out(*args(A, need - 16)) == lib.MLA_ERR_WORKSPACE
+    assert L.mla_attn_decode_out(*args(None, need)) == lib.MLA_ERR_WORKSPACE
+    assert L.mla_attn_decode_out(*args(A, need, wkv_b=None)) == lib.MLA_ERR_INVALID_ARG
+    assert L.mla_attn_decode_out(ctypes.byref(d), None, None, 384, None, None, 0, None, 0, 0, None, None, None, 0, 0,
+                                 None) == lib.MLA_OK
+    assert L.mla_decode_out_workspace_size(ctypes.byref(d), 2, 1 << 16, 300) == 0

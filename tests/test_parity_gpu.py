@@ -111,3 +111,39 @@ def test_full_long_context_sampled():
 
 def test_full_prefill_sampled():
     _sampled(4, [(0, 3), (3, 120)])
+
+
+def _decode_out(w, num_splits=0):
+    d = mla.dims_from(w.dims)
+    dev = to_dev(w)
+    q_abs = mla.absorb_q(d, dev["q"], dev["wkv_b"])
+    out = mla.attn_decode_out(d, q_abs, dev["q"], dev["kv"], dev["pe"], dev["cu_k"], dev["max_k"], dev["wkv_b"],
+                              num_splits=num_splits)
+    mla.device_status()
+    return out.float().cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("seqlens,splits", [([1, 200, 777], 0), ([4096, 33], 0), ([1000, 260], 7), ([0, 70, 0], 0)])
+def test_v3_decode_out_matches_oracle_and_the_two_calls(seqlens, splits):
+    """mla_attn_decode_out against the oracle, and bit for bit against mla_attn_decode + mla_out_proj
+    (the same kernels on the same inputs)."""
+    w = wl.make_workload("v3o", V3, [1] * len(seqlens), seqlens, seed=9)
+    got = _decode_out(w, splits)
+    assert_close(got, oracle.workload_naive(w), "bf16", "out")
+    two = run_path(w, num_splits=splits)["out"]
+    assert np.array_equal(got, two)
+
+
+def test_fp32_decode_out():
+    w = wl.make_workload("f32o", wl.TINY, [1, 1], [300, 5], seed=10)
+    assert_close(_decode_out(w), oracle.workload_naive(w), "f32", "out")
+
+
+def test_full_v3_decode_out_sampled():
+    """The benchmark's launch configuration (mla_attn_decode_out at the full V3 decode size),
+    checked on (sequence, head) pairs the oracle computes one by one."""
+    w = wl.workload(1)
+    got = _decode_out(w)
+    ref = oracle.workload_naive(w, pairs=[(0, 0), (5, 64), (7, 127)])
+    for (b, h), r in ref.items():
+        assert_close(got[b:b + 1, h, :], r, "bf16", f"seq {b} head {h}")
