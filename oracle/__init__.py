@@ -1,6 +1,7 @@
 """fp64 CPU oracle for MLA attention (test infrastructure only; see mla_oracle)."""
 from .mla_oracle import (head_view, visible_keys, softmax_rows, naive_head, mla_naive, mla_absorb,
                          workload_naive, workload_absorb)
+from .append_oracle import rms_norm, rope_interleaved, append_latent
 
 __all__ = ["head_view", "visible_keys", "softmax_rows", "naive_head", "mla_naive", "mla_absorb",
-           "workload_naive", "workload_absorb"]
+           "workload_naive", "workload_absorb", "rms_norm", "rope_interleaved", "append_latent"]
