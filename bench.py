@@ -53,6 +53,9 @@ def parse_args():
     p.add_argument("--workload", type=int, default=1, help="workload index (1 = DeepSeek-V3 decode b8 t4096)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
+    p.add_argument("--op", choices=["decode", "append"], default="decode",
+                   help="decode: the decode step (the benchmark); append: the latent-cache append alone")
+    p.add_argument("--tokens", type=int, default=65536, help="new tokens per append call (--op append)")
     return p.parse_args()
 
 
@@ -210,11 +213,73 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_append(args, rank, world):
+    """Time mla_append_latent (RMSNorm of the latent, RoPE of the rotary key, slot writes) on
+    `--tokens` new tokens of the DeepSeek-V3 shapes; one JSON line (single GPU)."""
+    import torch
+    from deepseek_mla_latent_b200 import mla
+    from deepseek_mla_latent_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    n, C, R = args.tokens, 512, 64
+    d = mla.dims_from(wl.V3)
+    g = torch.Generator(device="cpu").manual_seed(0)
+    dev = "cuda"
+    copies = 2 if n * (C + R) * 2 * 2 > L2_BYTES else min(16, max(2, math.ceil(2 * L2_BYTES / (n * (C + R) * 4))))
+    bufs = []
+    for _ in range(copies):
+        kv_new = torch.randn(n, C, generator=g).to(dev, torch.bfloat16)
+        pe_new = torch.randn(n, R, generator=g).to(dev, torch.bfloat16)
+        kvc = torch.empty(n, C, dtype=torch.bfloat16, device=dev)
+        pec = torch.empty(n, R, dtype=torch.bfloat16, device=dev)
+        bufs.append((kv_new, pe_new, kvc, pec))
+    gamma = torch.ones(C, dtype=torch.bfloat16, device=dev)
+    pos = (torch.arange(n, dtype=torch.int32) % 4096).to(dev)
+    slots = torch.randperm(n, generator=g).to(dev)
+    call = lambda k: mla.append_latent(d, bufs[k][0], bufs[k][1], pos, slots, bufs[k][2], bufs[k][3], gamma)
+    for i in range(max(3, args.warmup)):
+        call(i % copies)
+    graphs = []
+    for k in range(copies):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            call(k)
+        torch.cuda.current_stream().wait_stream(side)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            call(k)
+        graphs.append(gr)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        graphs[i % copies].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    mla.device_status()
+    us = e0.elapsed_time(e1) / args.steps * 1e3
+    alg_bytes = n * (C + R) * 2 * 2 + C * 2 + n * (4 + 8)
+    hbm, _, peak_kind = load_peaks()
+    gbs = alg_bytes / (us * 1e-6) / 1e9
+    print(json.dumps({
+        "metric": "MLA latent-cache append GB/s (1xB200)", "value": gbs, "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "us_per_call": us, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"append_v3_{n}_tokens", "tokens": n, "kv_lora_rank": C, "qk_rope": R,
+                   "l2": f"{copies} rotating input/cache copies"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "peak_kind": peak_kind},
+        "gpu_launches": args.steps}), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.op == "append":
+        run_append(args, rank, world)
         return
 
     import torch

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <type_traits>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -12,6 +14,7 @@
 #include "mla.h"
 #include "common.cuh"
 #include "simt.cuh"
+#include "append.cuh"
 #include "sm100.cuh"
 
 namespace {
@@ -367,6 +370,55 @@ mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* q_abs, c
                                     cu_seqlens_k, batch, n_q_rows, splits, o_lat, workspace, stream);
   return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, cu_seqlens_k,
                                batch, n_q_rows, splits, o_lat, workspace, stream);
+}
+
+mla_status_t mla_append_latent(const mla_dims_t* dims, const void* kv_new, const void* k_pe_new, const void* gamma,
+                               float eps, float rope_base, const int32_t* positions, const int64_t* slots,
+                               int64_t n_tokens, void* kv_cache, void* pe_cache, int64_t cache_rows,
+                               cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  const int vec = g.bf16 ? 8 : 4;
+  if (g.C % vec != 0 || g.C > mla::append::kMaxC || g.R % 2 != 0 || g.R > 64 * mla::append::kMaxPairsPerLane)
+    return MLA_ERR_UNSUPPORTED;
+  if (n_tokens < 0 || cache_rows < 0 || !(eps >= 0.f && eps < INFINITY) || !(rope_base > 0.f && rope_base < INFINITY))
+    return MLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MLA_OK;
+  if (!kv_new || !k_pe_new || !positions || !slots || !kv_cache || !pe_cache || !aligned16(kv_new) ||
+      !aligned16(kv_cache) || (gamma && !aligned16(gamma)))
+    return MLA_ERR_INVALID_ARG;
+  const int64_t per_block = (int64_t)mla::append::kWarpsPerBlock * mla::append::kTokensPerWarp;
+  const int64_t nblocks = (n_tokens + per_block - 1) / per_block;
+  if (nblocks >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  const unsigned blocks = (unsigned)nblocks;
+  const double log2_base = std::log2((double)rope_base);
+  const dim3 block(mla::append::kWarpsPerBlock * 32);
+  auto go = [&](auto type_tag, auto per_lane) {
+    using T = decltype(type_tag);
+    constexpr int P = decltype(per_lane)::value;
+    mla::append::append_kernel<T, P><<<blocks, block, 0, stream>>>(
+        static_cast<const T*>(kv_new), static_cast<const T*>(k_pe_new), static_cast<const T*>(gamma), eps,
+        log2_base, positions, slots, n_tokens, g.C, g.R, static_cast<T*>(kv_cache), static_cast<T*>(pe_cache),
+        cache_rows);
+  };
+  // 16-byte vectors per lane: bf16 rows hold 8 elements per vector, fp32 rows 4
+  const int per_lane = (g.C / vec + 31) / 32;
+  using I1 = std::integral_constant<int, 1>;
+  using I2 = std::integral_constant<int, 2>;
+  using I4 = std::integral_constant<int, 4>;
+  using I8 = std::integral_constant<int, 8>;
+  if (g.bf16) {
+    if (per_lane <= 1) go(mla_bf16{}, I1{});
+    else if (per_lane <= 2) go(mla_bf16{}, I2{});
+    else go(mla_bf16{}, I4{});
+  } else {
+    if (per_lane <= 1) go(0.f, I1{});
+    else if (per_lane <= 2) go(0.f, I2{});
+    else if (per_lane <= 4) go(0.f, I4{});
+    else go(0.f, I8{});
+  }
+  return launch_status();
 }
 
 mla_status_t mla_device_status(cudaStream_t stream, uint32_t* code_out) {

@@ -188,6 +188,31 @@ def out_proj(d: MlaDims, o_lat: torch.Tensor, wkv_b: torch.Tensor, out: Optional
     return out
 
 
+def append_latent(d: MlaDims, kv_new: torch.Tensor, k_pe_new: torch.Tensor, positions: torch.Tensor,
+                  slots: torch.Tensor, kv_cache: torch.Tensor, pe_cache: torch.Tensor,
+                  gamma: Optional[torch.Tensor] = None, eps: float = 1e-6, rope_base: float = 10000.0,
+                  stream=None) -> None:
+    """Write normalised latents and rotated rotary keys of new tokens into the caches (mla_append_latent)."""
+    dt = _dtype(d)
+    n = kv_new.shape[0]
+    C, R = d.kv_lora_rank, d.qk_rope_head_dim
+    _need(kv_new, "kv_new", dt, (n, C))
+    _need(k_pe_new, "k_pe_new", dt, (n, R))
+    _need(positions, "positions", torch.int32, (n,))
+    _need(slots, "slots", torch.int64, (n,))
+    _need(kv_cache, "kv_cache", dt)
+    _need(pe_cache, "pe_cache", dt)
+    if kv_cache.dim() != 2 or kv_cache.shape[1] != C or pe_cache.dim() != 2 or pe_cache.shape[1] != R or \
+            pe_cache.shape[0] != kv_cache.shape[0]:
+        raise ValueError("kv_cache must be [T, C] and pe_cache [T, R]")
+    if gamma is not None:
+        _need(gamma, "gamma", dt, (C,))
+    _check(LIB.mla_append_latent(ctypes.byref(d), _ptr(kv_new), _ptr(k_pe_new), _ptr(gamma), float(eps),
+                                 float(rope_base), _ptr(positions), _ptr(slots), n, _ptr(kv_cache), _ptr(pe_cache),
+                                 kv_cache.shape[0], _stream(stream)),
+           "mla_append_latent")
+
+
 def device_status(stream=None) -> int:
     """Synchronise the stream and raise MlaError if a device wait ran out; returns the error word."""
     word = ctypes.c_uint32(0)

@@ -222,6 +222,26 @@ MLA_API mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* 
 MLA_API mla_status_t mla_out_proj(const mla_dims_t* dims, const void* o_lat, const void* wkv_b, void* out,
                           int64_t n_rows, cudaStream_t stream);
 
+/* Append new tokens to the latent caches ("Absorb Implementation Cache Design":
+ * kv_cache holds the compressed key-value vector, pe_cache the rotary key;
+ * "Latent KV expansion with split": the compressed KV is RMS-normalised):
+ *   kv_cache[slots[n], c] = kv_new[n, c] / sqrt(mean_c(kv_new[n]^2) + eps) * gamma[c]
+ *   pe_cache[slots[n], 2i]   = a cos t - b sin t      (a, b) = k_pe_new[n, 2i], k_pe_new[n, 2i+1]
+ *   pe_cache[slots[n], 2i+1] = a sin t + b cos t      t = positions[n] * rope_base^(-2i/R)
+ *   kv_new      [n_tokens, C], k_pe_new [n_tokens, R] (before normalisation / rotation).
+ *   gamma       [C] RMSNorm gain, or NULL for 1.
+ *   eps         >= 0; rope_base > 0 (10000 for DeepSeek-V3).
+ *   positions   device int32 [n_tokens]: the token's index in its sequence.
+ *   slots       device int64 [n_tokens]: destination row of both caches; a slot
+ *               outside [0, cache_rows) is skipped.  Slots must be distinct.
+ *   kv_cache    [cache_rows, C], pe_cache [cache_rows, R], updated in place.
+ * Needs C a multiple of 8 (bf16) or 4 (fp32), C <= 1024, R even, R <= 128;
+ * other dims return MLA_ERR_UNSUPPORTED. */
+MLA_API mla_status_t mla_append_latent(const mla_dims_t* dims, const void* kv_new, const void* k_pe_new,
+                                       const void* gamma, float eps, float rope_base, const int32_t* positions,
+                                       const int64_t* slots, int64_t n_tokens, void* kv_cache, void* pe_cache,
+                                       int64_t cache_rows, cudaStream_t stream);
+
 /* Static text for a status code. */
 MLA_API const char* mla_status_string(mla_status_t status);
 

@@ -117,3 +117,18 @@ def test_decode_out_host_checks(lib):
     assert L.mla_attn_decode_out(ctypes.byref(d), None, None, 384, None, None, 0, None, 0, 0, None, None, None, 0, 0,
                                  None) == lib.MLA_OK
     assert L.mla_decode_out_workspace_size(ctypes.byref(d), 2, 1 << 16, 300) == 0
+
+
+def test_append_host_checks(lib):
+    L = lib.LIB
+    v3 = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
+    f = lambda *a: L.mla_append_latent(ctypes.byref(v3), *a)
+    assert f(A, A, None, 1e-6, 10000.0, A, A, 0, None, None, 0, None) == lib.MLA_OK            # nothing to write
+    assert f(A, A, None, 1e-6, 10000.0, A, A, -1, A, A, 8, None) == lib.MLA_ERR_INVALID_ARG    # negative count
+    assert f(A, A, None, -1.0, 10000.0, A, A, 4, A, A, 8, None) == lib.MLA_ERR_INVALID_ARG     # eps < 0
+    assert f(A, A, None, 1e-6, 0.0, A, A, 4, A, A, 8, None) == lib.MLA_ERR_INVALID_ARG         # base <= 0
+    assert f(A, A, None, 1e-6, 10000.0, None, A, 4, A, A, 8, None) == lib.MLA_ERR_INVALID_ARG  # no positions
+    assert f(A + 8, A, None, 1e-6, 10000.0, A, A, 4, A, A, 8, None) == lib.MLA_ERR_INVALID_ARG  # misaligned
+    odd = lib.make_dims(128, 500, 128, 64, 128, "bf16", 0.07)   # C not a multiple of 8
+    assert L.mla_append_latent(ctypes.byref(odd), A, A, None, 1e-6, 10000.0, A, A, 4, A, A, 8, None) \
+        == lib.MLA_ERR_UNSUPPORTED
