@@ -358,30 +358,30 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
         ptx::tc_fence_after();
         const uint32_t s_col = tmem + lane_base + kColS + sb * kTileQ;
         const int n_valid = (int)min64(kTileQ, u.j_end - (u.j_begin + (int64_t)jj * kTileQ));
-        // row max of the raw scores over the valid keys (scale >= 0 commutes with max); S stays in
-        // TMEM and is read 64 columns at a time, here and again for the exponentials, so few
-        // registers are live and the exponentials of a row can be issued back to back
+        // S comes out of TMEM in one round trip (all 128 columns) and the buffer is handed back at
+        // once, so that QK(jj+2) is not held up by the rest of this tile's softmax (the tensor
+        // core, and with it the release of the ring slots, would otherwise wait on it)
+        uint32_t a[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&a[32 * c]));
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::reg_fence32(&a[32 * c]);
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&s_free[sb]);
+        // row max of the raw scores over the valid keys (scale >= 0 commutes with max)
         float mx;
         {
           float m8[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
-#pragma unroll 1
-          for (int c2 = 0; c2 < 2; ++c2) {
-            uint32_t a[64];
-            ptx::tmem_ld32(s_col + 64 * c2, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-            ptx::tmem_ld32(s_col + 64 * c2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-            ptx::tmem_wait_ld();
-            ptx::reg_fence32(&a[0]);
-            ptx::reg_fence32(&a[32]);
-            if (n_valid >= 64 * (c2 + 1)) {
+          if (n_valid >= kTileQ) {
 #pragma unroll
-              for (int i = 0; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(a[i]));
-            } else {
+            for (int i = 0; i < 128; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(a[i]));
+          } else {
 #pragma unroll
-              for (int i = 0; i < 64; ++i)
-                if (64 * c2 + i < n_valid) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(a[i]));
-            }
+            for (int i = 0; i < 128; ++i)
+              if (i < n_valid) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(a[i]));
           }
           mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
           mx *= sl2;
@@ -408,24 +408,12 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
         uint32_t pk[2][32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          if (half >= nh) break;
           float ps0 = 0.f, ps1 = 0.f;
-          uint32_t a[64];
-          ptx::tmem_ld32(s_col + kTileN * half, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-          ptx::tmem_ld32(s_col + kTileN * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-          ptx::tmem_wait_ld();
-          ptx::reg_fence32(&a[0]);
-          ptx::reg_fence32(&a[32]);
-          if (half == nh - 1) {
-            // the last read of this S buffer: QK(jj+2) may overwrite it
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&s_free[sb]);
-          }
           if (kTileN * (half + 1) <= n_valid) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float e0 = fast_exp2(fmaf(__uint_as_float(a[2 * i]), sl2, -m_new));
-              const float e1 = fast_exp2(fmaf(__uint_as_float(a[2 * i + 1]), sl2, -m_new));
+              const float e0 = fast_exp2(fmaf(__uint_as_float(a[64 * half + 2 * i]), sl2, -m_new));
+              const float e1 = fast_exp2(fmaf(__uint_as_float(a[64 * half + 2 * i + 1]), sl2, -m_new));
               ps0 += e0;
               ps1 += e1;
               pk[half][i] = ptx::pack_bf16x2(e0, e1);
@@ -434,8 +422,8 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int k = kTileN * half + 2 * i;
-              float e0 = fast_exp2(fmaf(__uint_as_float(a[2 * i]), sl2, -m_new));
-              float e1 = fast_exp2(fmaf(__uint_as_float(a[2 * i + 1]), sl2, -m_new));
+              float e0 = fast_exp2(fmaf(__uint_as_float(a[64 * half + 2 * i]), sl2, -m_new));
+              float e1 = fast_exp2(fmaf(__uint_as_float(a[64 * half + 2 * i + 1]), sl2, -m_new));
               if (k >= n_valid) e0 = 0.f;
               if (k + 1 >= n_valid) e1 = 0.f;
               ps0 += e0;
