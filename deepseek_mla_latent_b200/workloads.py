@@ -18,7 +18,7 @@ sizes from "Latent KV expansion with split", workload line):
 
 Random numbers come from numpy's Philox4x32-10 counter-based generator keyed
 by (seed, stream), one stream per tensor: q=1, kv=2, pe=3, wkv_b=4,
-sequence lengths=5.  For the bf16 workloads every value is rounded to bf16
+sequence lengths=5, page placement of a paged cache=6.  For the bf16 workloads every value is rounded to bf16
 (round to nearest even) before either side sees it, so the oracle receives
 the exact operand values the GPU does.
 
@@ -37,7 +37,7 @@ from typing import List, Optional
 
 import numpy as np
 
-STREAM_Q, STREAM_KV, STREAM_PE, STREAM_W, STREAM_LEN = 1, 2, 3, 4, 5
+STREAM_Q, STREAM_KV, STREAM_PE, STREAM_W, STREAM_LEN, STREAM_PAGES = 1, 2, 3, 4, 5, 6
 
 
 @dataclasses.dataclass(frozen=True)
@@ -190,3 +190,49 @@ def workload_shape(index: int, seed: int = 0):
 def workload(index: int, seed: int = 0) -> Workload:
     name, dims, sq, sk = workload_shape(index, seed)
     return make_workload(name, dims, sq, sk, seed=seed)
+
+
+@dataclasses.dataclass
+class PagedCache:
+    """A workload's cache laid out in pages (see ``paged_cache``)."""
+    page_size: int
+    kv_cache: np.ndarray     # float32 [num_pages * page_size, C]
+    pe_cache: np.ndarray     # float32 [num_pages * page_size, R]
+    block_table: np.ndarray  # int32 [batch, max_pages]; -1 past a sequence's last page
+    seqlens_k: np.ndarray    # int32 [batch]
+
+    @property
+    def num_pages(self) -> int:
+        return self.kv_cache.shape[0] // self.page_size
+
+
+def paged_cache(w: Workload, page_size: int, seed: int = 0, spare_pages: int = 0, extra_columns: int = 0,
+                fill: float = float("nan")) -> PagedCache:
+    """Scatter a workload's packed cache into pages placed at random (stream 6).
+
+    Sequence b's key j goes to row table[b, j // page_size] * page_size + j % page_size.  The
+    pages of all sequences plus ``spare_pages`` unused ones are a random permutation of the
+    page indices; rows no key occupies (the tail of each sequence's last page, spare pages)
+    hold ``fill``.  The block table has ``extra_columns`` more columns than the longest
+    sequence needs; every entry past a sequence's last page is -1.
+    """
+    if page_size <= 0:
+        raise ValueError("page_size must be positive")
+    need = [(t + page_size - 1) // page_size for t in w.seqlens_k]
+    num_pages = sum(need) + spare_pages
+    perm = _rng(seed, STREAM_PAGES).permutation(num_pages)
+    C, R = w.kv.shape[1], w.pe.shape[1]
+    kv = np.full((num_pages * page_size, C), fill, dtype=np.float32)
+    pe = np.full((num_pages * page_size, R), fill, dtype=np.float32)
+    table = np.full((w.batch, max(need + [0]) + extra_columns), -1, dtype=np.int32)
+    cu = w.cu_seqlens_k
+    nxt = 0
+    for b, t in enumerate(w.seqlens_k):
+        for pg in range(need[b]):
+            phys = int(perm[nxt])
+            nxt += 1
+            table[b, pg] = phys
+            j0, j1 = pg * page_size, min(t, (pg + 1) * page_size)
+            kv[phys * page_size: phys * page_size + (j1 - j0)] = w.kv[cu[b] + j0: cu[b] + j1]
+            pe[phys * page_size: phys * page_size + (j1 - j0)] = w.pe[cu[b] + j0: cu[b] + j1]
+    return PagedCache(page_size, kv, pe, table, np.asarray(w.seqlens_k, dtype=np.int32))
