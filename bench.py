@@ -53,9 +53,11 @@ def parse_args():
     p.add_argument("--workload", type=int, default=1, help="workload index (1 = DeepSeek-V3 decode b8 t4096)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
-    p.add_argument("--op", choices=["decode", "append"], default="decode",
-                   help="decode: the decode step (the benchmark); append: the latent-cache append alone")
+    p.add_argument("--op", choices=["decode", "append", "paged"], default="decode",
+                   help="decode: the decode step (the benchmark); append: the latent-cache append alone; "
+                        "paged: the decode attention call over a paged cache beside the packed one")
     p.add_argument("--tokens", type=int, default=65536, help="new tokens per append call (--op append)")
+    p.add_argument("--page-size", type=int, default=64, help="tokens per page (--op paged)")
     return p.parse_args()
 
 
@@ -272,6 +274,85 @@ def run_append(args, rank, world):
         "gpu_launches": args.steps}), flush=True)
 
 
+def run_paged(args, rank, world):
+    """Time the decode attention call (attention kernel + split merge) over the workload's cache
+    scattered into randomly placed pages (mla_attn_paged), and the packed call on the same keys;
+    one JSON line (single GPU)."""
+    import torch
+    from deepseek_mla_latent_b200 import mla
+    from deepseek_mla_latent_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    dev = "cuda"
+    w = wl.workload(args.workload)
+    if any(s != 1 for s in w.seqlens_q):
+        raise SystemExit("--op paged times decode workloads")
+    pc = wl.paged_cache(w, args.page_size, seed=0, spare_pages=64, fill=0.0)
+    d = mla.dims_from(w.dims)
+    dt = torch.bfloat16
+    B, H, C = w.batch, w.dims.heads, w.dims.kv_lora_rank
+    max_k = max(w.seqlens_k)
+    t = lambda a, ty=dt: torch.from_numpy(np.ascontiguousarray(a)).to(device=dev, dtype=ty)
+    per_copy = (pc.kv_cache.size + pc.pe_cache.size + w.kv.size + w.pe.size) * 2
+    copies = min(16, max(2, math.ceil(ROTATE_MIN_BYTES / per_copy) + 1))
+    q, wkv_b = t(w.q), t(w.wkv_b)
+    q_abs = mla.absorb_q(d, q, wkv_b)
+    table, seqlens, cu_k = t(pc.block_table, torch.int32), t(pc.seqlens_k, torch.int32), t(w.cu_seqlens_k, torch.int32)
+    caches = [(t(pc.kv_cache), t(pc.pe_cache), t(w.kv), t(w.pe)) for _ in range(copies)]
+    o_lat = torch.empty((B, H, C), dtype=dt, device=dev)
+    ws = mla.workspace(d, B, B, max_k, 0, device=dev)
+    paged = lambda k: mla.attn_paged(d, q_abs, q, seqlens, max_k, caches[k][0], caches[k][1], table, pc.page_size,
+                                     o_lat=o_lat, ws=ws)
+    packed = lambda k: mla.attn_decode(d, q_abs, q, caches[k][2], caches[k][3], cu_k, max_k, o_lat, ws)
+
+    def capture(fn):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        return gr
+
+    for i in range(max(3, args.warmup)):
+        paged(i % copies)
+        packed(i % copies)
+    mla.device_status()
+    g_paged = [capture(lambda k=k: paged(k)) for k in range(copies)]
+    g_packed = [capture(lambda k=k: packed(k)) for k in range(copies)]
+    for i in range(max(3, args.warmup)):
+        g_paged[i % copies].replay()
+        g_packed[i % copies].replay()
+    torch.cuda.synchronize()
+
+    def timed(graphs):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(args.steps):
+            graphs[i % copies].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps * 1e3
+
+    us_paged, us_packed = timed(g_paged), timed(g_packed)
+    mla.device_status()
+    hbm, _, peak_kind = load_peaks()
+    alg_bytes = w.total_k * KV_BYTES_PER_TOKEN + B * H * (C + w.dims.qk_rope + C) * 2
+    gbs = alg_bytes / (us_paged * 1e-6) / 1e9
+    print(json.dumps({
+        "metric": "MLA paged-cache decode attention GB/s (1xB200)", "value": gbs, "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "us_per_call": us_paged, "packed_us_per_call": us_packed,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}_page{pc.page_size}", "batch": B, "seq_len_k": max_k,
+                   "page_size": pc.page_size, "num_pages": pc.num_pages,
+                   "num_splits": mla.decode_num_splits(d, B, max_k, 0),
+                   "l2": f"{copies} rotating copies of the paged and packed caches"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "peak_kind": peak_kind},
+        "gpu_launches": args.steps * (2 if mla.decode_num_splits(d, B, max_k, 0) > 1 else 1)}), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_env()
@@ -280,6 +361,9 @@ def main():
         return
     if args.op == "append":
         run_append(args, rank, world)
+        return
+    if args.op == "paged":
+        run_paged(args, rank, world)
         return
 
     import torch

@@ -17,6 +17,7 @@ enum : uint32_t {
   kErrTimeoutPeer = 1u << 4,       // waited too long for the partner CTA's scores
   kErrTimeoutDrain = 1u << 5,      // exit path waited too long for copies in flight
   kErrBadSchedule = 1u << 6,       // a work item pointed outside its buffers
+  kErrBadPage = 1u << 7,           // a block-table entry of a page holding keys lies outside the cache
 };
 
 // One word per device; set with atomicOr, read and cleared by mla_device_status.

@@ -88,7 +88,8 @@ template <typename T>
 mla_status_t simt_attention(const Geo& g, const void* q_abs, const void* q, int64_t q_row_stride,
                             const void* kv, const void* pe, int64_t kv_rows, const int32_t* cu_q, const int32_t* cu_k,
                             int batch,
-                            int64_t n_rows, int splits, void* o_lat, void* ws, cudaStream_t stream) {
+                            int64_t n_rows, int splits, void* o_lat, void* ws, cudaStream_t stream,
+                            const mla::sm100::PagedKv& paged = mla::sm100::PagedKv{}) {
   float* part_o = nullptr;
   float* part_ml = nullptr;
   if (splits > 1) {
@@ -97,11 +98,11 @@ mla_status_t simt_attention(const Geo& g, const void* q_abs, const void* q, int6
                                        align256((size_t)splits * n_rows * g.H * g.C * sizeof(float)));
   }
   dim3 grid((unsigned)n_rows, g.H, splits);
-  size_t smem = (size_t)(2 * g.C + g.R + mla::simt::kThreads + 32) * sizeof(float);
+  const size_t smem = mla::simt::attn_smem_bytes(g.C, g.R);
   mla::simt::attn_kernel<T><<<grid, mla::simt::kThreads, smem, stream>>>(
       static_cast<const T*>(q_abs), static_cast<const T*>(q), q_row_stride, static_cast<const T*>(kv),
-      static_cast<const T*>(pe), kv_rows, cu_q, cu_k, batch, n_rows, g.H, g.C, g.R, g.Dn, g.scale, splits,
-      static_cast<T*>(o_lat), part_o, part_ml);
+      static_cast<const T*>(pe), kv_rows, cu_q, cu_k, batch, paged.seqlens, paged.table, paged.stride, paged.page,
+      n_rows, g.H, g.C, g.R, g.Dn, g.scale, splits, static_cast<T*>(o_lat), part_o, part_ml);
   if (splits > 1) {
     mla::simt::combine_kernel<T><<<dim3((unsigned)n_rows, g.H), mla::simt::kThreads, 0, stream>>>(
         part_o, part_ml, splits, n_rows, g.H, g.C, static_cast<T*>(o_lat));
@@ -370,6 +371,48 @@ mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* q_abs, c
                                     cu_seqlens_k, batch, n_q_rows, splits, o_lat, workspace, stream);
   return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, cu_seqlens_k,
                                batch, n_q_rows, splits, o_lat, workspace, stream);
+}
+
+mla_status_t mla_attn_paged(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
+                            const int32_t* cu_seqlens_q, int64_t n_q_rows, const int32_t* seqlens_k, int32_t batch,
+                            int64_t max_seqlen_k, const void* kv_cache, const void* pe_cache, int64_t num_pages,
+                            int32_t page_size, const int32_t* block_table, int64_t max_pages_per_seq, void* o_lat,
+                            void* workspace, size_t workspace_bytes, int32_t num_splits, cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  const bool decode = cu_seqlens_q == nullptr;
+  if (batch < 0 || n_q_rows < 0 || max_seqlen_k < 0 || num_pages < 0 || page_size <= 0 || max_pages_per_seq < 0 ||
+      num_splits < 0 || num_splits > 256 || q_row_stride < (int64_t)g.H * (g.Dn + g.R) ||
+      (decode && n_q_rows != batch) || (!decode && num_splits > 1))
+    return MLA_ERR_INVALID_ARG;
+  if (num_pages > (int64_t{1} << 40) / page_size) return MLA_ERR_INVALID_ARG;
+  const int64_t kv_rows = num_pages * page_size;
+  if (g.family == 1 && page_size % 64 != 0) return MLA_ERR_UNSUPPORTED;
+  if (batch == 0 || n_q_rows == 0) return MLA_OK;
+  if (!q_abs || !q || !seqlens_k || !block_table || !o_lat || !aligned16(q_abs) || !aligned16(q) ||
+      !aligned16(o_lat))
+    return MLA_ERR_INVALID_ARG;
+  if (kv_rows > 0 && (!kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
+    return MLA_ERR_INVALID_ARG;
+  const int splits = resolve_splits(g, batch, n_q_rows, max_seqlen_k, num_splits, decode);
+  const size_t need = workspace_bytes_for(g, batch, n_q_rows, max_seqlen_k, splits, decode);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return MLA_ERR_WORKSPACE;
+  mla::sm100::PagedKv paged;
+  paged.seqlens = seqlens_k;
+  paged.table = block_table;
+  paged.stride = max_pages_per_seq;
+  paged.page = page_size;
+  if (g.family == 1) {
+    if ((q_row_stride * 2) % 16 != 0) return MLA_ERR_INVALID_ARG;
+    return mla::sm100::attention(q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, nullptr, batch,
+                                 n_q_rows, g.H, splits, g.scale, o_lat, workspace, stream, true, paged);
+  }
+  if (g.bf16)
+    return simt_attention<mla_bf16>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, nullptr,
+                                    batch, n_q_rows, splits, o_lat, workspace, stream, paged);
+  return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, nullptr, batch,
+                               n_q_rows, splits, o_lat, workspace, stream, paged);
 }
 
 mla_status_t mla_append_latent(const mla_dims_t* dims, const void* kv_new, const void* k_pe_new, const void* gamma,

@@ -98,15 +98,26 @@ __device__ __forceinline__ float block_reduce_sum(float v, float* red) {
   return r;
 }
 
+// Shared memory of attn_kernel in bytes: floats q_abs [C], q_pe [R], o [C], p [kThreads],
+// reduction scratch [32], then the cache row of each key of a chunk (int64 [kThreads]).
+__host__ __device__ constexpr size_t attn_floats(int C, int R) { return ((size_t)2 * C + R + kThreads + 32 + 1) & ~(size_t)1; }
+__host__ __device__ constexpr size_t attn_smem_bytes(int C, int R) {
+  return attn_floats(C, R) * sizeof(float) + kThreads * sizeof(int64_t);
+}
+
 // Attention for one (query row, head, split) per block, online softmax over
 // 128-key chunks.  With num_splits == 1 the normalised result goes straight to
 // o_lat; otherwise the unnormalised partial (o, running max m, running sum l)
 // goes to the workspace for attn_combine_kernel.  Keys visible to query i of
-// a chunk of s over a cache of t: j < t - s + i + 1.
+// a chunk of s over a cache of t: j < t - s + i + 1.  The cache is packed
+// (sequence b's keys in rows cu_k[b] ..) or, with a block table, paged: key j
+// in row table[b][j / page] * page + j % page; a page outside the cache reads
+// as zeros and raises kErrBadPage.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) attn_kernel(
     const T* __restrict__ q_abs, const T* __restrict__ q, int64_t q_row_stride, const T* __restrict__ kv,
     const T* __restrict__ pe, int64_t kv_rows, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int batch,
+    const int* __restrict__ seqlens_k, const int* __restrict__ block_table, int64_t bt_stride, int page_size,
     int64_t n_rows, int H, int C, int R, int Dn, float scale, int num_splits, T* __restrict__ o_lat,
     float* __restrict__ part_o, float* __restrict__ part_ml) {
   extern __shared__ float sm[];
@@ -115,11 +126,20 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(
   float* o = qp + R;         // [C]
   float* p = o + C;          // [kThreads]
   float* red = p + kThreads; // [32]
+  int64_t* krow = reinterpret_cast<int64_t*>(sm + attn_floats(C, R));   // [kThreads], -1 = zero row
   const int64_t n = blockIdx.x;
   const int h = blockIdx.y, split = blockIdx.z;
   const int b = cu_q ? find_sequence(cu_q, batch, n) : (int)n;
-  const int64_t k0 = min64(max64(0, __ldg(cu_k + b)), kv_rows);
-  const int64_t t = max64(0, min64((int64_t)__ldg(cu_k + b + 1), kv_rows) - k0);
+  int64_t k0, t;
+  const int* bt = nullptr;
+  if (block_table) {
+    bt = block_table + (int64_t)b * bt_stride;
+    k0 = 0;
+    t = max64(0, min64((int64_t)__ldg(seqlens_k + b), bt_stride * page_size));
+  } else {
+    k0 = min64(max64(0, __ldg(cu_k + b)), kv_rows);
+    t = max64(0, min64((int64_t)__ldg(cu_k + b + 1), kv_rows) - k0);
+  }
   int64_t s = 1, i = 0;
   if (cu_q) {
     const int64_t q0 = __ldg(cu_q + b);
@@ -144,11 +164,20 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(
     const int64_t j = j0 + threadIdx.x;
     float sc = -INFINITY;
     if (j < j_end) {
-      const T* kr = kv + (k0 + j) * (int64_t)C;
-      const T* pr = pe + (k0 + j) * (int64_t)R;
+      int64_t row = k0 + j;
+      if (bt) {
+        const int e = __ldg(bt + j / page_size);
+        row = (e < 0 || ((int64_t)e + 1) * page_size > kv_rows) ? -1 : (int64_t)e * page_size + j % page_size;
+        if (row < 0) raise_error(kErrBadPage);
+      }
+      krow[threadIdx.x] = row;
       float acc = 0.f;
-      for (int c = 0; c < C; ++c) acc = fmaf(qa[c], Elem<T>::load(kr + c), acc);
-      for (int r = 0; r < R; ++r) acc = fmaf(qp[r], Elem<T>::load(pr + r), acc);
+      if (row >= 0) {
+        const T* kr = kv + row * (int64_t)C;
+        const T* pr = pe + row * (int64_t)R;
+        for (int c = 0; c < C; ++c) acc = fmaf(qa[c], Elem<T>::load(kr + c), acc);
+        for (int r = 0; r < R; ++r) acc = fmaf(qp[r], Elem<T>::load(pr + r), acc);
+      }
       sc = acc * scale;
     }
     const float cmax = block_reduce_max(sc, red);
@@ -162,8 +191,8 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(
     const int cnt = (int)min64(kThreads, j_end - j0);
     for (int c = threadIdx.x; c < C; c += kThreads) {
       float acc = o[c] * alpha;
-      const T* kc = kv + (k0 + j0) * (int64_t)C + c;
-      for (int jj = 0; jj < cnt; ++jj) acc = fmaf(p[jj], Elem<T>::load(kc + (int64_t)jj * C), acc);
+      for (int jj = 0; jj < cnt; ++jj)
+        if (krow[jj] >= 0) acc = fmaf(p[jj], Elem<T>::load(kv + krow[jj] * (int64_t)C + c), acc);
       o[c] = acc;
     }
     __syncthreads();

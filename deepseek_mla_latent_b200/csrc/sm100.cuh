@@ -185,12 +185,25 @@ inline size_t partial_ml_offset(int H, int64_t n_q, int splits) {
   return align256((size_t)splits * n_q * H * 512 * 2);
 }
 
+// Addressing of a paged cache: sequence b holds seqlens[b] keys, key j in row
+// table[b * stride + j / page] * page + j % page.  table == nullptr: packed cache (cu_k).
+struct PagedKv {
+  const int32_t* seqlens = nullptr;
+  const int32_t* table = nullptr;
+  int64_t stride = 0;
+  int page = 0;
+};
+
 // merge = false (split runs only): leave the partials in the workspace for merge_out_proj
 // instead of merging them into o_lat.
 inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_stride, const void* kv, const void* pe,
                               int64_t kv_rows, const int32_t* cu_q, const int32_t* cu_k, int batch, int64_t n_q,
                               int H, int splits, float scale, void* o_lat, void* ws, cudaStream_t stream,
-                              bool merge = true) {
+                              bool merge = true, const PagedKv& paged = PagedKv{}) {
+  if (paged.table && (paged.page <= 0 || paged.page % kTileN != 0 || !paged.seqlens || paged.stride < 0))
+    return MLA_ERR_INVALID_ARG;
+  // pages of 64 * odd keys: the score CTA copies 64 keys at a time
+  const uint32_t score_rows = paged.table && paged.page % kTileQ != 0 ? kTileN : kTileQ;
   if (kv_rows >= (1LL << 31) || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
   const int64_t units = n_q * (H / 128) * splits;
   if (units == 0) return MLA_OK;
@@ -203,17 +216,17 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   const void* pe_base = kv_rows > 0 ? pe : q_abs;
   {
     // the cache as [8 latent blocks][rows][64 columns] (block stride 128 bytes): the score CTA
-    // copies two 64-column blocks of 128 keys at a time, the value CTA a whole 64-key tile
-    // (eight blocks) at a time
+    // copies two 64-column blocks of 128 keys at a time (one block of 64 keys with 64 * odd
+    // pages), the value CTA a whole 64-key tile (eight blocks) at a time
     const uint64_t d3[3] = {64, rows, 8}, st3[2] = {1024, 128};
-    const uint32_t bs[3] = {64, (uint32_t)kTileQ, 2};
+    const uint32_t bs[3] = {64, score_rows, score_rows == kTileQ ? 2u : 1u};
     if (!make_map(&tkv_s, kv_base, 3, d3, st3, bs, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     const uint32_t bv[3] = {64, (uint32_t)kTileN, 8};
     if (!make_map(&tkv_v, kv_base, 3, d3, st3, bv, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
   {
     const uint64_t d[2] = {64, rows}, st[1] = {128};
-    const uint32_t b[2] = {64, (uint32_t)kTileQ};     // 64 rotary columns x 128 keys
+    const uint32_t b[2] = {64, score_rows};           // 64 rotary columns x 128 (or 64) keys
     if (!make_map(&tpe, pe_base, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
   {
@@ -234,6 +247,11 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   p.q_abs = static_cast<const __nv_bfloat16*>(q_abs);
   p.cu_q = cu_q;
   p.cu_k = cu_k;
+  p.seqlens_k = paged.seqlens;
+  p.block_table = paged.table;
+  p.bt_stride = paged.stride;
+  p.page_size = paged.page;
+  p.score_copy_rows = (int)score_rows;
   p.batch = batch;
   p.heads = H;
   p.head_groups = H / 128;

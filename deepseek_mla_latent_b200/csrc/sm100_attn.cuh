@@ -24,8 +24,8 @@
 // The score CTA never waits for the value CTA except for a free P slot (four
 // slots), so the pair forms a pipeline instead of exchanging partial scores
 // every tile.  Each CTA streams its own copy of the kv rows: the score CTA
-// from HBM (it also prefetches its key range into L2), the value CTA a little
-// later from L2, so HBM sees each cache byte once.  N = 128 matters: with one
+// from HBM, the value CTA a little later from L2, so HBM sees each cache byte
+// once.  N = 128 matters: with one
 // elected lane issuing, a 128 x 64 x 16 MMA takes 48 cycles where 32 would be
 // full rate, while N >= 128 runs at full rate.
 //
@@ -52,6 +52,14 @@
 // factors (and rescale O when one moved), zero the tail rows of the last
 // tile's values, and release the P V product; warp 8 loads, warp 9 issues
 // the MMAs and hands P slots back; warps 0-7 run the epilogue.
+//
+// The cache is packed (sequence b's keys in rows cu_k[b] ..) or paged: key j
+// of sequence b in row table[b][j / page] * page + j % page, pages of a
+// multiple of 64 keys ("What is DeepSeek Sparse Attention (DSA)?", section
+// "How DSA works (conceptual)": the serving runtime keeps the KV cache in
+// pages for continuous batching).  Paging changes only which rows the copies
+// start at (CacheRows); with pages of 64 * odd keys a 128-key score copy
+// becomes two 64-key copies.
 //
 // Every wait is bounded; a wait that runs out raises the device error word
 // and the thread takes its exit path.
@@ -112,7 +120,13 @@ static_assert(ValueLayout::kP + 1024 <= ValueLayout::kSlot, "P slot too small");
 struct AttnParams {
   const __nv_bfloat16* q_abs;   // [n_q, H, 512]
   const int* cu_q;              // [batch+1] for chunked prefill, nullptr for decode
-  const int* cu_k;              // [batch+1]
+  const int* cu_k;              // [batch+1] packed cache: first row of each sequence
+  const int* seqlens_k;         // [batch] paged cache: keys per sequence
+  const int* block_table;       // [batch, bt_stride] paged cache: page of each run of page_size keys;
+                                // nullptr for a packed cache
+  int64_t bt_stride;
+  int page_size;                // rows per page, a multiple of 64
+  int score_copy_rows;          // keys per score-side copy: 128, or 64 when pages are 64 * odd
   int batch;
   int heads;
   int head_groups;              // heads / 128
@@ -135,7 +149,7 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // its sequence (whose first cache row is k0); nt = number of 64-key P tiles.
 struct UnitRange {
   int64_t row, k0, j_begin, j_end;
-  int hg, sp, nt;
+  int b, hg, sp, nt;
 };
 
 __device__ __forceinline__ UnitRange unit_range(const AttnParams& p, int64_t unit) {
@@ -145,8 +159,17 @@ __device__ __forceinline__ UnitRange unit_range(const AttnParams& p, int64_t uni
   u.hg = (int)((unit % per_row) / p.num_splits);
   u.sp = (int)(unit % p.num_splits);
   const int b = p.cu_q ? find_sequence(p.cu_q, p.batch, u.row) : (int)u.row;
-  u.k0 = min64(max64(0, __ldg(p.cu_k + b)), p.kv_rows);
-  const int64_t t = max64(0, min64((int64_t)__ldg(p.cu_k + b + 1), p.kv_rows) - u.k0);
+  u.b = b;
+  int64_t t;
+  if (p.block_table) {
+    // keys are addressed through the block table (CacheRows); a sequence holds at most as
+    // many keys as its row of the table has pages for
+    u.k0 = 0;
+    t = max64(0, min64((int64_t)__ldg(p.seqlens_k + b), p.bt_stride * p.page_size));
+  } else {
+    u.k0 = min64(max64(0, __ldg(p.cu_k + b)), p.kv_rows);
+    t = max64(0, min64((int64_t)__ldg(p.cu_k + b + 1), p.kv_rows) - u.k0);
+  }
   int64_t visible = t;
   if (p.cu_q) {
     // query i of s new queries (aligned to the end of the cache) sees keys 0 .. t - s + i
@@ -161,6 +184,54 @@ __device__ __forceinline__ UnitRange unit_range(const AttnParams& p, int64_t uni
   u.nt = (int)((u.j_end - u.j_begin + kTileN - 1) / kTileN);
   return u;
 }
+
+// Cache row of each key a unit loads, for one warp whose lanes all ask for the same key, keys
+// non-decreasing from call to call.  Packed cache: the sequence's first row plus the key.
+// Paged cache: key j of sequence b sits in row table[b][j / page] * page + j % page.  Lane l
+// holds the table entry of page win + l, and the next 32 entries are already loading when the
+// window moves on, so the copies wait on the table only once, at the start.
+struct CacheRows {
+  const int* bt;        // the sequence's row of the block table, nullptr for a packed cache
+  int64_t base;         // packed cache: the sequence's first row
+  int64_t n_entries;    // entries in the table row
+  int64_t rows;         // cache rows
+  int64_t win;
+  int page, cur, nxt;
+
+  __device__ __forceinline__ int entry(int64_t i) const { return i < n_entries ? __ldg(bt + i) : -1; }
+
+  __device__ __forceinline__ void init(const AttnParams& p, const UnitRange& u, uint32_t lane) {
+    bt = p.block_table ? p.block_table + (int64_t)u.b * p.bt_stride : nullptr;
+    base = u.k0;
+    rows = p.kv_rows;
+    n_entries = p.bt_stride;
+    page = p.page_size;
+    if (bt) {
+      win = u.j_begin / page;
+      cur = entry(win + lane);
+      nxt = entry(win + 32 + lane);
+    }
+  }
+
+  // Row of key j (counted from the sequence's first key).  A page outside the cache gives row
+  // `rows`, past the end of the tensor maps, which the copies fill with zeros; when the page
+  // holds a key the unit attends to (j < j_end) the device error word records it.
+  __device__ __forceinline__ int row(int64_t j, int64_t j_end, uint32_t lane) {
+    if (!bt) return (int)(base + j);
+    const int64_t pg = j / page;
+    while (pg >= win + 32) {
+      cur = nxt;
+      win += 32;
+      nxt = entry(win + 32 + lane);
+    }
+    const int e = __shfl_sync(0xffffffffu, cur, (int)(pg - win));
+    if (e < 0 || ((int64_t)e + 1) * page > rows) {
+      if (j < j_end && lane == 0) raise_error(kErrBadPage);
+      return (int)rows;
+    }
+    return (int)((int64_t)e * page + j % page);
+  }
+};
 
 // Barrier slots (8 bytes each) in the 512-byte barrier area of either role.
 namespace bar {
@@ -197,7 +268,6 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
   const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id();
   const int ntp = u.nt;                        // 64-key P tiles
   const int ntq = (ntp + 1) / 2;               // 128-key score tiles
-  const int64_t key_base = u.k0 + u.j_begin;
   const int head0 = u.hg * 128;
 
   if (warp == kProducerWarp) {
@@ -213,16 +283,24 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
         ptx::tma_load_3d(smem + L::kOffQpe, tmap_qpe, q_full, 128, head0, (int)u.row);
       }
       __syncwarp();
+      CacheRows cache;
+      cache.init(p, u, lane);
+      // pages of 64 * odd keys: each 128-key tile is two 64-key copies (rows r0, r1) per block
+      const bool halves = p.score_copy_rows != kTileQ;
       bool ok = true;
       for (int jj = 0; ok && jj < ntq; ++jj) {
-        const int key = (int)(key_base + (int64_t)jj * kTileQ);
+        const int64_t j0 = u.j_begin + (int64_t)jj * kTileQ;
+        const int r0 = cache.row(j0, u.j_end, lane);
+        const int r1 = halves ? cache.row(j0 + kTileQ / 2, u.j_end, lane) : 0;
         // the rotary block of the tile
         const int ps = jj % L::kPeSlots;
         bool w = ptx::mbar_wait(&pe_empty[ps], ((jj / L::kPeSlots) & 1) ^ 1, kErrTimeoutStageFree);
         if (!__all_sync(0xffffffffu, w)) break;
         if (ptx::elect_one()) {
           ptx::mbar_arrive_expect_tx(&pe_full[ps], L::kBlock);
-          ptx::tma_load_2d(smem + L::kOffPe + ps * L::kBlock, tmap_pe, &pe_full[ps], 0, key);
+          uint8_t* dst = smem + L::kOffPe + ps * L::kBlock;
+          ptx::tma_load_2d(dst, tmap_pe, &pe_full[ps], 0, r0);
+          if (halves) ptx::tma_load_2d(dst + L::kBlock / 2, tmap_pe, &pe_full[ps], 0, r1);
         }
         __syncwarp();
         pe_issued = jj + 1;
@@ -236,7 +314,16 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           if (ptx::elect_one()) {
             ptx::mbar_arrive_expect_tx(&u_full[slot], L::kLat);
-            ptx::tma_load_3d(smem + slot * L::kLat, tmap_kv, &u_full[slot], 0, key, 2 * k);
+            uint8_t* dst = smem + slot * L::kLat;
+            if (!halves) {
+              ptx::tma_load_3d(dst, tmap_kv, &u_full[slot], 0, r0, 2 * k);
+            } else {
+              // 64 keys x 64 columns per copy; the 8 KB offsets keep the 128-byte swizzle phase
+              for (int blk = 0; blk < 2; ++blk) {
+                ptx::tma_load_3d(dst + blk * L::kBlock, tmap_kv, &u_full[slot], 0, r0, 2 * k + blk);
+                ptx::tma_load_3d(dst + blk * L::kBlock + L::kBlock / 2, tmap_kv, &u_full[slot], 0, r1, 2 * k + blk);
+              }
+            }
           }
           __syncwarp();
           lat_issued = li + 1;
@@ -557,7 +644,6 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
   uint64_t* idle = bars + bar::kValueIdle;
   const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id();
   const int nt = u.nt;
-  const int64_t key_base = u.k0 + u.j_begin;
 
   if (warp == kProducerWarp) {
     // ============================================================ producer
@@ -568,6 +654,8 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
         ptx::prefetch_tmap(tmap_out);
       }
       __syncwarp();
+      CacheRows cache;
+      cache.init(p, u, lane);
       // The first P tile arrives several microseconds in; loading values before then would only
       // add to the start-up burst on HBM (these rows reach L2 through the score CTA meanwhile).
       bool w0 = ptx::mbar_wait<true>(&p_full[0], 0, kErrTimeoutPeer);
@@ -575,8 +663,8 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
         const int st = j % L::kStages;
         const bool w = ptx::mbar_wait(&v_empty[st], ((j / L::kStages) & 1) ^ 1, kErrTimeoutStageFree);
         if (!__all_sync(0xffffffffu, w)) break;
+        const int key = cache.row(u.j_begin + (int64_t)j * kTileN, u.j_end, lane);
         if (ptx::elect_one()) {
-          const int key = (int)(key_base + (int64_t)j * kTileN);
           ptx::mbar_arrive_expect_tx(&v_full[st], L::kStage);
           // one copy for the whole tile: eight 64-column blocks of 64 keys (the map's third axis
           // steps through the latent blocks), laid out block after block

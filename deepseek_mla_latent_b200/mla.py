@@ -174,6 +174,45 @@ def attn_prefill_chunk(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, cu_seql
     return o_lat
 
 
+def attn_paged(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, seqlens_k: torch.Tensor, max_seqlen_k: int,
+               kv_cache: torch.Tensor, pe_cache: torch.Tensor, block_table: torch.Tensor, page_size: int,
+               cu_seqlens_q: Optional[torch.Tensor] = None, o_lat: Optional[torch.Tensor] = None,
+               ws: Optional[torch.Tensor] = None, num_splits: int = 0, stream=None) -> torch.Tensor:
+    """Attention over a paged cache (mla_attn_paged): decode when cu_seqlens_q is None, else a
+    chunked prefill.  kv_cache [num_pages * page_size, C], pe_cache [num_pages * page_size, R],
+    block_table int32 [batch, max_pages_per_seq], seqlens_k int32 [batch]."""
+    dt = _dtype(d)
+    batch = seqlens_k.numel()
+    n = q_abs.shape[0]
+    H, C, R = d.num_heads, d.kv_lora_rank, d.qk_rope_head_dim
+    rs = _q_row_stride(q, d)
+    _need(q_abs, "q_abs", dt, (n, H, C))
+    _need(q, "q", dt, contiguous=False)
+    _need(kv_cache, "kv_cache", dt)
+    _need(pe_cache, "pe_cache", dt)
+    _need(seqlens_k, "seqlens_k", torch.int32, (batch,))
+    _need(block_table, "block_table", torch.int32)
+    if cu_seqlens_q is not None:
+        _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, (batch + 1,))
+    if block_table.dim() != 2 or block_table.shape[0] != batch:
+        raise ValueError("block_table must be [batch, max_pages_per_seq]")
+    if (kv_cache.dim() != 2 or kv_cache.shape[1] != C or pe_cache.dim() != 2 or pe_cache.shape[1] != R
+            or pe_cache.shape[0] != kv_cache.shape[0] or page_size <= 0 or kv_cache.shape[0] % page_size != 0):
+        raise ValueError("kv_cache must be [num_pages * page_size, C] and pe_cache [num_pages * page_size, R]")
+    if o_lat is None:
+        o_lat = torch.empty((n, H, C), dtype=dt, device=q_abs.device)
+    _need(o_lat, "o_lat", dt, (n, H, C))
+    if ws is None:
+        ws = workspace(d, batch, n, max_seqlen_k, num_splits, device=q_abs.device)
+    wsb = ws.numel() if ws is not None else 0
+    _check(LIB.mla_attn_paged(ctypes.byref(d), _ptr(q_abs), _ptr(q), rs, _ptr(cu_seqlens_q), n, _ptr(seqlens_k),
+                              batch, int(max_seqlen_k), _ptr(kv_cache), _ptr(pe_cache),
+                              kv_cache.shape[0] // page_size, int(page_size), _ptr(block_table),
+                              block_table.shape[1], _ptr(o_lat), _ptr(ws), wsb, num_splits, _stream(stream)),
+           "mla_attn_paged")
+    return o_lat
+
+
 def out_proj(d: MlaDims, o_lat: torch.Tensor, wkv_b: torch.Tensor, out: Optional[torch.Tensor] = None,
              stream=None) -> torch.Tensor:
     dt = _dtype(d)

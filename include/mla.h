@@ -37,6 +37,8 @@
  *    as 0, and a query row that sees no key gets zeros.
  *  - Device-side waits are bounded.  A wait that runs out sets a device
  *    error word instead of trapping; mla_device_status reports it.
+ *  - mla_attn_paged reads the same caches through a block table instead
+ *    (pages of page_size tokens); its description gives the addressing.
  */
 #ifndef MLA_B200_H_
 #define MLA_B200_H_
@@ -210,6 +212,42 @@ MLA_API mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* 
                                     int64_t max_seqlen_q, int64_t max_seqlen_k,
                                     const void* kv_cache, const void* pe_cache, int64_t kv_rows, void* o_lat,
                                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Attention over a PAGED latent cache, decode or chunked prefill.
+ * ("What is DeepSeek Sparse Attention (DSA)?", section "How DSA works
+ * (conceptual)": the serving runtime keeps the KV cache in pages for
+ * continuous batching.)  Same arithmetic as mla_attn_decode (cu_seqlens_q
+ * NULL) and mla_attn_prefill_chunk (cu_seqlens_q given); only the addressing
+ * of the cache differs:
+ *   key j of sequence b sits in row  block_table[b * max_pages_per_seq + j / page_size]
+ *                                    * page_size + j % page_size
+ *   of kv_cache [num_pages * page_size, C] and pe_cache [num_pages * page_size, R].
+ *   seqlens_k        device int32 [batch]: keys of each sequence (the current
+ *                    token included); a length is capped at
+ *                    max_pages_per_seq * page_size.
+ *   block_table      device int32 [batch, max_pages_per_seq] row-major.  Only
+ *                    the entries of pages that hold keys are read.  Such an
+ *                    entry outside [0, num_pages) reads as a page of zeros and
+ *                    sets bit 1<<7 of the device error word (mla_device_status
+ *                    then returns MLA_ERR_DEVICE_TIMEOUT with that code).
+ *   page_size        > 0; the tensor-core kernels need a multiple of 64
+ *                    (others return MLA_ERR_UNSUPPORTED); multiples of 128
+ *                    copy twice as many keys per TMA transfer.
+ *   cu_seqlens_q     NULL for decode (one query per sequence, n_q_rows ==
+ *                    batch), else as for mla_attn_prefill_chunk (then
+ *                    num_splits must be 0 or 1).
+ *   max_seqlen_k     host upper bound of the key counts (plans the splits).
+ *   o_lat            [n_q_rows, H, C] written.
+ *   workspace        at least mla_workspace_size(dims, batch, n_q_rows,
+ *                    max_seqlen_k, num_splits) bytes.
+ * num_pages * page_size must stay below 2^31 for the tensor-core kernels. */
+MLA_API mla_status_t mla_attn_paged(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
+                                    const int32_t* cu_seqlens_q, int64_t n_q_rows, const int32_t* seqlens_k,
+                                    int32_t batch, int64_t max_seqlen_k, const void* kv_cache,
+                                    const void* pe_cache, int64_t num_pages, int32_t page_size,
+                                    const int32_t* block_table, int64_t max_pages_per_seq, void* o_lat,
+                                    void* workspace, size_t workspace_bytes, int32_t num_splits,
+                                    cudaStream_t stream);
 
 /* Output projection: out[n,h,d] = sum_c o_lat[n,h,c] * wkv_b[h*(Dn+Dv)+Dn+d, c].
  * ("Absorb Path Execution", the last einsum, with the tail rows of wkv_b.)

@@ -132,3 +132,29 @@ def test_append_host_checks(lib):
     odd = lib.make_dims(128, 500, 128, 64, 128, "bf16", 0.07)   # C not a multiple of 8
     assert L.mla_append_latent(ctypes.byref(odd), A, A, None, 1e-6, 10000.0, A, A, 4, A, A, 8, None) \
         == lib.MLA_ERR_UNSUPPORTED
+
+
+def test_paged_host_checks(lib):
+    L = lib.LIB
+    d = lib.make_dims(8, 64, 32, 16, 32, "f32", 0.1)
+    v3 = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
+    need = L.mla_workspace_size(ctypes.byref(d), 2, 2, 1 << 12, 4)
+
+    def call(dims=d, cu_q=None, n_q=2, seqlens=A, batch=2, num_pages=64, page=64, table=A, stride=64,
+             ws=A, wsb=need, splits=4):
+        return L.mla_attn_paged(ctypes.byref(dims), A, A, 384, cu_q, n_q, seqlens, batch, 1 << 12, A, A, num_pages,
+                                page, table, stride, A, ws, wsb, splits, None)
+
+    assert call(batch=0, n_q=0) == lib.MLA_OK
+    assert call(page=0) == lib.MLA_ERR_INVALID_ARG
+    assert call(num_pages=-1) == lib.MLA_ERR_INVALID_ARG
+    assert call(stride=-1) == lib.MLA_ERR_INVALID_ARG
+    assert call(table=None) == lib.MLA_ERR_INVALID_ARG
+    assert call(seqlens=None) == lib.MLA_ERR_INVALID_ARG
+    assert call(n_q=3) == lib.MLA_ERR_INVALID_ARG                 # decode has one query per sequence
+    assert call(cu_q=A, n_q=5, splits=4) == lib.MLA_ERR_INVALID_ARG  # prefill takes no splits
+    assert call(ws=None) == lib.MLA_ERR_WORKSPACE
+    assert call(wsb=need - 16) == lib.MLA_ERR_WORKSPACE
+    # the tensor-core kernels copy 64-key tiles: smaller pages are not built for them
+    assert L.mla_attn_paged(ctypes.byref(v3), A, A, 128 * 192, None, 2, A, 2, 1 << 12, A, A, 64, 32, A, 128, A,
+                            A, 1 << 30, 0, None) == lib.MLA_ERR_UNSUPPORTED
