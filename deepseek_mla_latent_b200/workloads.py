@@ -18,7 +18,8 @@ sizes from "Latent KV expansion with split", workload line):
 
 Random numbers come from numpy's Philox4x32-10 counter-based generator keyed
 by (seed, stream), one stream per tensor: q=1, kv=2, pe=3, wkv_b=4,
-sequence lengths=5, page placement of a paged cache=6.  For the bf16 workloads every value is rounded to bf16
+sequence lengths=5, page placement of a paged cache=6, RMSNorm gain of the
+expansion inputs=7.  For the bf16 workloads every value is rounded to bf16
 (round to nearest even) before either side sees it, so the oracle receives
 the exact operand values the GPU does.
 
@@ -37,7 +38,7 @@ from typing import List, Optional
 
 import numpy as np
 
-STREAM_Q, STREAM_KV, STREAM_PE, STREAM_W, STREAM_LEN, STREAM_PAGES = 1, 2, 3, 4, 5, 6
+STREAM_Q, STREAM_KV, STREAM_PE, STREAM_W, STREAM_LEN, STREAM_PAGES, STREAM_GAMMA = 1, 2, 3, 4, 5, 6, 7
 
 
 @dataclasses.dataclass(frozen=True)
@@ -236,3 +237,29 @@ def paged_cache(w: Workload, page_size: int, seed: int = 0, spare_pages: int = 0
             kv[phys * page_size: phys * page_size + (j1 - j0)] = w.kv[cu[b] + j0: cu[b] + j1]
             pe[phys * page_size: phys * page_size + (j1 - j0)] = w.pe[cu[b] + j0: cu[b] + j1]
     return PagedCache(page_size, kv, pe, table, np.asarray(w.seqlens_k, dtype=np.int32))
+
+
+@dataclasses.dataclass
+class ExpandInputs:
+    """Inputs of the latent KV expansion (see ``expand_inputs``)."""
+    dims: Dims
+    batch: int
+    seq_len: int
+    kv_c: np.ndarray       # float32 [batch * seq_len, C], before RMSNorm
+    gamma: np.ndarray      # float32 [C]
+    wkv_b: np.ndarray      # float32 [H * (Dn + Dv), C]
+
+
+def expand_inputs(dims: Dims, batch: int, seq_len: int, seed: int = 0) -> ExpandInputs:
+    """Compressed KV rows before normalisation: N(0,1) rows times a per-row scale 2^U(-2, 2)
+    (so the RMSNorm matters), gain 1 + N(0, 0.1^2), wkv_b N(0, 0.02^2) (bf16-rounded for bf16)."""
+    n, C = batch * seq_len, dims.kv_lora_rank
+    rng = _rng(seed, STREAM_KV)
+    kv = rng.standard_normal((n, C), dtype=np.float32) * np.exp2(rng.uniform(-2, 2, (n, 1))).astype(np.float32)
+    gamma = (1.0 + 0.1 * _rng(seed, STREAM_GAMMA).standard_normal(C)).astype(np.float32)
+    w = _rng(seed, STREAM_W).standard_normal((dims.heads * (dims.qk_nope + dims.v_head), C),
+                                             dtype=np.float32) * np.float32(0.02)
+    if dims.dtype == "bf16":
+        kv, gamma, w = (round_to_bf16(a) for a in (kv, gamma, w))
+    return ExpandInputs(dims, batch, seq_len, np.ascontiguousarray(kv), np.ascontiguousarray(gamma),
+                        np.ascontiguousarray(w))
