@@ -53,9 +53,12 @@ def parse_args():
     p.add_argument("--workload", type=int, default=1, help="workload index (1 = DeepSeek-V3 decode b8 t4096)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
-    p.add_argument("--op", choices=["decode", "append", "paged"], default="decode",
+    p.add_argument("--op", choices=["decode", "append", "paged", "expand"], default="decode",
                    help="decode: the decode step (the benchmark); append: the latent-cache append alone; "
-                        "paged: the decode attention call over a paged cache beside the packed one")
+                        "paged: the decode attention call over a paged cache beside the packed one; "
+                        "expand: the latent KV expansion")
+    p.add_argument("--batch", type=int, default=4, help="sequences per expansion call (--op expand)")
+    p.add_argument("--seq-len", type=int, default=1024, help="tokens per sequence (--op expand)")
     p.add_argument("--tokens", type=int, default=65536, help="new tokens per append call (--op append)")
     p.add_argument("--page-size", type=int, default=64, help="tokens per page (--op paged)")
     return p.parse_args()
@@ -353,6 +356,66 @@ def run_paged(args, rank, world):
         "gpu_launches": args.steps * (2 if mla.decode_num_splits(d, B, max_k, 0) > 1 else 1)}), flush=True)
 
 
+def run_expand(args, rank, world):
+    """Time mla_expand_kv (RMSNorm of the compressed KV, projection to all heads, head-major
+    split into K_nope and V) at DeepSeek-V3 shapes; one JSON line (single GPU)."""
+    import torch
+    from deepseek_mla_latent_b200 import mla
+    from deepseek_mla_latent_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    dev = "cuda"
+    B, S = args.batch, args.seq_len
+    e = wl.expand_inputs(wl.V3, B, S, seed=0)
+    d = mla.dims_from(wl.V3)
+    H, C = wl.V3.heads, wl.V3.kv_lora_rank
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device=dev, dtype=torch.bfloat16)
+    n = B * S
+    out_bytes = n * H * 256 * 2
+    # outputs above L2 evict the inputs between calls; below it, rotate enough copies
+    copies = 2 if out_bytes > L2_BYTES else min(16, max(2, math.ceil(2 * L2_BYTES / out_bytes)))
+    sets = [(t(e.kv_c), t(e.wkv_b), torch.empty((B, H, S, 128), dtype=torch.bfloat16, device=dev),
+             torch.empty((B, H, S, 128), dtype=torch.bfloat16, device=dev)) for _ in range(copies)]
+    gamma = t(e.gamma)
+    call = lambda k: mla.expand_kv(d, sets[k][0], sets[k][1], B, S, gamma=gamma, k_nope=sets[k][2], v=sets[k][3])
+    for i in range(max(3, args.warmup)):
+        call(i % copies)
+    mla.device_status()
+    graphs = []
+    for k in range(copies):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            call(k)
+        torch.cuda.current_stream().wait_stream(side)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            call(k)
+        graphs.append(gr)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        graphs[i % copies].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    mla.device_status()
+    us = e0.elapsed_time(e1) / args.steps * 1e3
+    flop = 2.0 * n * H * 256 * C
+    alg_bytes = n * C * 2 + H * 256 * C * 2 + C * 2 + out_bytes
+    hbm, tf_burst, peak_kind = load_peaks()   # the burst bf16 figure: a kernel timed alone
+    tflops = flop / (us * 1e-6) / 1e12
+    print(json.dumps({
+        "metric": "MLA latent KV expansion TFLOP/s (1xB200)", "value": tflops, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "us_per_call": us, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"expand_v3_b{B}_s{S}", "batch": B, "seq_len": S, "heads": H, "kv_lora_rank": C,
+                   "l2": f"{copies} rotating input/output sets ({out_bytes / 2**20:.0f} MiB written per call)"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_burst, "unit": "TFLOP/s",
+                     "frac": tflops / tf_burst, "peak_kind": peak_kind + " (burst)",
+                     "hbm_gbs": alg_bytes / (us * 1e-6) / 1e9, "hbm_frac": alg_bytes / (us * 1e-6) / 1e9 / hbm},
+        "gpu_launches": args.steps}), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_env()
@@ -364,6 +427,9 @@ def main():
         return
     if args.op == "paged":
         run_paged(args, rank, world)
+        return
+    if args.op == "expand":
+        run_expand(args, rank, world)
         return
 
     import torch

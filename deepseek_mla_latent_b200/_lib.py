@@ -40,6 +40,7 @@ SIGNATURES = {
     "mla_attn_paged": (_I32, [_DP, _P, _P, _I64, _P, _I64, _P, _I32, _I64, _P, _P, _I64, _I32, _P, _I64, _P, _P,
                               _SZ, _I32, _P]),
     "mla_out_proj": (_I32, [_DP, _P, _P, _P, _I64, _P]),
+    "mla_expand_kv": (_I32, [_DP, _P, _P, ctypes.c_float, _P, _I64, _I64, _P, _P, _P]),
     "mla_append_latent": (_I32, [_DP, _P, _P, _P, ctypes.c_float, ctypes.c_float, _P, _P, _I64, _P, _P, _I64, _P]),
     "mla_status_string": (ctypes.c_char_p, [_I32]),
     "mla_device_status": (_I32, [_P, ctypes.POINTER(ctypes.c_uint32)]),

@@ -415,6 +415,37 @@ mla_status_t mla_attn_paged(const mla_dims_t* dims, const void* q_abs, const voi
                                n_q_rows, splits, o_lat, workspace, stream, paged);
 }
 
+mla_status_t mla_expand_kv(const mla_dims_t* dims, const void* kv_c, const void* gamma, float eps,
+                           const void* wkv_b, int64_t batch, int64_t seq_len, void* k_nope, void* v,
+                           cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (batch < 0 || seq_len < 0 || !(eps >= 0.f && eps < INFINITY)) return MLA_ERR_INVALID_ARG;
+  if (batch > 0 && seq_len > ((int64_t)1 << 40) / batch) return MLA_ERR_INVALID_ARG;
+  const int64_t n_tokens = batch * seq_len;
+  if (n_tokens == 0) return MLA_OK;
+  if (!kv_c || !wkv_b || !k_nope || !v || !aligned16(kv_c) || !aligned16(wkv_b) || !aligned16(k_nope) ||
+      !aligned16(v) || (gamma && !aligned16(gamma)))
+    return MLA_ERR_INVALID_ARG;
+  if (g.family == 1)
+    return mla::sm100::expand_kv(kv_c, gamma, eps, wkv_b, batch, seq_len, g.H, k_nope, v, device_sm_count(),
+                                 stream);
+  if (n_tokens >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  const dim3 grid((unsigned)n_tokens, g.H);
+  const size_t smem = (size_t)(g.C + 32) * sizeof(float);
+  if (g.bf16)
+    mla::simt::expand_kernel<mla_bf16><<<grid, mla::simt::kThreads, smem, stream>>>(
+        static_cast<const mla_bf16*>(kv_c), static_cast<const mla_bf16*>(gamma), eps,
+        static_cast<const mla_bf16*>(wkv_b), seq_len, g.H, g.C, g.Dn, g.Dv, static_cast<mla_bf16*>(k_nope),
+        static_cast<mla_bf16*>(v));
+  else
+    mla::simt::expand_kernel<float><<<grid, mla::simt::kThreads, smem, stream>>>(
+        static_cast<const float*>(kv_c), static_cast<const float*>(gamma), eps, static_cast<const float*>(wkv_b),
+        seq_len, g.H, g.C, g.Dn, g.Dv, static_cast<float*>(k_nope), static_cast<float*>(v));
+  return launch_status();
+}
+
 mla_status_t mla_append_latent(const mla_dims_t* dims, const void* kv_new, const void* k_pe_new, const void* gamma,
                                float eps, float rope_base, const int32_t* positions, const int64_t* slots,
                                int64_t n_tokens, void* kv_cache, void* pe_cache, int64_t cache_rows,

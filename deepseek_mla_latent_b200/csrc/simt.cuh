@@ -239,5 +239,39 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(
   }
 }
 
+// Latent KV expansion for one (token, head) per block: x = kv_c[tok] / sqrt(mean(kv_c[tok]^2) + eps)
+// * gamma, then the head's Dn key rows and Dv value rows of wkv_b against x.  Outputs
+// [batch, H, seq_len, Dn] and [batch, H, seq_len, Dv]; grid (tokens, H), 128 threads,
+// shared memory (C + 32) floats.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) expand_kernel(
+    const T* __restrict__ kv_c, const T* __restrict__ gamma, float eps, const T* __restrict__ wkv_b,
+    int64_t seq_len, int H, int C, int Dn, int Dv, T* __restrict__ k_nope, T* __restrict__ v) {
+  extern __shared__ float xs[];   // [C]
+  float* red = xs + C;            // [32]
+  const int64_t tok = blockIdx.x;
+  const int h = blockIdx.y;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < C; c += kThreads) {
+    const float x = Elem<T>::load(kv_c + tok * C + c);
+    xs[c] = x;
+    ss = fmaf(x, x, ss);
+  }
+  ss = block_reduce_sum(ss, red);
+  const float r = rsqrtf(ss / (float)C + eps);
+  for (int c = threadIdx.x; c < C; c += kThreads) xs[c] *= r * (gamma ? Elem<T>::load(gamma + c) : 1.f);
+  __syncthreads();
+  const int64_t b = tok / seq_len, s = tok % seq_len;
+  const T* w = wkv_b + (int64_t)h * (Dn + Dv) * C;
+  for (int d = threadIdx.x; d < Dn + Dv; d += kThreads) {
+    float acc = 0.f;
+    for (int c = 0; c < C; ++c) acc = fmaf(xs[c], Elem<T>::load(w + (int64_t)d * C + c), acc);
+    if (d < Dn)
+      Elem<T>::store(k_nope + ((b * H + h) * seq_len + s) * Dn + d, acc);
+    else
+      Elem<T>::store(v + ((b * H + h) * seq_len + s) * Dv + (d - Dn), acc);
+  }
+}
+
 }  // namespace simt
 }  // namespace mla

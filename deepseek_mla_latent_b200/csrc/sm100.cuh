@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "mla.h"
 #include "sm100_attn.cuh"
+#include "sm100_expand.cuh"
 #include "sm100_merge_proj.cuh"
 #include "sm100_proj.cuh"
 
@@ -303,6 +304,40 @@ inline mla_status_t merge_out_proj(const void* ws, int splits, int64_t n_q, int 
   return launch(true, merge_proj_kernel, dim3((unsigned)H, (unsigned)((n_q + kMpRows - 1) / kMpRows)),
                 dim3(kMergeProjThreads), smem, stream, tw, part_o, part_ml, splits, (int)n_q, H,
                 static_cast<__nv_bfloat16*>(out));
+}
+
+// Latent KV expansion: K_nope and V [batch, H, seq_len, 128] from kv_c [batch * seq_len, 512].
+inline mla_status_t expand_kv(const void* kv_c, const void* gamma, float eps, const void* wkv_b, int64_t batch,
+                              int64_t seq_len, int H, void* k_nope, void* v, int sms, cudaStream_t stream) {
+  const int64_t n_tokens = batch * seq_len;
+  if (n_tokens == 0) return MLA_OK;
+  if (n_tokens >= (1LL << 31) || (int64_t)H * 256 >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  CUtensorMap tx, tw;
+  {
+    // kv_c as [8 latent blocks][tokens][64 columns] (block stride 128 bytes): one box is a
+    // 128-token tile, all eight blocks
+    const uint64_t d[3] = {64, (uint64_t)n_tokens, 8}, st[2] = {1024, 128};
+    const uint32_t b[3] = {64, 128, 8};
+    if (!make_map(&tx, kv_c, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
+  {
+    const uint64_t d[2] = {512, (uint64_t)H * 256}, st[1] = {1024};
+    const uint32_t b[2] = {64, 256};   // 64 latent columns of one head's 256 rows
+    if (!make_map(&tw, wkv_b, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
+  ExpandParams p;
+  p.gamma = static_cast<const __nv_bfloat16*>(gamma);
+  p.eps = eps;
+  p.n_tokens = n_tokens;
+  p.seq_len = seq_len;
+  p.heads = H;
+  p.n_items = (n_tokens + 127) / 128 * H;
+  p.k_nope = static_cast<__nv_bfloat16*>(k_nope);
+  p.v = static_cast<__nv_bfloat16*>(v);
+  const int64_t grid = p.n_items < sms ? p.n_items : sms;
+  constexpr size_t smem = expand_smem_bytes();
+  if (!set_smem(expand_kernel, smem)) return MLA_ERR_CUDA;
+  return launch(false, expand_kernel, dim3((unsigned)grid), dim3(kExThreads), smem, stream, tx, tw, p);
 }
 
 }  // namespace sm100

@@ -227,6 +227,28 @@ def out_proj(d: MlaDims, o_lat: torch.Tensor, wkv_b: torch.Tensor, out: Optional
     return out
 
 
+def expand_kv(d: MlaDims, kv_c: torch.Tensor, wkv_b: torch.Tensor, batch: int, seq_len: int,
+              gamma: Optional[torch.Tensor] = None, eps: float = 1e-6, k_nope: Optional[torch.Tensor] = None,
+              v: Optional[torch.Tensor] = None, stream=None):
+    """Latent KV expansion (mla_expand_kv): K_nope [batch, H, seq_len, Dn] and V [batch, H, seq_len, Dv]
+    from the compressed rows kv_c [batch * seq_len, C]."""
+    dt = _dtype(d)
+    H, C, Dn, Dv = d.num_heads, d.kv_lora_rank, d.qk_nope_head_dim, d.v_head_dim
+    _need(kv_c, "kv_c", dt, (batch * seq_len, C))
+    _need(wkv_b, "wkv_b", dt, (H * (Dn + Dv), C))
+    if gamma is not None:
+        _need(gamma, "gamma", dt, (C,))
+    if k_nope is None:
+        k_nope = torch.empty((batch, H, seq_len, Dn), dtype=dt, device=kv_c.device)
+    if v is None:
+        v = torch.empty((batch, H, seq_len, Dv), dtype=dt, device=kv_c.device)
+    _need(k_nope, "k_nope", dt, (batch, H, seq_len, Dn))
+    _need(v, "v", dt, (batch, H, seq_len, Dv))
+    _check(LIB.mla_expand_kv(ctypes.byref(d), _ptr(kv_c), _ptr(gamma), float(eps), _ptr(wkv_b), batch, seq_len,
+                             _ptr(k_nope), _ptr(v), _stream(stream)), "mla_expand_kv")
+    return k_nope, v
+
+
 def append_latent(d: MlaDims, kv_new: torch.Tensor, k_pe_new: torch.Tensor, positions: torch.Tensor,
                   slots: torch.Tensor, kv_cache: torch.Tensor, pe_cache: torch.Tensor,
                   gamma: Optional[torch.Tensor] = None, eps: float = 1e-6, rope_base: float = 10000.0,

@@ -260,6 +260,24 @@ MLA_API mla_status_t mla_attn_paged(const mla_dims_t* dims, const void* q_abs, c
 MLA_API mla_status_t mla_out_proj(const mla_dims_t* dims, const void* o_lat, const void* wkv_b, void* out,
                           int64_t n_rows, cudaStream_t stream);
 
+/* Latent KV expansion, the naive path's materialisation ("Latent KV expansion
+ * with split", the operation's description; its output is the per-head keys
+ * and values "Naive Path Execution" consumes):
+ *   x[t]               = kv_c[t] / sqrt(mean_c(kv_c[t]^2) + eps) * gamma
+ *   k_nope[b, h, s, d] = sum_c x[b*S+s, c] * wkv_b[h*(Dn+Dv) + d, c]        d < Dn
+ *   v[b, h, s, d]      = sum_c x[b*S+s, c] * wkv_b[h*(Dn+Dv) + Dn + d, c]   d < Dv
+ *   kv_c    [batch * seq_len, C] row-major (compressed KV before normalisation;
+ *           packed tokens of ragged sequences may pass batch = 1).
+ *   gamma   [C] RMSNorm gain, or NULL for 1.   eps >= 0.
+ *   wkv_b   [H*(Dn+Dv), C] row-major.
+ *   k_nope  [batch, H, seq_len, Dn] and v [batch, H, seq_len, Dv], written.
+ * bf16 DeepSeek-V3 shapes run on the tcgen05 kernel (the normalised row is
+ * rounded to bf16 after the gain, the row's RMS factor scales the fp32
+ * products); other shapes on a CUDA-core kernel. */
+MLA_API mla_status_t mla_expand_kv(const mla_dims_t* dims, const void* kv_c, const void* gamma, float eps,
+                                   const void* wkv_b, int64_t batch, int64_t seq_len, void* k_nope, void* v,
+                                   cudaStream_t stream);
+
 /* Append new tokens to the latent caches ("Absorb Implementation Cache Design":
  * kv_cache holds the compressed key-value vector, pe_cache the rotary key;
  * "Latent KV expansion with split": the compressed KV is RMS-normalised):

@@ -158,3 +158,15 @@ def test_paged_host_checks(lib):
     # the tensor-core kernels copy 64-key tiles: smaller pages are not built for them
     assert L.mla_attn_paged(ctypes.byref(v3), A, A, 128 * 192, None, 2, A, 2, 1 << 12, A, A, 64, 32, A, 128, A,
                             A, 1 << 30, 0, None) == lib.MLA_ERR_UNSUPPORTED
+
+
+def test_expand_host_checks(lib):
+    L = lib.LIB
+    v3 = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
+    f = lambda *a: L.mla_expand_kv(ctypes.byref(v3), *a)
+    assert f(A, None, 1e-6, A, 0, 128, A, A, None) == lib.MLA_OK              # no tokens
+    assert f(A, None, 1e-6, A, -1, 128, A, A, None) == lib.MLA_ERR_INVALID_ARG
+    assert f(A, None, -1.0, A, 1, 128, A, A, None) == lib.MLA_ERR_INVALID_ARG   # eps < 0
+    assert f(None, None, 1e-6, A, 1, 128, A, A, None) == lib.MLA_ERR_INVALID_ARG
+    assert f(A, A + 8, 1e-6, A, 1, 128, A, A, None) == lib.MLA_ERR_INVALID_ARG  # misaligned gain
+    assert f(A, None, 1e-6, A, 1 << 30, 1 << 30, A, A, None) == lib.MLA_ERR_INVALID_ARG   # token count overflows
