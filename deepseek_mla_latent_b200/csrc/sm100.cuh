@@ -334,6 +334,7 @@ inline mla_status_t expand_kv(const void* kv_c, const void* gamma, float eps, co
   p.n_items = (n_tokens + 127) / 128 * H;
   p.k_nope = static_cast<__nv_bfloat16*>(k_nope);
   p.v = static_cast<__nv_bfloat16*>(v);
+  p.vec32 = ((reinterpret_cast<uintptr_t>(k_nope) | reinterpret_cast<uintptr_t>(v)) & 31u) == 0;
   const int64_t grid = p.n_items < sms ? p.n_items : sms;
   constexpr size_t smem = expand_smem_bytes();
   if (!set_smem(expand_kernel, smem)) return MLA_ERR_CUDA;

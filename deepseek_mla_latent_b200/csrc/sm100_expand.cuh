@@ -62,6 +62,7 @@ struct ExpandParams {
   int64_t n_items;              // ceil(n_tokens / 128) * heads
   __nv_bfloat16* k_nope;        // [batch, heads, seq_len, 128]
   __nv_bfloat16* v;             // [batch, heads, seq_len, 128]
+  int vec32;                    // both outputs 32-byte aligned: whole-sector stores
 };
 
 __global__ void __launch_bounds__(kExThreads, 1)
@@ -251,14 +252,20 @@ __global__ void __launch_bounds__(kExThreads, 1)
         ptx::tmem_ld32(tmem + lane_base + 256 * ab + 32 * c, v);
         ptx::tmem_wait_ld();
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>((c < 4 ? p.k_nope : p.v) + row + 32 * (c & 3));
+          __nv_bfloat16* dst = (c < 4 ? p.k_nope : p.v) + row + 32 * (c & 3);
+          uint32_t pk[16];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t* x = &v[8 * q];
-            dst[q] = make_uint4(ptx::pack_bf16x2(__uint_as_float(x[0]) * r, __uint_as_float(x[1]) * r),
-                                ptx::pack_bf16x2(__uint_as_float(x[2]) * r, __uint_as_float(x[3]) * r),
-                                ptx::pack_bf16x2(__uint_as_float(x[4]) * r, __uint_as_float(x[5]) * r),
-                                ptx::pack_bf16x2(__uint_as_float(x[6]) * r, __uint_as_float(x[7]) * r));
+          for (int q = 0; q < 16; ++q)
+            pk[q] = ptx::pack_bf16x2(__uint_as_float(v[2 * q]) * r, __uint_as_float(v[2 * q + 1]) * r);
+          if (p.vec32) {
+            // a lane's row is 256 bytes: 32-byte stores fill whole L2 sectors (16-byte stores from
+            // lanes 256 bytes apart would each write half a sector)
+            ptx::st_global_v8(dst, *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]));
+            ptx::st_global_v8(dst + 16, *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]));
+          } else {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) d4[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
         }
       }

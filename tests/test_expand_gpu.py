@@ -67,3 +67,24 @@ def test_full_expand_sampled():
         rk, rv = oracle.expand_kv(rows, e.gamma, 1e-6, e.wkv_b, dd.heads, dd.qk_nope, dd.v_head, 1, len(s_idx))
         assert_close(k[b][:, s_idx], rk[0], "bf16", f"k_nope batch {b}")
         assert_close(v[b][:, s_idx], rv[0], "bf16", f"v batch {b}")
+
+
+def test_v3_expand_outputs_16_byte_aligned():
+    """Outputs that are 16- but not 32-byte aligned take the 16-byte store path; same result."""
+    e = wl.expand_inputs(wl.V3, 1, 130, seed=10)
+    d = mla.dims_from(e.dims)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=torch.bfloat16)
+    n = 128 * 130 * 128
+    kb = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    vb = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    k = kb[8:].view(1, 128, 130, 128)
+    v = vb[8:].view(1, 128, 130, 128)
+    assert k.data_ptr() % 32 == 16
+    mla.expand_kv(d, t(e.kv_c), t(e.wkv_b), 1, 130, gamma=t(e.gamma), k_nope=k, v=v)
+    k2, v2 = mla.expand_kv(d, t(e.kv_c), t(e.wkv_b), 1, 130, gamma=t(e.gamma))
+    mla.device_status()
+    assert torch.equal(k, k2) and torch.equal(v, v2)
+    dd = e.dims
+    rk, rv = oracle.expand_kv(e.kv_c, e.gamma, 1e-6, e.wkv_b, dd.heads, dd.qk_nope, dd.v_head, 1, 130)
+    assert_close(k.float().cpu().numpy().astype(np.float64), rk, "bf16", "k_nope")
+    assert_close(v.float().cpu().numpy().astype(np.float64), rv, "bf16", "v")
