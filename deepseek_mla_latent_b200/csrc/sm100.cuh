@@ -277,9 +277,10 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
     const uint32_t b[3] = {64, 32, 1};
     if (!make_map(&tout, p.out, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
-  if (!set_smem(latent_attn_kernel, kAttnSmem)) return MLA_ERR_CUDA;
-  mla_status_t st = launch(true, latent_attn_kernel, dim3((unsigned)(2 * units)), dim3(kAttnThreads), kAttnSmem,
-                           stream, tkv_s, tpe, tqpe, tkv_v, tqa, tout, p);
+  auto kern = paged.table ? latent_attn_kernel<true> : latent_attn_kernel<false>;
+  if (!set_smem(kern, kAttnSmem)) return MLA_ERR_CUDA;
+  mla_status_t st = launch(true, kern, dim3((unsigned)(2 * units)), dim3(kAttnThreads), kAttnSmem, stream, tkv_s,
+                           tpe, tqpe, tkv_v, tqa, tout, p);
   if (st != MLA_OK || splits <= 1 || !merge) return st;
   const int64_t pairs_per_block = kMergeThreads / 64;   // two warps per (row, head)
   const int64_t merge_blocks = (n_q * H + pairs_per_block - 1) / pairs_per_block;

@@ -189,7 +189,9 @@ __device__ __forceinline__ UnitRange unit_range(const AttnParams& p, int64_t uni
 // non-decreasing from call to call.  Packed cache: the sequence's first row plus the key.
 // Paged cache: key j of sequence b sits in row table[b][j / page] * page + j % page.  Lane l
 // holds the table entry of page win + l, and the next 32 entries are already loading when the
-// window moves on, so the copies wait on the table only once, at the start.
+// window moves on, so the copies wait on the table only once, at the start.  The packed
+// form (kPaged = false) compiles to the first row plus the key and nothing else.
+template <bool kPaged>
 struct CacheRows {
   const int* bt;        // the sequence's row of the block table, nullptr for a packed cache
   int64_t base;         // packed cache: the sequence's first row
@@ -201,23 +203,23 @@ struct CacheRows {
   __device__ __forceinline__ int entry(int64_t i) const { return i < n_entries ? __ldg(bt + i) : -1; }
 
   __device__ __forceinline__ void init(const AttnParams& p, const UnitRange& u, uint32_t lane) {
-    bt = p.block_table ? p.block_table + (int64_t)u.b * p.bt_stride : nullptr;
     base = u.k0;
+    bt = nullptr;
+    if (!kPaged) return;
+    bt = p.block_table + (int64_t)u.b * p.bt_stride;
     rows = p.kv_rows;
     n_entries = p.bt_stride;
     page = p.page_size;
-    if (bt) {
-      win = u.j_begin / page;
-      cur = entry(win + lane);
-      nxt = entry(win + 32 + lane);
-    }
+    win = u.j_begin / page;
+    cur = entry(win + lane);
+    nxt = entry(win + 32 + lane);
   }
 
   // Row of key j (counted from the sequence's first key).  A page outside the cache gives row
   // `rows`, past the end of the tensor maps, which the copies fill with zeros; when the page
   // holds a key the unit attends to (j < j_end) the device error word records it.
   __device__ __forceinline__ int row(int64_t j, int64_t j_end, uint32_t lane) {
-    if (!bt) return (int)(base + j);
+    if (!kPaged) return (int)(base + j);
     const int64_t pg = j / page;
     while (pg >= win + 32) {
       cur = nxt;
@@ -247,6 +249,7 @@ constexpr int kTmemSlot = 63;
 constexpr uint32_t kColQ = 0, kColS = 256;
 
 // ---------------------------------------------------------------- score CTA
+template <bool kPaged>
 __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const UnitRange& u, const AttnParams& p,
                                            const CUtensorMap* tmap_kv, const CUtensorMap* tmap_pe,
                                            const CUtensorMap* tmap_qpe, const CUtensorMap* tmap_qabs) {
@@ -283,10 +286,10 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
         ptx::tma_load_3d(smem + L::kOffQpe, tmap_qpe, q_full, 128, head0, (int)u.row);
       }
       __syncwarp();
-      CacheRows cache;
+      CacheRows<kPaged> cache;
       cache.init(p, u, lane);
       // pages of 64 * odd keys: each 128-key tile is two 64-key copies (rows r0, r1) per block
-      const bool halves = p.score_copy_rows != kTileQ;
+      const bool halves = kPaged && p.score_copy_rows != kTileQ;
       bool ok = true;
       for (int jj = 0; ok && jj < ntq; ++jj) {
         const int64_t j0 = u.j_begin + (int64_t)jj * kTileQ;
@@ -630,6 +633,7 @@ __device__ __forceinline__ void store_o_tma(uint8_t* buf, uint32_t t_base, uint3
   __syncwarp();
 }
 
+template <bool kPaged>
 __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const UnitRange& u, const AttnParams& p,
                                            const CUtensorMap* tmap_kv, const CUtensorMap* tmap_out) {
   using L = ValueLayout;
@@ -654,7 +658,7 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
         ptx::prefetch_tmap(tmap_out);
       }
       __syncwarp();
-      CacheRows cache;
+      CacheRows<kPaged> cache;
       cache.init(p, u, lane);
       // The first P tile arrives several microseconds in; loading values before then would only
       // add to the start-up burst on HBM (these rows reach L2 through the score CTA meanwhile).
@@ -819,6 +823,8 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
 
 // ---------------------------------------------------------------- the kernel
 // One cluster of two CTAs per work unit (query row, 128-head group, split).
+// kPaged: the cache is read through a block table (one instance per cache kind).
+template <bool kPaged>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tmap_kv_score, const __grid_constant__ CUtensorMap tmap_pe,
                        const __grid_constant__ CUtensorMap tmap_qpe, const __grid_constant__ CUtensorMap tmap_kv_value,
@@ -888,9 +894,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     u.nt = 0;
   }
   if (rank == 0)
-    score_role(smem, tmem, u, p, &tmap_kv_score, &tmap_pe, &tmap_qpe, &tmap_qabs);
+    score_role<kPaged>(smem, tmem, u, p, &tmap_kv_score, &tmap_pe, &tmap_qpe, &tmap_qabs);
   else
-    value_role(smem, tmem, u, p, &tmap_kv_value, &tmap_out);
+    value_role<kPaged>(smem, tmem, u, p, &tmap_kv_value, &tmap_out);
 
   ptx::tc_fence_before();
   __syncthreads();
