@@ -135,3 +135,19 @@ def test_full_v3_decode_paged_sampled():
     for (b, h), r in ref.items():
         assert_close(out[b:b + 1, h, :], r, "bf16", f"seq {b} head {h}")
     assert np.array_equal(o_lat, run_path(w)["o_lat"])
+
+
+def test_v3_block_sparse_decode_selection():
+    """Block-sparse decode: each sequence attends to 20 of its pages, chosen at random and
+    listed in random order (a selection like a sparse-attention indexer's), given to
+    mla_attn_paged as the block table; against the oracle over the same selection.  The
+    split plan is made for the full length (4096), so most splits are empty."""
+    w = wl.make_workload("v3sp", V3, [1, 1], [4096, 2048], seed=18)
+    pc = wl.paged_cache(w, 64, seed=7)
+    rng = np.random.default_rng(1)
+    sel = np.full((2, 20), -1, dtype=np.int32)
+    for b, t in enumerate(w.seqlens_k):
+        sel[b] = pc.block_table[b, rng.choice(t // 64, size=20, replace=False)]
+    sp = wl.PagedCache(64, pc.kv_cache, pc.pe_cache, sel, np.full(2, 20 * 64, dtype=np.int32))
+    _, out = _run_paged(w, sp)
+    assert_close(out, _oracle_paged(w, sp), "bf16", "block-sparse decode")
