@@ -169,8 +169,8 @@ MLA_API mla_status_t mla_attn_decode_out(const mla_dims_t* dims, const void* q_a
 /* Size of the device scratch array behind mla_attn_decode_static_scratch. */
 #define MLA_STATIC_SCRATCH_BYTES (32u << 20)
 
-/* mla_attn_decode without a caller-provided workspace.  The paper has no
- * counterpart to this call; it exists for callers that cannot allocate
+/* mla_attn_decode without a caller-provided workspace.  The method as
+ * described has no counterpart to this call; it exists for callers that cannot allocate
  * device memory: code that only receives input and output buffers from a
  * host framework with no allocator to call, and code on a path where
  * cudaMalloc is not allowed or would synchronise the device (inside a

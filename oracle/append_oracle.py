@@ -12,7 +12,7 @@ expansion with split" (kernelindex.com) states that the compressed KV is
 RMS-normalised.  Appending one new token therefore writes
     kv_cache[slot] = kv / sqrt(mean(kv^2) + eps) * gamma
     pe_cache[slot] = RoPE(k_pe, position)
-Readings where the pages are silent (each listed in the design notes): the
+Readings where the cited pages are silent (each listed in the design notes): the
 RMSNorm epsilon and gain are inputs (eps = 1e-6 and gamma = 1 in the
 workloads); RoPE rotates interleaved pairs (x[2i], x[2i+1]) by the angle
 position * base^(-2i/R) with base 10000; the position is the token's index in

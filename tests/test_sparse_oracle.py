@@ -1,7 +1,7 @@
 """Block-sparse decode as attention over selected pages: the fine-grained sparse attention step
 of DeepSeek Sparse Attention ("What is DeepSeek Sparse Attention (DSA)?", section "How DSA works
 (conceptual)": exact attention over the shortlisted spans only), at the granularity of cache
-pages.  The pages define no indexer, so the selection is an input; a selection is a block table
+pages.  The cited page defines no indexer, so the selection is an input; a selection is a block table
 listing the chosen pages, and mla_attn_paged computes it.  These pins hold the oracle's reading
 to dense attention."""
 import numpy as np
