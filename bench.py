@@ -186,6 +186,13 @@ def cpu_baseline_oracle(w, seconds: float):
                       f"{el:.1f} s, scaled to the whole step"}
 
 
+def workload_config(w, world: int) -> dict:
+    """The `config` keys both arms report for a workload."""
+    return {"workload": w.name, "batch": w.batch, "heads": w.dims.heads, "kv_lora_rank": w.dims.kv_lora_rank,
+            "qk_rope": w.dims.qk_rope, "seq_len_k": max(w.seqlens_k), "queries_per_seq": 1,
+            "parallelism": "replicas" if world > 1 else "single"}
+
+
 def run_reference(args, rank, world):
     from deepseek_mla_latent_b200 import workloads as wl
     if rank != 0:
@@ -209,8 +216,7 @@ def run_reference(args, rank, world):
     line = {"metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us_step / 1e3, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "batch": B, "heads": H, "seq_len_k": max(w.seqlens_k),
-                       "queries_per_seq": 1, "parallelism": "replicas"},
+            "config": workload_config(w, world),
             "cpu_baseline": {"value": us_step, "unit": UNIT, "cores": int(cores), "kind": "oracle",
                              "sample": f"each step: one (sequence, head) pair of {len(pairs)}, naive fp64 path, "
                                        "scaled to the whole step"},
@@ -563,8 +569,7 @@ def main():
             "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us_step / 1e3, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32", "data": "synthetic",
-            "config": {"workload": w.name, "batch": B, "heads": H, "kv_lora_rank": C, "qk_rope": w.dims.qk_rope,
-                       "seq_len_k": max_k, "queries_per_seq": 1, "parallelism": "replicas" if world > 1 else "single",
+            "config": {**workload_config(w, world),
                        "l2": f"inputs larger than L2: {copies} rotating copies of q, kv, pe and wkv_b "
                              f"({copies * per_copy / 2**20:.0f} MiB), steps back to back between two events"},
             "tokens_per_s": world * B / (us_step / 1e6),
