@@ -170,3 +170,28 @@ def test_expand_host_checks(lib):
     assert f(None, None, 1e-6, A, 1, 128, A, A, None) == lib.MLA_ERR_INVALID_ARG
     assert f(A, A + 8, 1e-6, A, 1, 128, A, A, None) == lib.MLA_ERR_INVALID_ARG  # misaligned gain
     assert f(A, None, 1e-6, A, 1 << 30, 1 << 30, A, A, None) == lib.MLA_ERR_INVALID_ARG   # token count overflows
+
+
+@pytest.mark.parametrize("batch", [1, 2, 8, 37, 64, 74, 75, 300])
+@pytest.mark.parametrize("max_k", [1, 128, 129, 4096, 131072])
+def test_decode_split_plan(lib, batch, max_k):
+    """The automatic split plan of the tensor-core decode: at least one split, never more
+    splits than 128-key score tiles, and with more than one split no more (row, split) units
+    than CTA pairs of a 148-SM GPU (the host has no device here, so the planner uses 148).
+    An explicit split count is used as given, and the workspace grows with the splits."""
+    L = lib.LIB
+    v3 = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
+    s = L.mla_decode_num_splits(ctypes.byref(v3), batch, max_k, 0)
+    tiles = -(-max_k // 128)
+    assert 1 <= s <= max(1, tiles)
+    if s > 1:
+        assert batch * s <= 74
+    assert L.mla_decode_num_splits(ctypes.byref(v3), batch, max_k, 5) == 5
+    w1 = L.mla_workspace_size(ctypes.byref(v3), batch, batch, max_k, 1)
+    w2 = L.mla_workspace_size(ctypes.byref(v3), batch, batch, max_k, 2)
+    w9 = L.mla_workspace_size(ctypes.byref(v3), batch, batch, max_k, 9)
+    assert w1 <= w2 < w9
+    # the partials alone: bf16 [splits, batch, H, 512]
+    assert w9 >= 9 * batch * 128 * 512 * 2
+    out = L.mla_decode_out_workspace_size(ctypes.byref(v3), batch, max_k, 9)
+    assert out >= w9 + batch * 128 * 512 * 2
