@@ -302,9 +302,14 @@ MLA_API mla_status_t mla_append_latent(const mla_dims_t* dims, const void* kv_ne
 MLA_API const char* mla_status_string(mla_status_t status);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
- * current device.  Returns MLA_ERR_DEVICE_TIMEOUT if a bounded wait in an
- * earlier kernel ran out (its code is stored in *code_out when non-NULL),
- * MLA_ERR_CUDA if the stream reports an error, MLA_OK otherwise. */
+ * current device.  Returns MLA_ERR_DEVICE_TIMEOUT if an earlier kernel set a
+ * bit of the word (stored in *code_out when non-NULL), MLA_ERR_CUDA if the
+ * stream reports an error, MLA_OK otherwise.  Bits: 1<<0 a consumer waited too
+ * long for a TMA tile, 1<<1 a producer for a free stage, 1<<2 a wait for a
+ * tensor-core commit, 1<<3 the score products for P, 1<<4 a wait on the partner
+ * CTA, 1<<5 an exit path for copies in flight, 1<<6 a work item outside its
+ * buffers (or a misaligned shared-memory base), 1<<7 a block-table entry of a
+ * page that holds keys lies outside the cache (mla_attn_paged). */
 MLA_API mla_status_t mla_device_status(cudaStream_t stream, uint32_t* code_out);
 
 /* Which kernel family a call with these dims runs: 1 = tcgen05 tensor-core
