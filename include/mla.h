@@ -306,7 +306,7 @@ MLA_API const char* mla_status_string(mla_status_t status);
  * bit of the word (stored in *code_out when non-NULL), MLA_ERR_CUDA if the
  * stream reports an error, MLA_OK otherwise.  Bits: 1<<0 a consumer waited too
  * long for a TMA tile, 1<<1 a producer for a free stage, 1<<2 a wait for a
- * tensor-core commit, 1<<3 the score products for P, 1<<4 a wait on the partner
+ * tensor-core commit, 1<<3 a wait on the softmax threads (P, q_abs in TMEM), 1<<4 a wait on the partner
  * CTA, 1<<5 an exit path for copies in flight, 1<<6 a work item outside its
  * buffers (or a misaligned shared-memory base), 1<<7 a block-table entry of a
  * page that holds keys lies outside the cache (mla_attn_paged). */
