@@ -53,10 +53,11 @@ def parse_args():
     p.add_argument("--workload", type=int, default=1, help="workload index (1 = DeepSeek-V3 decode b8 t4096)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
-    p.add_argument("--op", choices=["decode", "append", "paged", "expand"], default="decode",
+    p.add_argument("--op", choices=["decode", "append", "paged", "expand", "prefill"], default="decode",
                    help="decode: the decode step (the benchmark); append: the latent-cache append alone; "
                         "paged: the decode attention call over a paged cache beside the packed one; "
-                        "expand: the latent KV expansion")
+                        "expand: the latent KV expansion; prefill: the chunked-prefill step "
+                        "(workload 4 unless --workload names another prefill workload)")
     p.add_argument("--batch", type=int, default=4, help="sequences per expansion call (--op expand)")
     p.add_argument("--seq-len", type=int, default=1024, help="tokens per sequence (--op expand)")
     p.add_argument("--tokens", type=int, default=65536, help="new tokens per append call (--op append)")
@@ -362,6 +363,77 @@ def run_paged(args, rank, world):
         "gpu_launches": args.steps * (2 if mla.decode_num_splits(d, B, max_k, 0) > 1 else 1)}), flush=True)
 
 
+def prefill_attention_flop(w) -> float:
+    """Algorithmic flop of the absorb-form attention of a chunked prefill: 2 * H * (576 + 512)
+    per (query, visible key), query i of s new queries over t keys seeing t - s + i + 1."""
+    per_pair = 2.0 * w.dims.heads * (w.dims.kv_lora_rank + w.dims.qk_rope + w.dims.kv_lora_rank)
+    visible = 0
+    for s, t in zip(w.seqlens_q, w.seqlens_k):
+        visible += sum(max(0, min(t, t - s + i + 1)) for i in range(s))
+    return per_pair * visible
+
+
+def run_prefill(args, rank, world):
+    """Time the chunked-prefill step (mla_absorb_q -> mla_attn_prefill_chunk -> mla_out_proj) and
+    the attention call alone on a prefill workload; one JSON line (single GPU)."""
+    import torch
+    from deepseek_mla_latent_b200 import mla
+    from deepseek_mla_latent_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    idx = args.workload if any(s > 1 for s in wl.workload_shape(args.workload)[2]) else 4
+    w = wl.workload(idx)
+    d = mla.dims_from(w.dims)
+    dt = torch.bfloat16
+    t = lambda a, ty=dt: torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=ty)
+    q, kv, pe, wkv_b = t(w.q), t(w.kv), t(w.pe), t(w.wkv_b)
+    cu_q, cu_k = t(w.cu_seqlens_q, torch.int32), t(w.cu_seqlens_k, torch.int32)
+    n, H, C = w.n_q, w.dims.heads, w.dims.kv_lora_rank
+    max_q, max_k = max(w.seqlens_q), max(w.seqlens_k)
+    q_abs = torch.empty((n, H, C), dtype=dt, device="cuda")
+    o_lat = torch.empty((n, H, C), dtype=dt, device="cuda")
+    out = torch.empty((n, H, w.dims.v_head), dtype=dt, device="cuda")
+    ws = mla.workspace(d, w.batch, n, max_k, 0, device="cuda")
+
+    def attention():
+        mla.attn_prefill_chunk(d, q_abs, q, cu_q, cu_k, max_q, max_k, kv, pe, o_lat, ws)
+
+    def step():
+        mla.absorb_q(d, q, wkv_b, q_abs)
+        attention()
+        mla.out_proj(d, o_lat, wkv_b, out)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    mla.device_status()
+
+    def timed(fn):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps * 1e3
+
+    us_step, us_attn = timed(step), timed(attention)
+    mla.device_status()
+    hbm, tf, peak_kind = load_peaks()
+    attn_flop = prefill_attention_flop(w)
+    proj_flop = 2 * 2.0 * n * H * w.dims.qk_nope * C
+    attn_tf = attn_flop / (us_attn * 1e-6) / 1e12
+    print(json.dumps({
+        "metric": "MLA absorb chunked-prefill TFLOP/s (1xB200)", "value": attn_tf, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "us_per_step": us_step, "attn_us_per_call": us_attn,
+        "step_tflops": (attn_flop + proj_flop) / (us_step * 1e-6) / 1e12, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "queries_per_seq": max_q, "seq_len_k": max_k,
+                   "l2": "the step moves over 1 GB (q_abs and o_lat of 4096 rows), far above L2"},
+        "roofline": {"bound": "tensor", "achieved": attn_tf, "peak": tf, "unit": "TFLOP/s", "frac": attn_tf / tf,
+                     "peak_kind": peak_kind + " (burst)"},
+        "gpu_launches": args.steps * 3}), flush=True)
+
+
 def run_expand(args, rank, world):
     """Time mla_expand_kv (RMSNorm of the compressed KV, projection to all heads, head-major
     split into K_nope and V) at DeepSeek-V3 shapes; one JSON line (single GPU)."""
@@ -436,6 +508,9 @@ def main():
         return
     if args.op == "expand":
         run_expand(args, rank, world)
+        return
+    if args.op == "prefill":
+        run_prefill(args, rank, world)
         return
 
     import torch
