@@ -35,3 +35,19 @@ def test_reference_arm_other_ranks_print_nothing():
     r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_prefill_flop_count_closed_form():
+    """Workload 4: 4 sequences, query i of 1024 sees 3073 + i of 4096 keys, and each (query,
+    visible key) pair costs 2 * 128 * (512 + 64 + 512) flop."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from deepseek_mla_latent_b200 import workloads as wl
+    _, dims, sq, sk = wl.workload_shape(4)
+
+    class W:
+        pass
+    w = W()
+    w.dims, w.seqlens_q, w.seqlens_k = dims, sq, sk
+    pairs = 4 * (1024 * 3073 + 1023 * 1024 // 2)
+    assert bench.prefill_attention_flop(w) == pairs * 2 * 128 * (512 + 64 + 512)
