@@ -44,6 +44,132 @@ L2_BYTES = 126 << 20                           # B200 L2
 ROTATE_MIN_BYTES = 2 * L2_BYTES                # traffic between two uses of one input copy
 
 
+MIN_TIMED_MS = 200.0                           # least total length of a repeated timed region
+
+
+def decode_algorithmic(w):
+    """Algorithmic bytes and flop of one decode attention call: the cache rows (kv + pe) of every
+    visible key, and per query row q_abs, q_pe in and o_lat out; 2 * H * (576 + 512) flop per key."""
+    B, H, C = w.batch, w.dims.heads, w.dims.kv_lora_rank
+    alg_bytes = w.total_k * KV_BYTES_PER_TOKEN + B * H * (C + w.dims.qk_rope + C) * 2
+    return alg_bytes, w.total_k * H * FLOP_PER_TOKEN_PER_HEAD
+
+
+class DecodeBench:
+    """A decode workload resident on the GPU in rotating copies (together larger than twice L2),
+    with CUDA graphs of the public calls: the whole step (absorb, attention, merge fused into the
+    output projection), the attention call (attention kernel + split merge) and the attention
+    kernel alone (split partials left in the workspace)."""
+
+    def __init__(self, w, dev, warmup):
+        import torch
+        from deepseek_mla_latent_b200 import mla
+        self.w, self.dev = w, dev
+        self.d = d = mla.dims_from(w.dims)
+        self.dt = dt = torch.bfloat16 if w.dims.dtype == "bf16" else torch.float32
+        B, H, C, Dv = w.batch, w.dims.heads, w.dims.kv_lora_rank, w.dims.v_head
+        max_k = max(w.seqlens_k)
+        cu_k = torch.from_numpy(w.cu_seqlens_k).to(dev)
+        host = [torch.from_numpy(a).to(dtype=dt) for a in (w.q, w.kv, w.pe, w.wkv_b)]
+        self.per_copy = sum(t.numel() * t.element_size() for t in host)
+        self.copies = min(16, max(2, math.ceil(ROTATE_MIN_BYTES / self.per_copy) + 1))
+        self.inputs = [[t.to(dev) for t in host] for _ in range(self.copies)]   # (q, kv, pe, wkv_b) per copy
+        del host
+        bufs = {"q_abs": torch.empty((B, H, C), dtype=dt, device=dev),
+                "o_lat": torch.empty((B, H, C), dtype=dt, device=dev),
+                "out": torch.empty((B, H, Dv), dtype=dt, device=dev),
+                "ws": mla.workspace(d, B, B, max_k, 0, device=dev),
+                "ws_out": mla.decode_out_workspace(d, B, max_k, 0, device=dev)}
+        self.stream = torch.cuda.current_stream()
+        inputs = self.inputs
+
+        def step(k):
+            q, kv, pe, wkv_b = inputs[k]
+            q_abs = mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
+            return mla.attn_decode_out(d, q_abs, q, kv, pe, cu_k, max_k, wkv_b, bufs["out"], bufs["ws_out"])
+
+        def attention_call(k):
+            q, kv, pe, _ = inputs[k]
+            mla.attn_decode(d, bufs["q_abs"], q, kv, pe, cu_k, max_k, bufs["o_lat"], bufs["ws"])
+
+        def attention_kernel(k):
+            q, kv, pe, _ = inputs[k]
+            mla.attn_decode_partials(d, bufs["q_abs"], q, kv, pe, cu_k, max_k, bufs["ws"])
+
+        self.step = step
+        for i in range(max(3, warmup)):
+            step(i % self.copies)
+        mla.device_status()
+
+        def capture(fn):
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                fn()
+            torch.cuda.current_stream().wait_stream(side)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                fn()
+            return graph
+
+        # The timed steps replay CUDA graphs captured from the same calls, so host-side launch
+        # work does not leave the GPU idle inside the timed region.
+        self.g_step = [capture(lambda k=k: step(k)) for k in range(self.copies)]
+        self.g_attn = [capture(lambda k=k: attention_call(k)) for k in range(self.copies)]
+        self.g_kern = [capture(lambda k=k: attention_kernel(k)) for k in range(self.copies)]
+        for i in range(max(3, warmup)):
+            for g in (self.g_step, self.g_attn, self.g_kern):
+                g[i % self.copies].replay()
+        mla.device_status()
+
+    def timed(self, graphs, n, world=1):
+        """Milliseconds for exactly n replays, back to back between two events on the stream."""
+        import torch
+        import torch.distributed as dist
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for i in range(n):
+            graphs[i % self.copies].replay()
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return e0.elapsed_time(e1)
+
+
+def other_configs(args, dev, hbm, tf):
+    """The ragged, long-context and chunked-prefill workloads, each timed on its own, for the
+    same JSON line: step and attention times and the fraction of the roofline that binds."""
+    import torch
+    from deepseek_mla_latent_b200 import workloads as wl
+    res = {}
+    for idx in (2, 3):
+        w = wl.workload(idx)
+        b = DecodeBench(w, dev, 3)
+        n = 50
+        step_ms = statistics.mean(b.timed(b.g_step, n) for _ in range(3))
+        attn_ms = statistics.mean(b.timed(b.g_attn, n) for _ in range(3))
+        kern_ms = statistics.mean(b.timed(b.g_kern, n) for _ in range(3))
+        alg_bytes, alg_flop = decode_algorithmic(w)
+        gbs = alg_bytes / (kern_ms / n * 1e-3) / 1e9
+        res[w.name] = {"step_us": step_ms / n * 1e3, "attn_call_us": attn_ms / n * 1e3,
+                       "attn_kernel_us": kern_ms / n * 1e3, "attn_cache_gbs": gbs, "bound": "hbm",
+                       "frac": gbs / hbm, "tensor_frac": alg_flop / (kern_ms / n * 1e-3) / 1e12 / tf,
+                       "steps": n, "repeats": 3, "tokens": w.total_k}
+        del b
+        torch.cuda.empty_cache()
+    w = wl.workload(4)
+    us_step, us_attn, attn_flop, proj_flop, err = prefill_timings(w, 5, 3, prefill_check_pairs(w))
+    tflops = attn_flop / (us_attn * 1e-6) / 1e12
+    res[w.name] = {"step_us": us_step, "attn_call_us": us_attn, "attn_tflops": tflops, "bound": "tensor",
+                   "frac": tflops / tf, "parity_max_rel_err": err, "steps": 5}
+    torch.cuda.empty_cache()
+    return res
+
+
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -52,6 +178,8 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", type=int, default=1, help="workload index (1 = DeepSeek-V3 decode b8 t4096)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra-configs", action="store_true",
+                   help="skip the ragged, long-context and chunked-prefill workloads in the decode line")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     p.add_argument("--op", choices=["decode", "append", "paged", "expand", "prefill"], default="decode",
                    help="decode: the decode step (the benchmark); append: the latent-cache append alone; "
@@ -165,15 +293,25 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def host_cores():
+    """(cores this process may run on, BLAS threads the oracle's matrix products use)."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        cores = os.cpu_count() or 1
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        blas = cores
+    return int(cores), int(blas)
+
+
 def cpu_baseline_oracle(w, seconds: float):
     """Time the fp64 oracle (naive path) on (sequence, head) pairs of the workload for
     about `seconds`, and scale to one whole step (all sequences x all heads)."""
     import oracle
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:  # noqa: BLE001
-        cores = os.cpu_count() or 1
+    cores, blas = host_cores()
     H, B = w.dims.heads, w.batch
     pairs = [(b, h) for h in range(H) for b in range(B)]
     done, t0 = 0, time.perf_counter()
@@ -182,7 +320,8 @@ def cpu_baseline_oracle(w, seconds: float):
         done += 1
     el = time.perf_counter() - t0
     per_pair = el / done
-    return {"value": per_pair * len(pairs) * 1e6, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+    return {"value": per_pair * len(pairs) * 1e6, "unit": UNIT, "cores": cores, "blas_threads": blas,
+            "kind": "oracle", "value_kind": "scaled from a timed sample",
             "sample": f"{done} of {len(pairs)} (sequence, head) pairs of the same workload, naive fp64 path, "
                       f"{el:.1f} s, scaled to the whole step"}
 
@@ -195,16 +334,15 @@ def workload_config(w, world: int) -> dict:
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle on the host cores.  Each timed step runs one (sequence,
+    head) pair of the workload and is scaled by the number of pairs to one whole step, so
+    `value` and `ms_per_step` are scaled from a timed sample (`value_kind` says so)."""
     from deepseek_mla_latent_b200 import workloads as wl
     if rank != 0:
         return
     w = wl.workload(args.workload)
     import oracle
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:  # noqa: BLE001
-        cores = os.cpu_count() or 1
+    cores, blas = host_cores()
     H, B = w.dims.heads, w.batch
     pairs = [(b, h) for h in range(H) for b in range(B)]
     for i in range(args.warmup):
@@ -217,10 +355,13 @@ def run_reference(args, rank, world):
     line = {"metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us_step / 1e3, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "value_kind": f"scaled from a timed sample: {args.steps} of {len(pairs)} (sequence, head) pairs "
+                          f"timed ({el:.2f} s), times {len(pairs)} / {args.steps}",
             "config": workload_config(w, world),
-            "cpu_baseline": {"value": us_step, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "cpu_baseline": {"value": us_step, "unit": UNIT, "cores": cores, "blas_threads": blas,
+                             "kind": "oracle", "value_kind": "scaled from a timed sample",
                              "sample": f"each step: one (sequence, head) pair of {len(pairs)}, naive fp64 path, "
-                                       "scaled to the whole step"},
+                                       f"scaled to the whole step ({args.steps} pairs timed, {el:.2f} s)"},
             "e2e": {"value": us_step, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -373,15 +514,13 @@ def prefill_attention_flop(w) -> float:
     return per_pair * visible
 
 
-def run_prefill(args, rank, world):
+def prefill_timings(w, steps: int, warmup: int, check_pairs=()):
     """Time the chunked-prefill step (mla_absorb_q -> mla_attn_prefill_chunk -> mla_out_proj) and
-    the attention call alone on a prefill workload; one JSON line (single GPU)."""
+    the attention call alone on one GPU.  With `check_pairs`, the step's output for those
+    (sequence, head) pairs is first compared with the oracle (max error relative to max|oracle|).
+    Returns (us_step, us_attn, attention flop, projection flop, max relative error or None)."""
     import torch
     from deepseek_mla_latent_b200 import mla
-    from deepseek_mla_latent_b200 import workloads as wl
-    torch.cuda.set_device(0)
-    idx = args.workload if any(s > 1 for s in wl.workload_shape(args.workload)[2]) else 4
-    w = wl.workload(idx)
     d = mla.dims_from(w.dims)
     dt = torch.bfloat16
     t = lambda a, ty=dt: torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=ty)
@@ -402,7 +541,19 @@ def run_prefill(args, rank, world):
         attention()
         mla.out_proj(d, o_lat, wkv_b, out)
 
-    for _ in range(max(3, args.warmup)):
+    err = None
+    if check_pairs:
+        import oracle
+        step()
+        mla.device_status()
+        got = out.float().cpu().numpy()
+        ref = oracle.workload_naive(w, pairs=list(check_pairs))
+        cq = w.cu_seqlens_q
+        err = 0.0
+        for (b, h), r in ref.items():
+            e = float(np.max(np.abs(got[cq[b]:cq[b + 1], h, :] - r))) / max(float(np.max(np.abs(r))), 1e-30)
+            err = max(err, e)
+    for _ in range(max(3, warmup)):
         step()
     mla.device_status()
 
@@ -410,28 +561,59 @@ def run_prefill(args, rank, world):
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for _ in range(args.steps):
+        for _ in range(steps):
             fn()
         e1.record()
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / args.steps * 1e3
+        return e0.elapsed_time(e1) / steps * 1e3
 
     us_step, us_attn = timed(step), timed(attention)
     mla.device_status()
-    hbm, tf, peak_kind = load_peaks()
     attn_flop = prefill_attention_flop(w)
-    proj_flop = 2 * 2.0 * n * H * w.dims.qk_nope * C
+    proj_flop = 2.0 * n * H * C * (w.dims.qk_nope + w.dims.v_head)
+    return us_step, us_attn, attn_flop, proj_flop, err
+
+
+def prefill_check_pairs(w):
+    """(sequence, head) pairs the prefill benchmark checks against the oracle: one head of every
+    sequence (all its query rows, first and last included) and heads 0 and 127 of sequence 0."""
+    H = w.dims.heads
+    return sorted({(b, (37 * b + 5) % H) for b in range(w.batch)} | {(0, 0), (0, H - 1)})
+
+
+def run_prefill(args, rank, world):
+    """Time the chunked-prefill step and the attention call alone on a prefill workload; one
+    JSON line.  One GPU: under a multi-rank launch rank 0 alone runs and prints."""
+    if world > 1 and rank != 0:
+        return
+    import torch
+    from deepseek_mla_latent_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    idx = args.workload if any(s > 1 for s in wl.workload_shape(args.workload)[2]) else 4
+    w = wl.workload(idx)
+    us_step, us_attn, attn_flop, proj_flop, err = prefill_timings(w, args.steps, args.warmup,
+                                                                   prefill_check_pairs(w))
+    hbm, tf, peak_kind = load_peaks()
     attn_tf = attn_flop / (us_attn * 1e-6) / 1e12
-    print(json.dumps({
+    line = {
         "metric": "MLA absorb chunked-prefill TFLOP/s (1xB200)", "value": attn_tf, "unit": "TFLOP/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "us_per_step": us_step, "attn_us_per_call": us_attn,
         "step_tflops": (attn_flop + proj_flop) / (us_step * 1e-6) / 1e12, "higher_is_better": True,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "queries_per_seq": max_q, "seq_len_k": max_k,
+        "config": {"workload": w.name, "batch": w.batch, "queries_per_seq": max(w.seqlens_q),
+                   "seq_len_k": max(w.seqlens_k),
                    "l2": "the step moves over 1 GB (q_abs and o_lat of 4096 rows), far above L2"},
+        "parity": {"pairs": len(prefill_check_pairs(w)), "max_rel_err": err, "tol": 2e-2},
         "roofline": {"bound": "tensor", "achieved": attn_tf, "peak": tf, "unit": "TFLOP/s", "frac": attn_tf / tf,
                      "peak_kind": peak_kind + " (burst)"},
-        "gpu_launches": args.steps * 3}), flush=True)
+        "gpu_launches": args.steps * 3}
+    if not args.no_cpu_baseline:
+        cpu = cpu_baseline_oracle(w, args.cpu_seconds)
+        # the oracle's time for the whole step, in the line's unit (the same algorithmic flop)
+        cpu["value"] = attn_flop / (cpu["value"] * 1e-6) / 1e12
+        cpu["unit"] = "TFLOP/s"
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
 
 
 def run_expand(args, rank, world):
@@ -525,56 +707,8 @@ def main():
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     w = wl.workload(args.workload)
-    d = mla.dims_from(w.dims)
-    dt = torch.bfloat16 if w.dims.dtype == "bf16" else torch.float32
-    B, H, C, Dv = w.batch, w.dims.heads, w.dims.kv_lora_rank, w.dims.v_head
-    max_k = max(w.seqlens_k)
-    cu_k = torch.from_numpy(w.cu_seqlens_k).to(dev)
-    host = [torch.from_numpy(a).to(dtype=dt) for a in (w.q, w.kv, w.pe, w.wkv_b)]
-    per_copy = sum(t.numel() * t.element_size() for t in host)
-    copies = min(16, max(2, math.ceil(ROTATE_MIN_BYTES / per_copy) + 1))
-    inputs = [[t.to(dev) for t in host] for _ in range(copies)]   # (q, kv, pe, wkv_b) per copy
-    bufs = {"q_abs": torch.empty((B, H, C), dtype=dt, device=dev),
-            "o_lat": torch.empty((B, H, C), dtype=dt, device=dev),
-            "out": torch.empty((B, H, Dv), dtype=dt, device=dev),
-            "ws": mla.workspace(d, B, B, max_k, 0, device=dev),
-            "ws_out": mla.decode_out_workspace(d, B, max_k, 0, device=dev)}
-    stream = torch.cuda.current_stream()
-
-    def step(k):
-        # the whole hot path through the public calls: absorb, then attention (+ merge) and the
-        # output projection in one call (mla_attn_decode_out)
-        q, kv, pe, wkv_b = inputs[k]
-        q_abs = mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
-        return mla.attn_decode_out(d, q_abs, q, kv, pe, cu_k, max_k, wkv_b, bufs["out"], bufs["ws_out"])
-
-    def attention_call(k):
-        q, kv, pe, _ = inputs[k]
-        mla.attn_decode(d, bufs["q_abs"], q, kv, pe, cu_k, max_k, bufs["o_lat"], bufs["ws"])
-
-    for i in range(max(3, args.warmup)):
-        step(i % copies)
-    mla.device_status()
-
-    # The timed steps replay CUDA graphs captured from the same calls, so host-side
-    # launch work does not leave the GPU idle inside the timed region.
-    def capture(fn):
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
-            fn()
-        torch.cuda.current_stream().wait_stream(side)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            fn()
-        return graph
-
-    g_step = [capture(lambda k=k: step(k)) for k in range(copies)]
-    g_attn = [capture(lambda k=k: attention_call(k)) for k in range(copies)]
-    for i in range(max(3, args.warmup)):
-        g_step[i % copies].replay()
-        g_attn[i % copies].replay()
-    mla.device_status()
+    bench = DecodeBench(w, dev, args.warmup)
+    d, B, H, C, Dv, dt = bench.d, w.batch, w.dims.heads, w.dims.kv_lora_rank, w.dims.v_head, bench.dt
 
     sampler = None
     if rank == 0:
@@ -587,28 +721,26 @@ def main():
         sampler.start()
         time.sleep(0.3)
 
-    def timed(graphs, n):
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(n):
-            graphs[i % copies].replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        return e0.elapsed_time(e1)
+    # Each measurement times exactly K steps between two events (barrier and synchronize on both
+    # sides); it is repeated, the same number of times on every rank, until the timed region has
+    # lasted at least MIN_TIMED_MS in all, so that the clock samples see the GPU under load.
+    def repeated(graphs):
+        first = reduce_max([bench.timed(graphs, args.steps, world)], dev)[0]
+        reps = max(1, min(1000, math.ceil(MIN_TIMED_MS / max(first, 1e-3))))
+        runs = [first] + [bench.timed(graphs, args.steps, world) for _ in range(reps - 1)]
+        runs = reduce_max(runs, dev)
+        return statistics.mean(runs), len(runs)
 
-    total_ms = timed(g_step, args.steps)
-    # the attention call alone (its kernel + split merge), for the roofline figure
-    attn_total_ms = timed(g_attn, args.steps)
+    total_ms, reps = repeated(bench.g_step)
+    # the attention call alone (attention kernel + split merge) and the attention kernel alone
+    # (the split partials left in the workspace, mla_attn_decode_partials)
+    attn_total_ms, _ = repeated(bench.g_attn)
+    kern_total_ms, _ = repeated(bench.g_kern)
     clocks = sampler.stop() if sampler else None
     mla.device_status()
-    total_ms, attn_total_ms = reduce_max([total_ms, attn_total_ms], dev)
     us_step = total_ms / args.steps * 1e3
     mean_attn_ms = attn_total_ms / args.steps
+    mean_kern_ms = kern_total_ms / args.steps
 
     # End to end through the same public calls: pinned host q -> device, step, out -> pinned host,
     # the K steps back to back between two events, inputs rotating over the same copies.
@@ -616,44 +748,47 @@ def main():
     out_pinned = torch.empty((B, H, Dv), dtype=dt).pin_memory()
     e2e_steps = min(args.steps, 500)
     for i in range(3):
-        inputs[i % copies][0].copy_(q_pinned, non_blocking=True)
-        out_pinned.copy_(step(i % copies), non_blocking=True)
+        bench.inputs[i % bench.copies][0].copy_(q_pinned, non_blocking=True)
+        out_pinned.copy_(bench.step(i % bench.copies), non_blocking=True)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e2e_s, e2e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_s.record(stream)
+    e2e_s.record(bench.stream)
     for i in range(e2e_steps):
-        k = i % copies
-        inputs[k][0].copy_(q_pinned, non_blocking=True)
-        out_pinned.copy_(step(k), non_blocking=True)
-    e2e_e.record(stream)
+        k = i % bench.copies
+        bench.inputs[k][0].copy_(q_pinned, non_blocking=True)
+        out_pinned.copy_(bench.step(k), non_blocking=True)
+    e2e_e.record(bench.stream)
     torch.cuda.synchronize()
     e2e_ms, = reduce_max([e2e_s.elapsed_time(e2e_e)], dev)
     e2e_us = e2e_ms / e2e_steps * 1e3
 
     if rank == 0:
         hbm, tf, peak_kind = load_peaks()
-        tokens = w.total_k
-        alg_bytes = tokens * KV_BYTES_PER_TOKEN + B * H * (C + w.dims.qk_rope + C) * 2
-        alg_flop = tokens * H * FLOP_PER_TOKEN_PER_HEAD
-        attn_s = mean_attn_ms / 1e3
-        achieved_gbs = alg_bytes / attn_s / 1e9
+        alg_bytes, alg_flop = decode_algorithmic(w)
+        attn_s, kern_s = mean_attn_ms / 1e3, mean_kern_ms / 1e3
+        achieved_gbs = alg_bytes / kern_s / 1e9
         traffic = profiled_traffic(w.name)
         line = {
             "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us_step / 1e3, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32", "data": "synthetic",
             "config": {**workload_config(w, world),
-                       "l2": f"inputs larger than L2: {copies} rotating copies of q, kv, pe and wkv_b "
-                             f"({copies * per_copy / 2**20:.0f} MiB), steps back to back between two events"},
+                       "l2": f"inputs larger than L2: {bench.copies} rotating copies of q, kv, pe and wkv_b "
+                             f"({bench.copies * bench.per_copy / 2**20:.0f} MiB), steps back to back between "
+                             "two events"},
+            "repeats": reps,
             "tokens_per_s": world * B / (us_step / 1e6),
-            "attn_kernel_us": mean_attn_ms * 1e3,
+            "attn_kernel_us": mean_kern_ms * 1e3,
+            "attn_call_us": mean_attn_ms * 1e3,
             "attn_cache_gbs": achieved_gbs,
-            "attn_tflops": alg_flop / attn_s / 1e12,
+            "attn_call_gbs": alg_bytes / attn_s / 1e9,
+            "attn_tflops": alg_flop / kern_s / 1e12,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": achieved_gbs / hbm, "traffic": traffic, "peak_kind": peak_kind,
-                         "tensor_frac": alg_flop / attn_s / 1e12 / tf},
+                         "kernel": "latent attention kernel alone (CUDA events around its launches)",
+                         "tensor_frac": alg_flop / kern_s / 1e12 / tf},
             "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": int(q_pinned.numel() * q_pinned.element_size()),
                     "d2h_bytes_per_step": int(out_pinned.numel() * out_pinned.element_size())},
             "gpu_launches": None,
@@ -662,9 +797,13 @@ def main():
             "kernel_source_hash": kernel_source_hash(),
         }
         # absorb_q + attention + output projection (with the split merge fused in), one launch each
-        splits = mla.decode_num_splits(d, B, max_k, 0)
-        line["gpu_launches"] = args.steps * 3
+        splits = mla.decode_num_splits(d, B, max(w.seqlens_k), 0)
+        line["gpu_launches"] = args.steps * reps * 3
         line["config"]["num_splits"] = splits
+        if world == 1 and not args.no_extra_configs:
+            del bench
+            torch.cuda.empty_cache()
+            line["other_configs"] = other_configs(args, dev, hbm, tf)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_oracle(w, args.cpu_seconds)
         print(json.dumps(line), flush=True)

@@ -290,6 +290,40 @@ mla_status_t mla_attn_decode_static_scratch(const mla_dims_t* dims, const void* 
                          stream);
 }
 
+size_t mla_partials_workspace_size(const mla_dims_t* dims, int32_t batch, int64_t max_seqlen_k,
+                                   int32_t num_splits) {
+  Geo g;
+  if (!dims || !geo_of(dims, &g) || g.family != 1 || batch < 0 || max_seqlen_k < 0 || num_splits < 0 ||
+      num_splits > 256)
+    return 0;
+  const int splits = resolve_splits(g, batch, batch, max_seqlen_k, num_splits, true);
+  return mla::sm100::workspace_bytes(g.H, batch, splits, /*partials=*/true);
+}
+
+mla_status_t mla_attn_decode_partials(const mla_dims_t* dims, const void* q_abs, const void* q,
+                                      int64_t q_row_stride, const void* kv_cache, const void* pe_cache,
+                                      int64_t kv_rows, const int32_t* cu_seqlens_k, int32_t batch,
+                                      int64_t max_seqlen_k, void* workspace, size_t workspace_bytes,
+                                      int32_t num_splits, cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (g.family != 1) return MLA_ERR_UNSUPPORTED;
+  if (batch < 0 || max_seqlen_k < 0 || kv_rows < 0 || num_splits < 0 || num_splits > 256 ||
+      q_row_stride < (int64_t)g.H * (g.Dn + g.R) || (q_row_stride * 2) % 16 != 0)
+    return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!q_abs || !q || !cu_seqlens_k || !aligned16(q_abs) || !aligned16(q)) return MLA_ERR_INVALID_ARG;
+  if (kv_rows > 0 && (!kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
+    return MLA_ERR_INVALID_ARG;
+  const int splits = resolve_splits(g, batch, batch, max_seqlen_k, num_splits, true);
+  const size_t need = mla::sm100::workspace_bytes(g.H, batch, splits, /*partials=*/true);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return MLA_ERR_WORKSPACE;
+  return mla::sm100::attention(q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, nullptr, cu_seqlens_k, batch,
+                               batch, g.H, splits, g.scale, nullptr, workspace, stream, /*merge=*/false,
+                               mla::sm100::PagedKv{}, /*partials=*/true);
+}
+
 size_t mla_decode_out_workspace_size(const mla_dims_t* dims, int32_t batch, int64_t max_seqlen_k,
                                      int32_t num_splits) {
   Geo g;

@@ -175,8 +175,8 @@ inline int auto_decode_splits(int batch, int H, int64_t max_seqlen_k, int sms) {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline size_t workspace_bytes(int H, int64_t n_q, int splits) {
-  if (splits <= 1) return 0;
+inline size_t workspace_bytes(int H, int64_t n_q, int splits, bool partials = false) {
+  if (splits <= 1 && !partials) return 0;
   // bf16 partial O per (split, row, head) + fp32 (reference max, row sum)
   return align256((size_t)splits * n_q * H * 512 * 2) + align256((size_t)splits * n_q * H * 2 * sizeof(float));
 }
@@ -196,11 +196,12 @@ struct PagedKv {
 };
 
 // merge = false (split runs only): leave the partials in the workspace for merge_out_proj
-// instead of merging them into o_lat.
+// instead of merging them into o_lat.  partials = true: write the partial form (also for one
+// split) and never merge; o_lat is not used.
 inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_stride, const void* kv, const void* pe,
                               int64_t kv_rows, const int32_t* cu_q, const int32_t* cu_k, int batch, int64_t n_q,
                               int H, int splits, float scale, void* o_lat, void* ws, cudaStream_t stream,
-                              bool merge = true, const PagedKv& paged = PagedKv{}) {
+                              bool merge = true, const PagedKv& paged = PagedKv{}, bool partials = false) {
   if (paged.table && (paged.page <= 0 || paged.page % kTileN != 0 || !paged.seqlens || paged.stride < 0))
     return MLA_ERR_INVALID_ARG;
   // pages of 64 * odd keys: the score CTA copies 64 keys at a time
@@ -257,6 +258,7 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   p.heads = H;
   p.head_groups = H / 128;
   p.num_splits = splits;
+  p.partials = (splits > 1 || partials) ? 1 : 0;
   p.kv_rows = kv_rows;
   p.n_q = n_q;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -264,16 +266,16 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   p.part_ml = nullptr;
 
   __nv_bfloat16* part_o = nullptr;
-  if (splits > 1) {
+  if (p.partials) {
     part_o = static_cast<__nv_bfloat16*>(ws);
     p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + partial_ml_offset(H, n_q, splits));
   }
-  p.out = splits > 1 ? part_o : static_cast<__nv_bfloat16*>(o_lat);
+  p.out = p.partials ? part_o : static_cast<__nv_bfloat16*>(o_lat);
   CUtensorMap tout;
   {
     // the epilogue's output rows (o_lat, or the bf16 split partials) as [8 latent blocks][rows][64]:
     // boxes of 32 heads x 64 columns (an epilogue warp writes four of them)
-    const uint64_t d[3] = {64, (uint64_t)(splits > 1 ? splits : 1) * n_q * H, 8}, st[2] = {1024, 128};
+    const uint64_t d[3] = {64, (uint64_t)(p.partials ? splits : 1) * n_q * H, 8}, st[2] = {1024, 128};
     const uint32_t b[3] = {64, 32, 1};
     if (!make_map(&tout, p.out, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
@@ -281,7 +283,7 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   if (!set_smem(kern, kAttnSmem)) return MLA_ERR_CUDA;
   mla_status_t st = launch(true, kern, dim3((unsigned)(2 * units)), dim3(kAttnThreads), kAttnSmem, stream, tkv_s,
                            tpe, tqpe, tkv_v, tqa, tout, p);
-  if (st != MLA_OK || splits <= 1 || !merge) return st;
+  if (st != MLA_OK || splits <= 1 || !merge || partials) return st;
   const int64_t pairs_per_block = kMergeThreads / 64;   // two warps per (row, head)
   const int64_t merge_blocks = (n_q * H + pairs_per_block - 1) / pairs_per_block;
   return launch(true, merge_splits_kernel, dim3((unsigned)merge_blocks), dim3(kMergeThreads), 0, stream,

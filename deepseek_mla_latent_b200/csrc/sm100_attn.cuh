@@ -131,6 +131,7 @@ struct AttnParams {
   int heads;
   int head_groups;              // heads / 128
   int num_splits;
+  int partials;                 // 1: write the split partial form (O relative to m, and (m, l)) even for one split
   int64_t kv_rows;
   int64_t n_q;
   float scale_log2;             // softmax_scale * log2(e)
@@ -573,7 +574,7 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
           const float l1 = end_l[h], m1 = ntq > 1 ? m_slot(1)[h] : -INFINITY;
           const float m_fin = fmaxf(m_used, m1);
           const float lt = l * fast_exp2(m_used - m_fin) + (m1 == -INFINITY ? 0.f : l1 * fast_exp2(m1 - m_fin));
-          if (p.num_splits > 1) {
+          if (p.partials) {
             const int64_t slot = ((int64_t)u.sp * p.n_q + u.row) * p.heads + head0 + h;
             reinterpret_cast<float2*>(p.part_ml)[slot] = make_float2(m_fin, lt);
           }
@@ -581,7 +582,7 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
                             __float_as_uint(lt));
         }
       }
-    } else if (p.num_splits > 1 && g == 0) {
+    } else if (p.partials && g == 0) {
       // a split with no key contributes nothing to the merge
       const int64_t slot = ((int64_t)u.sp * p.n_q + u.row) * p.heads + head0 + h;
       reinterpret_cast<float2*>(p.part_ml)[slot] = make_float2(-INFINITY, 0.f);
@@ -800,7 +801,7 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
     const int c = (int)(warp >> 2);
 
     if (nt == 0) {
-      if (p.num_splits == 1) {
+      if (!p.partials) {
         uint4* dst = reinterpret_cast<uint4*>(p.o_lat + (u.row * p.heads + u.hg * 128 + h) * 512 + 256 * c);
         for (int v = 0; v < 32; ++v) dst[v] = make_uint4(0, 0, 0, 0);
       }
@@ -810,8 +811,8 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
       w = w && ptx::mbar_wait<true>(l_full, 0, kErrTimeoutPeer);   // also before exit: it writes here
       if (__all_sync(0xffffffffu, w)) {
         ptx::tc_fence_after();
-        const float inv = p.num_splits > 1 ? 1.f : 1.f / reinterpret_cast<const float*>(smem + L::kOffL)[h];
-        const int64_t row0 = (p.num_splits > 1 ? ((int64_t)u.sp * p.n_q + u.row) * p.heads : u.row * p.heads) +
+        const float inv = p.partials ? 1.f : 1.f / reinterpret_cast<const float*>(smem + L::kOffL)[h];
+        const int64_t row0 = (p.partials ? ((int64_t)u.sp * p.n_q + u.row) * p.heads : u.row * p.heads) +
                              u.hg * 128 + 32 * qd;
         // the value stages are idle once the last P V product finished: 16 KB of boxes per warp
         store_o_tma(smem + warp * 16384, tmem + lane_base + 256 * c, lane, inv, tmap_out, (int32_t)row0, 4 * c);

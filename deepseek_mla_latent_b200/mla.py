@@ -15,7 +15,7 @@ from typing import Optional
 
 import torch
 
-from ._lib import LIB, MLA_DTYPE_BF16, MlaDims, MlaError, _check, dims_from, make_dims  # noqa: F401
+from ._lib import LIB, MLA_DTYPE_BF16, MLA_ERR_UNSUPPORTED, MlaDims, MlaError, _check, dims_from, make_dims  # noqa: F401
 
 
 def _dtype(d: MlaDims) -> torch.dtype:
@@ -107,6 +107,51 @@ def attn_decode(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, kv: torch.Tens
                                batch, int(max_seqlen_k), _ptr(o_lat), _ptr(ws), wsb, num_splits, _stream(stream)),
            "mla_attn_decode")
     return o_lat
+
+
+def partials_workspace(d: MlaDims, batch: int, max_seqlen_k: int, num_splits: int = 0,
+                       device="cuda") -> torch.Tensor:
+    nbytes = int(LIB.mla_partials_workspace_size(ctypes.byref(d), batch, max_seqlen_k, num_splits))
+    if nbytes == 0:
+        raise MlaError(MLA_ERR_UNSUPPORTED, "mla_partials_workspace_size: dims without the partial form")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def attn_decode_partials(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, kv: torch.Tensor, pe: torch.Tensor,
+                         cu_seqlens_k: torch.Tensor, max_seqlen_k: int, ws: Optional[torch.Tensor] = None,
+                         num_splits: int = 0, stream=None) -> torch.Tensor:
+    """Decode attention leaving the split partials in the workspace (mla_attn_decode_partials);
+    returns the workspace (split_partials views it)."""
+    dt = _dtype(d)
+    batch = cu_seqlens_k.numel() - 1
+    H, C, R = d.num_heads, d.kv_lora_rank, d.qk_rope_head_dim
+    rs = _q_row_stride(q, d)
+    _need(q_abs, "q_abs", dt, (batch, H, C))
+    _need(q, "q", dt, contiguous=False)
+    _need(kv, "kv", dt)
+    _need(pe, "pe", dt)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    if kv.dim() != 2 or kv.shape[1] != C or pe.dim() != 2 or pe.shape[1] != R or pe.shape[0] != kv.shape[0]:
+        raise ValueError("kv must be [T, C] and pe [T, R]")
+    if ws is None:
+        ws = partials_workspace(d, batch, max_seqlen_k, num_splits, device=q_abs.device)
+    _need(ws, "workspace", torch.uint8)
+    _check(LIB.mla_attn_decode_partials(ctypes.byref(d), _ptr(q_abs), _ptr(q), rs, _ptr(kv), _ptr(pe), kv.shape[0],
+                                        _ptr(cu_seqlens_k), batch, int(max_seqlen_k), _ptr(ws), ws.numel(),
+                                        num_splits, _stream(stream)),
+           "mla_attn_decode_partials")
+    return ws
+
+
+def split_partials(d: MlaDims, ws: torch.Tensor, batch: int, splits: int):
+    """Views of the partial form mla_attn_decode_partials leaves in `ws`: O [splits, batch, H, C]
+    (bf16) and (m, l) [splits, batch, H, 2] (fp32), as include/mla.h lays them out."""
+    H, C = d.num_heads, d.kv_lora_rank
+    o_bytes = splits * batch * H * C * 2
+    off = (o_bytes + 255) // 256 * 256
+    o = ws[:o_bytes].view(torch.bfloat16).view(splits, batch, H, C)
+    ml = ws[off:off + splits * batch * H * 8].view(torch.float32).view(splits, batch, H, 2)
+    return o, ml
 
 
 def decode_out_workspace(d: MlaDims, batch: int, max_seqlen_k: int, num_splits: int = 0,

@@ -166,6 +166,36 @@ MLA_API mla_status_t mla_attn_decode_out(const mla_dims_t* dims, const void* q_a
                                          int64_t max_seqlen_k, const void* wkv_b, void* out, void* workspace,
                                          size_t workspace_bytes, int32_t num_splits, cudaStream_t stream);
 
+/* Bytes of workspace mla_attn_decode_partials needs (num_splits as for
+ * mla_attn_decode; 0 = automatic).  0 for dims the call does not support. */
+MLA_API size_t mla_partials_workspace_size(const mla_dims_t* dims, int32_t batch, int64_t max_seqlen_k,
+                                           int32_t num_splits);
+
+/* Decode attention without the split merge: the per-split partial results are
+ * left in the workspace for the caller to combine (a caller that spreads one
+ * sequence's key range over several GPUs merges partials from all of them).
+ * ("Absorb Path Execution", the score and latent value einsums over one key
+ * range each; the merge rule below is the log-sum-exp combination of
+ * softmaxes over disjoint key ranges.)  Arguments as in mla_attn_decode,
+ * without o_lat.  With S = mla_decode_num_splits(dims, batch, max_seqlen_k,
+ * num_splits), the workspace then holds, for split s of sequence b and head h:
+ *   O[s, b, h, 0..C-1]  bf16 at byte 0: sum over the split's keys j of
+ *                       2^(x_j - m) kv[j], where x_j = score_j * scale * log2(e);
+ *   (m, l)[s, b, h]     two fp32 at byte offset align256(S * batch * H * C * 2):
+ *                       m = the split's reference (>= max_j x_j - 8 when the split
+ *                       has keys), l = sum_j 2^(x_j - m);
+ * and o_lat[b, h] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with
+ * M = max_s m_s.  A split without keys has m = -inf, l = 0 and leaves its O
+ * rows unwritten.  Only the tensor-core kernels have this form (bf16
+ * DeepSeek-V3 shapes); other dims return MLA_ERR_UNSUPPORTED.
+ *   workspace  at least mla_partials_workspace_size(dims, batch, max_seqlen_k,
+ *              num_splits) bytes, 16-byte aligned. */
+MLA_API mla_status_t mla_attn_decode_partials(const mla_dims_t* dims, const void* q_abs, const void* q,
+                                              int64_t q_row_stride, const void* kv_cache, const void* pe_cache,
+                                              int64_t kv_rows, const int32_t* cu_seqlens_k, int32_t batch,
+                                              int64_t max_seqlen_k, void* workspace, size_t workspace_bytes,
+                                              int32_t num_splits, cudaStream_t stream);
+
 /* Size of the device scratch array behind mla_attn_decode_static_scratch. */
 #define MLA_STATIC_SCRATCH_BYTES (32u << 20)
 

@@ -195,3 +195,23 @@ def test_decode_split_plan(lib, batch, max_k):
     assert w9 >= 9 * batch * 128 * 512 * 2
     out = L.mla_decode_out_workspace_size(ctypes.byref(v3), batch, max_k, 9)
     assert out >= w9 + batch * 128 * 512 * 2
+
+
+def test_partials_entry_point_host_checks(lib):
+    """mla_attn_decode_partials exists only on the tensor-core kernels and needs its workspace."""
+    d = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
+    if lib.LIB.mla_kernel_family(ctypes.byref(d)) != 1:
+        pytest.skip("tensor-core family not selected")
+    n = lib.LIB.mla_partials_workspace_size(ctypes.byref(d), 8, 4096, 9)
+    assert n >= 9 * 8 * 128 * 512 * 2 + 9 * 8 * 128 * 8
+    assert lib.LIB.mla_partials_workspace_size(ctypes.byref(d), 8, 4096, 1) >= 8 * 128 * 512 * 2
+    f32 = lib.make_dims(8, 64, 32, 16, 32, "f32", 0.1)
+    assert lib.LIB.mla_partials_workspace_size(ctypes.byref(f32), 1, 128, 0) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.LIB.mla_attn_decode_partials(ctypes.byref(f32), fake, fake, 56, fake, fake, 128, fake, 1, 128, fake,
+                                          1 << 20, 0, None)
+    assert st == lib.MLA_ERR_UNSUPPORTED
+    # a workspace smaller than the size function reports is refused before any launch
+    st = lib.LIB.mla_attn_decode_partials(ctypes.byref(d), fake, fake, 128 * 192, fake, fake, 8 * 4096, fake, 8,
+                                          4096, fake, 16, 9, None)
+    assert st == lib.MLA_ERR_WORKSPACE

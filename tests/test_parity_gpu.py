@@ -95,22 +95,34 @@ def _sampled(index, pairs, num_splits=0):
         assert_close(got[cq[b]:cq[b + 1], h, :], r, w.dims.dtype, f"workload {index} seq {b} head {h}")
 
 
+def _cover_rows(n_seq, H, seed, row=0):
+    """One head per sequence (spread over the heads by a seeded draw) plus heads 0, 63, 64 and
+    127 of one sequence: every sequence, and with it every split unit of every row, is compared."""
+    rng = np.random.default_rng(seed)
+    pairs = {(b, int(rng.integers(0, H))) for b in range(n_seq)}
+    pairs |= {(row, h) for h in (0, H // 2 - 1, H // 2, H - 1)}
+    return sorted(pairs)
+
+
 def test_full_v3_decode_sampled():
-    _sampled(1, [(0, 0), (3, 77), (7, 127)])
+    _sampled(1, _cover_rows(8, 128, seed=11, row=3))
 
 
 def test_full_ragged_sampled():
     _, _, _, sk = wl.workload_shape(2)
     longest, shortest = int(np.argmax(sk)), int(np.argmin(sk))
-    _sampled(2, [(longest, 5), (shortest, 100), (31, 64)])
+    pairs = set(_cover_rows(len(sk), 128, seed=12, row=longest)) | {(shortest, 100)}
+    _sampled(2, sorted(pairs))
 
 
 def test_full_long_context_sampled():
-    _sampled(3, [(0, 1), (1, 126)])
+    _sampled(3, _cover_rows(2, 128, seed=13, row=1))
 
 
 def test_full_prefill_sampled():
-    _sampled(4, [(0, 3), (3, 120)])
+    """Every sequence of the chunked-prefill workload (all of its query rows, first and last
+    included, are compared for each pair), heads 0, 63, 64 and 127 of one of them."""
+    _sampled(4, _cover_rows(4, 128, seed=14, row=2))
 
 
 def _decode_out(w, num_splits=0):
@@ -141,9 +153,38 @@ def test_fp32_decode_out():
 
 def test_full_v3_decode_out_sampled():
     """The benchmark's launch configuration (mla_attn_decode_out at the full V3 decode size),
-    checked on (sequence, head) pairs the oracle computes one by one."""
+    checked on (sequence, head) pairs the oracle computes one by one: one head of every
+    sequence and heads 0, 63, 64 and 127 of one."""
     w = wl.workload(1)
     got = _decode_out(w)
-    ref = oracle.workload_naive(w, pairs=[(0, 0), (5, 64), (7, 127)])
+    ref = oracle.workload_naive(w, pairs=_cover_rows(8, 128, seed=15, row=5))
     for (b, h), r in ref.items():
         assert_close(got[b:b + 1, h, :], r, "bf16", f"seq {b} head {h}")
+
+
+@pytest.mark.parametrize("seqlens,splits", [([1000, 260, 0], 7), ([4096, 33], 0), ([300, 5], 1)])
+def test_v3_decode_partials_merge_to_the_decode_result(seqlens, splits):
+    """mla_attn_decode_partials: the partial form, merged here by the log-sum-exp rule the header
+    states, equals the oracle's o_lat; splits without keys carry m = -inf and l = 0."""
+    w = wl.make_workload("v3part", V3, [1] * len(seqlens), seqlens, seed=16)
+    d = mla.dims_from(w.dims)
+    dev = to_dev(w)
+    q_abs = mla.absorb_q(d, dev["q"], dev["wkv_b"])
+    ws = mla.attn_decode_partials(d, q_abs, dev["q"], dev["kv"], dev["pe"], dev["cu_k"], dev["max_k"],
+                                  num_splits=splits)
+    mla.device_status()
+    S = mla.decode_num_splits(d, w.batch, dev["max_k"], splits)
+    o, ml = mla.split_partials(d, ws, w.batch, S)
+    o = o.float().cpu().numpy().astype(np.float64)
+    ml = ml.cpu().numpy().astype(np.float64)
+    m, l = ml[..., 0], ml[..., 1]
+    M = np.max(m, axis=0)
+    wgt = np.where(np.isfinite(m), np.exp2(m - np.where(np.isfinite(M), M, 0.0)), 0.0)
+    den = np.sum(wgt * l, axis=0)
+    num = np.sum(wgt[..., None] * np.where(wgt[..., None] > 0, o, 0.0), axis=0)
+    merged = np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)
+    _, o_lat, _ = oracle.workload_absorb(w)
+    assert_close(merged, o_lat, "bf16", "merged partials")
+    for b, t in enumerate(seqlens):
+        if t == 0:
+            assert np.all(np.isneginf(m[:, b])) and np.all(l[:, b] == 0)
