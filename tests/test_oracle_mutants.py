@@ -167,3 +167,49 @@ def test_append_slot_off_by_one_is_caught(monkeypatch):
         return orig(kv_new, k_pe_new, gamma, eps, positions, np.asarray(slots) + 1, kv_cache, pe_cache, base)
     monkeypatch.setattr(oracle, "append_latent", off_by_one)
     assert _fails(APPEND_PINS)
+
+
+# ---------------------------------------------------------------- token-granular selection
+import test_sparse_oracle as TS  # noqa: E402
+from oracle import sparse_oracle  # noqa: E402
+
+
+def _select_mutant(kind):
+    def f(kv_cache, pe_cache, indices, counts):
+        kv_cache, pe_cache, idx = np.asarray(kv_cache), np.asarray(pe_cache), np.asarray(indices)
+        rows = kv_cache.shape[0]
+        kvs, pes, lens = [], [], []
+        for b, n in enumerate(counts):
+            n = int(n)
+            if kind == "count_minus_one":
+                n = max(0, n - 1)
+            sel = idx[b, :n].astype(np.int64)
+            if kind == "plus_one":
+                sel = sel + 1
+            elif kind == "unique":
+                sel = np.unique(sel)
+            if kind == "no_bounds":
+                sel = np.clip(sel, 0, rows - 1)
+            elif np.any((sel < 0) | (sel >= rows)):
+                raise ValueError("outside")
+            kvs.append(kv_cache[sel])
+            pes.append(pe_cache[sel])
+            lens.append(len(sel))
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        return np.concatenate(kvs), np.concatenate(pes), cu
+    return f
+
+
+SPARSE_PINS = [TS.test_gather_selected_hand_example, TS.test_selected_row_outside_the_cache_is_an_error,
+               TS.test_selecting_every_token_in_any_order_is_dense_decode,
+               TS.test_one_selected_token_returns_its_projected_value,
+               TS.test_selection_is_attention_over_those_tokens_only]
+
+
+@pytest.mark.parametrize("kind", ["plus_one", "count_minus_one", "unique", "no_bounds"])
+def test_sparse_pins_catch(monkeypatch, kind):
+    assert not _fails(SPARSE_PINS)
+    m = _select_mutant(kind)
+    monkeypatch.setattr(oracle, "gather_selected", m)
+    monkeypatch.setattr(sparse_oracle, "gather_selected", m)
+    assert _fails(SPARSE_PINS), kind
