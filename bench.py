@@ -165,7 +165,8 @@ def other_configs(args, dev, hbm, tf):
     us_step, us_attn, attn_flop, proj_flop, err = prefill_timings(w, 5, 3, prefill_check_pairs(w))
     tflops = attn_flop / (us_attn * 1e-6) / 1e12
     res[w.name] = {"step_us": us_step, "attn_call_us": us_attn, "attn_tflops": tflops, "bound": "tensor",
-                   "frac": tflops / tf, "parity_max_rel_err": err, "steps": 5}
+                   "frac": tflops / tf, "parity_max_rel_err": err, "steps": 5,
+                   "naive_path": naive_path_line(w, 5, 3, tf)}
     torch.cuda.empty_cache()
     return res
 
@@ -181,15 +182,17 @@ def parse_args():
     p.add_argument("--no-extra-configs", action="store_true",
                    help="skip the ragged, long-context and chunked-prefill workloads in the decode line")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
-    p.add_argument("--op", choices=["decode", "append", "paged", "expand", "prefill"], default="decode",
+    p.add_argument("--op", choices=["decode", "append", "paged", "expand", "prefill", "sparse"], default="decode",
                    help="decode: the decode step (the benchmark); append: the latent-cache append alone; "
                         "paged: the decode attention call over a paged cache beside the packed one; "
                         "expand: the latent KV expansion; prefill: the chunked-prefill step "
-                        "(workload 4 unless --workload names another prefill workload)")
+                        "(workload 4 unless --workload names another prefill workload); sparse: decode "
+                        "over --topk selected rows per sequence beside the dense call")
     p.add_argument("--batch", type=int, default=4, help="sequences per expansion call (--op expand)")
     p.add_argument("--seq-len", type=int, default=1024, help="tokens per sequence (--op expand)")
     p.add_argument("--tokens", type=int, default=65536, help="new tokens per append call (--op append)")
     p.add_argument("--page-size", type=int, default=64, help="tokens per page (--op paged)")
+    p.add_argument("--topk", type=int, default=2048, help="selected rows per sequence (--op sparse)")
     return p.parse_args()
 
 
@@ -221,27 +224,37 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# The sources that define the latent attention kernel (the roofline's dominant kernel): an ncu
+# summary of it stays valid while these files are unchanged.
+ATTN_KERNEL_SOURCES = ("common.cuh", "sm100_ptx.cuh", "sm100_attn.cuh")
+
+
+def kernel_source_hash(names=None) -> str:
+    """sha256 prefix over the library's CUDA sources (or the named files among them)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "deepseek_mla_latent_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
+        if name.endswith((".cu", ".cuh")) and (names is None or name in names):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
+def attn_kernel_hash() -> str:
+    return kernel_source_hash(ATTN_KERNEL_SOURCES)
+
+
 def profiled_traffic(workload_name: str):
     """DRAM bytes per launch of the attention kernel from the committed ncu summary,
-    if it was taken on the current kernel sources; else None."""
+    if it was taken on the current sources of that kernel; else None."""
     path = os.path.join(ROOT, "profiles", f"attn_decode_{workload_name}.md")
     try:
         text = open(path).read()
     except OSError:
         return None
-    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    m_hash = re.search(r"attn_kernel_source_hash:\s*([0-9a-f]+)", text)
     m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_bytes or m_hash.group(1) != attn_kernel_hash():
         return None
     return float(m_bytes.group(1))
 
@@ -504,6 +517,99 @@ def run_paged(args, rank, world):
         "gpu_launches": args.steps * (2 if mla.decode_num_splits(d, B, max_k, 0) > 1 else 1)}), flush=True)
 
 
+def run_sparse(args, rank, world):
+    """Time token-granular sparse decode (mla_attn_sparse_decode: the selected rows gathered into
+    one page per sequence, then the paged attention and split merge) with `--topk` random rows of
+    each sequence's cache, beside the dense decode call on the same cache; one JSON line (single GPU)."""
+    if world > 1 and rank != 0:
+        return
+    import torch
+    from deepseek_mla_latent_b200 import mla
+    from deepseek_mla_latent_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    dev = "cuda"
+    w = wl.workload(args.workload)
+    if any(s != 1 for s in w.seqlens_q):
+        raise SystemExit("--op sparse times decode workloads")
+    d = mla.dims_from(w.dims)
+    dt = torch.bfloat16
+    B, H, C = w.batch, w.dims.heads, w.dims.kv_lora_rank
+    topk = args.topk
+    rng = np.random.default_rng(0)
+    idx = np.full((B, topk), -1, dtype=np.int32)
+    counts = np.zeros(B, dtype=np.int32)
+    cu = w.cu_seqlens_k
+    for b in range(B):
+        n = min(topk, int(cu[b + 1] - cu[b]))
+        idx[b, :n] = rng.choice(np.arange(cu[b], cu[b + 1]), size=n, replace=False)
+        counts[b] = n
+    t = lambda a, ty=dt: torch.from_numpy(np.ascontiguousarray(a)).to(device=dev, dtype=ty)
+    per_copy = (w.kv.size + w.pe.size) * 2
+    copies = min(16, max(2, math.ceil(ROTATE_MIN_BYTES / per_copy) + 1))
+    q, wkv_b = t(w.q), t(w.wkv_b)
+    q_abs = mla.absorb_q(d, q, wkv_b)
+    ti, tc, cu_k = t(idx, torch.int32), t(counts, torch.int32), t(cu, torch.int32)
+    caches = [(t(w.kv), t(w.pe)) for _ in range(copies)]
+    o_lat = torch.empty((B, H, C), dtype=dt, device=dev)
+    ws_s = torch.empty(int(mla.LIB.mla_sparse_workspace_size(ctypes_byref(d), B, topk, 0)), dtype=torch.uint8,
+                       device=dev)
+    ws_d = mla.workspace(d, B, B, max(w.seqlens_k), 0, device=dev)
+    sparse = lambda k: mla.attn_sparse_decode(d, q_abs, q, caches[k][0], caches[k][1], ti, tc, o_lat=o_lat, ws=ws_s)
+    dense = lambda k: mla.attn_decode(d, q_abs, q, caches[k][0], caches[k][1], cu_k, max(w.seqlens_k), o_lat, ws_d)
+
+    def capture(fn):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        return gr
+
+    for i in range(max(3, args.warmup)):
+        sparse(i % copies)
+        dense(i % copies)
+    mla.device_status()
+    g_s = [capture(lambda k=k: sparse(k)) for k in range(copies)]
+    g_d = [capture(lambda k=k: dense(k)) for k in range(copies)]
+    torch.cuda.synchronize()
+
+    def timed(graphs):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(args.steps):
+            graphs[i % copies].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps * 1e3
+
+    us_s, us_d = timed(g_s), timed(g_d)
+    mla.device_status()
+    hbm, _, peak_kind = load_peaks()
+    sel = int(counts.sum())
+    # the selected rows are read once from the cache, written to and read back from the page scratch
+    alg_bytes = sel * KV_BYTES_PER_TOKEN + B * H * (C + w.dims.qk_rope + C) * 2
+    gbs = alg_bytes / (us_s * 1e-6) / 1e9
+    print(json.dumps({
+        "metric": "MLA token-sparse decode attention GB/s (1xB200)", "value": gbs, "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "us_per_call": us_s, "dense_us_per_call": us_d,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}_top{topk}", "batch": B, "seq_len_k": max(w.seqlens_k), "topk": topk,
+                   "selected_rows": sel, "num_splits": mla.decode_num_splits(d, B, topk, 0),
+                   "l2": f"{copies} rotating copies of the cache"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "peak_kind": peak_kind, "algorithmic_bytes": "selected rows once (1152 B each) + q_abs, q_pe in, "
+                                                                 "o_lat out"},
+        "gpu_launches": args.steps * (3 if mla.decode_num_splits(d, B, topk, 0) > 1 else 2)}), flush=True)
+
+
+def ctypes_byref(x):
+    import ctypes
+    return ctypes.byref(x)
+
+
 def prefill_attention_flop(w) -> float:
     """Algorithmic flop of the absorb-form attention of a chunked prefill: 2 * H * (576 + 512)
     per (query, visible key), query i of s new queries over t keys seeing t - s + i + 1."""
@@ -574,6 +680,88 @@ def prefill_timings(w, steps: int, warmup: int, check_pairs=()):
     return us_step, us_attn, attn_flop, proj_flop, err
 
 
+def expanded_prefill_flop(w):
+    """Algorithmic flop of the naive-path prefill: the expansion of every cache row
+    (2 * H * (Dn + Dv) * C per row) and the per-head attention, 2 * H * (Dn + R + Dv) per
+    (query, visible key) pair."""
+    dd = w.dims
+    expand = 2.0 * w.total_k * dd.heads * (dd.qk_nope + dd.v_head) * dd.kv_lora_rank
+    per_pair = 2.0 * dd.heads * (dd.qk_nope + dd.qk_rope + dd.v_head)
+    visible = sum(max(0, min(t, t - s + i + 1)) for s, t in zip(w.seqlens_q, w.seqlens_k) for i in range(s))
+    return expand, per_pair * visible
+
+
+def expanded_prefill_timings(w, steps: int, warmup: int, check_pairs=()):
+    """Time the naive-path chunked prefill on one GPU: mla_expand_kv over the whole packed cache,
+    then mla_attn_prefill_expanded.  Returns (us_step, us_attn, expansion flop, attention flop,
+    max relative error against the oracle on `check_pairs` or None)."""
+    import torch
+    from deepseek_mla_latent_b200 import mla
+    d = mla.dims_from(w.dims)
+    dt = torch.bfloat16
+    t = lambda a, ty=dt: torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=ty)
+    q, kv, pe, wkv_b = t(w.q), t(w.kv), t(w.pe), t(w.wkv_b)
+    cu_q, cu_k = t(w.cu_seqlens_q, torch.int32), t(w.cu_seqlens_k, torch.int32)
+    T, H = kv.shape[0], w.dims.heads
+    max_q = max(w.seqlens_q)
+    k = torch.empty((1, H, T, w.dims.qk_nope), dtype=dt, device="cuda")
+    v = torch.empty((1, H, T, w.dims.v_head), dtype=dt, device="cuda")
+    out = torch.empty((w.n_q, H, w.dims.v_head), dtype=dt, device="cuda")
+
+    def attention():
+        mla.attn_prefill_expanded(d, q, k[0], v[0], pe, cu_q, cu_k, max_q, out)
+
+    def step():
+        mla.expand_kv(d, kv, wkv_b, 1, T, eps=1e-6, k_nope=k, v=v)
+        attention()
+
+    err = None
+    if check_pairs:
+        import oracle
+        step()
+        mla.device_status()
+        got = out.float().cpu().numpy()
+        dd = w.dims
+        ref = oracle.mla_naive(w.q, oracle.rms_norm(w.kv, None, 1e-6), w.pe, w.wkv_b, w.cu_seqlens_q,
+                               w.cu_seqlens_k, dd.heads, dd.qk_nope, dd.qk_rope, dd.v_head, dd.scale,
+                               pairs=list(check_pairs))
+        cq = w.cu_seqlens_q
+        err = 0.0
+        for (b, h), r in ref.items():
+            e = float(np.max(np.abs(got[cq[b]:cq[b + 1], h, :] - r))) / max(float(np.max(np.abs(r))), 1e-30)
+            err = max(err, e)
+    for _ in range(max(3, warmup)):
+        step()
+    mla.device_status()
+
+    def timed(fn):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps * 1e3
+
+    us_step, us_attn = timed(step), timed(attention)
+    mla.device_status()
+    ex_flop, at_flop = expanded_prefill_flop(w)
+    return us_step, us_attn, ex_flop, at_flop, err
+
+
+def naive_path_line(w, steps, warmup, tf):
+    """The naive path of the same chunked prefill (expansion + per-head attention) for the JSON line."""
+    import torch
+    x_step, x_attn, ex_flop, at_flop, x_err = expanded_prefill_timings(w, steps, warmup, prefill_check_pairs(w))
+    torch.cuda.empty_cache()
+    at_tf = at_flop / (x_attn * 1e-6) / 1e12
+    return {"us_per_step": x_step, "attn_us_per_call": x_attn, "expand_us": x_step - x_attn,
+            "step_tflops": (ex_flop + at_flop) / (x_step * 1e-6) / 1e12, "attn_tflops": at_tf,
+            "attn_frac": at_tf / tf, "flop": {"expansion": ex_flop, "attention": at_flop},
+            "parity_max_rel_err": x_err}
+
+
 def prefill_check_pairs(w):
     """(sequence, head) pairs the prefill benchmark checks against the oracle: one head of every
     sequence (all its query rows, first and last included) and heads 0 and 127 of sequence 0."""
@@ -594,6 +782,7 @@ def run_prefill(args, rank, world):
     us_step, us_attn, attn_flop, proj_flop, err = prefill_timings(w, args.steps, args.warmup,
                                                                    prefill_check_pairs(w))
     hbm, tf, peak_kind = load_peaks()
+    naive = naive_path_line(w, args.steps, args.warmup, tf)
     attn_tf = attn_flop / (us_attn * 1e-6) / 1e12
     line = {
         "metric": "MLA absorb chunked-prefill TFLOP/s (1xB200)", "value": attn_tf, "unit": "TFLOP/s", "n_gpus": 1,
@@ -604,6 +793,7 @@ def run_prefill(args, rank, world):
                    "seq_len_k": max(w.seqlens_k),
                    "l2": "the step moves over 1 GB (q_abs and o_lat of 4096 rows), far above L2"},
         "parity": {"pairs": len(prefill_check_pairs(w)), "max_rel_err": err, "tol": 2e-2},
+        "naive_path": naive,
         "roofline": {"bound": "tensor", "achieved": attn_tf, "peak": tf, "unit": "TFLOP/s", "frac": attn_tf / tf,
                      "peak_kind": peak_kind + " (burst)"},
         "gpu_launches": args.steps * 3}
@@ -693,6 +883,9 @@ def main():
         return
     if args.op == "prefill":
         run_prefill(args, rank, world)
+        return
+    if args.op == "sparse":
+        run_sparse(args, rank, world)
         return
 
     import torch
@@ -795,6 +988,7 @@ def main():
             "clocks": clocks,
             "kernel_family": mla.kernel_family(d),
             "kernel_source_hash": kernel_source_hash(),
+            "attn_kernel_source_hash": attn_kernel_hash(),
         }
         # absorb_q + attention + output projection (with the split merge fused in), one launch each
         splits = mla.decode_num_splits(d, B, max(w.seqlens_k), 0)

@@ -42,6 +42,10 @@ SIGNATURES = {
     "mla_attn_paged": (_I32, [_DP, _P, _P, _I64, _P, _I64, _P, _I32, _I64, _P, _P, _I64, _I32, _P, _I64, _P, _P,
                               _SZ, _I32, _P]),
     "mla_out_proj": (_I32, [_DP, _P, _P, _P, _I64, _P]),
+    "mla_sparse_workspace_size": (_SZ, [_DP, _I32, _I32, _I32]),
+    "mla_attn_sparse_decode": (_I32, [_DP, _P, _P, _I64, _P, _P, _I64, _P, _I64, _P, _I32, _I32, _P, _P, _SZ, _I32,
+                                      _P]),
+    "mla_attn_prefill_expanded": (_I32, [_DP, _P, _I64, _P, _P, _P, _I64, _P, _P, _I32, _I64, _I64, _P, _P]),
     "mla_expand_kv": (_I32, [_DP, _P, _P, ctypes.c_float, _P, _I64, _I64, _P, _P, _P]),
     "mla_append_latent": (_I32, [_DP, _P, _P, _P, ctypes.c_float, ctypes.c_float, _P, _P, _I64, _P, _P, _I64, _P]),
     "mla_status_string": (ctypes.c_char_p, [_I32]),

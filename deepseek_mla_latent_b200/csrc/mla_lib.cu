@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "append.cuh"
+#include "gather.cuh"
 #include "sm100.cuh"
 
 namespace {
@@ -144,6 +145,29 @@ void* static_scratch_for_current_device() {
     g_scratch_ptr[dev] = ptr;
   }
   return g_scratch_ptr[dev];
+}
+
+// Sparse decode workspace: the gathered latent and rotary rows (one page of `page` rows per
+// sequence), the per-sequence key counts and block table, then the paged attention's workspace.
+struct SparseLayout {
+  int64_t page;
+  size_t off_pe, off_lens, off_table, off_attn, total;
+};
+
+bool sparse_layout(const Geo& g, int32_t batch, int32_t max_topk, int32_t num_splits, SparseLayout* s) {
+  const size_t esz = g.bf16 ? 2 : 4;
+  if ((g.C * esz) % 16 != 0 || (g.R * esz) % 16 != 0 || g.C * esz > 2 * 32 * 16 || g.R * esz > 32 * 16)
+    return false;
+  s->page = g.family == 1 ? ((int64_t)max_topk + 127) / 128 * 128 : (max_topk > 0 ? max_topk : 1);
+  if (s->page <= 0) s->page = 128;
+  const size_t rows = (size_t)batch * (size_t)s->page;
+  s->off_pe = align256(rows * g.C * esz);
+  s->off_lens = s->off_pe + align256(rows * g.R * esz);
+  s->off_table = s->off_lens + align256((size_t)batch * 4);
+  s->off_attn = s->off_table + align256((size_t)batch * 4);
+  const int splits = resolve_splits(g, batch, batch, max_topk, num_splits, true);
+  s->total = s->off_attn + workspace_bytes_for(g, batch, batch, max_topk, splits, true);
+  return true;
 }
 
 }  // namespace
@@ -407,6 +431,25 @@ mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* q_abs, c
                                batch, n_q_rows, splits, o_lat, workspace, stream);
 }
 
+mla_status_t mla_attn_prefill_expanded(const mla_dims_t* dims, const void* q, int64_t q_row_stride,
+                                       const void* k_nope, const void* v, const void* pe_cache, int64_t kv_rows,
+                                       const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch,
+                                       int64_t n_q_rows, int64_t max_seqlen_q, void* out, cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (g.family != 1) return MLA_ERR_UNSUPPORTED;
+  if (batch < 0 || n_q_rows < 0 || max_seqlen_q < 0 || kv_rows < 0 || q_row_stride < (int64_t)g.H * (g.Dn + g.R) ||
+      (q_row_stride * 2) % 16 != 0)
+    return MLA_ERR_INVALID_ARG;
+  if (batch == 0 || n_q_rows == 0) return MLA_OK;
+  if (!q || !cu_seqlens_q || !cu_seqlens_k || !out || !aligned16(q) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
+  if (kv_rows > 0 && (!k_nope || !v || !pe_cache || !aligned16(k_nope) || !aligned16(v) || !aligned16(pe_cache)))
+    return MLA_ERR_INVALID_ARG;
+  return mla::sm100::attention_expanded(q, q_row_stride, k_nope, v, pe_cache, kv_rows, cu_seqlens_q, cu_seqlens_k,
+                                        batch, n_q_rows, max_seqlen_q, g.H, g.scale, out, device_sm_count(), stream);
+}
+
 mla_status_t mla_attn_paged(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
                             const int32_t* cu_seqlens_q, int64_t n_q_rows, const int32_t* seqlens_k, int32_t batch,
                             int64_t max_seqlen_k, const void* kv_cache, const void* pe_cache, int64_t num_pages,
@@ -447,6 +490,55 @@ mla_status_t mla_attn_paged(const mla_dims_t* dims, const void* q_abs, const voi
                                     batch, n_q_rows, splits, o_lat, workspace, stream, paged);
   return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, nullptr, batch,
                                n_q_rows, splits, o_lat, workspace, stream, paged);
+}
+
+size_t mla_sparse_workspace_size(const mla_dims_t* dims, int32_t batch, int32_t max_topk, int32_t num_splits) {
+  Geo g;
+  SparseLayout sl;
+  if (!dims || !geo_of(dims, &g) || batch < 0 || max_topk < 0 || num_splits < 0 || num_splits > 256) return 0;
+  if (!sparse_layout(g, batch, max_topk, num_splits, &sl)) return 0;
+  return sl.total;
+}
+
+mla_status_t mla_attn_sparse_decode(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
+                                    const void* kv_cache, const void* pe_cache, int64_t kv_rows,
+                                    const int32_t* indices, int64_t index_stride, const int32_t* counts,
+                                    int32_t batch, int32_t max_topk, void* o_lat, void* workspace,
+                                    size_t workspace_bytes, int32_t num_splits, cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (batch < 0 || max_topk < 0 || kv_rows < 0 || num_splits < 0 || num_splits > 256 ||
+      index_stride < max_topk || q_row_stride < (int64_t)g.H * (g.Dn + g.R))
+    return MLA_ERR_INVALID_ARG;
+  SparseLayout sl;
+  if (!sparse_layout(g, batch, max_topk, num_splits, &sl)) return MLA_ERR_UNSUPPORTED;
+  if (batch == 0) return MLA_OK;
+  if ((int64_t)batch * sl.page >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  if (!q_abs || !q || !counts || !o_lat || !aligned16(q_abs) || !aligned16(q) || !aligned16(o_lat))
+    return MLA_ERR_INVALID_ARG;
+  if (max_topk > 0 && (!indices || !kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
+    return MLA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < sl.total || !aligned16(workspace)) return MLA_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  void* kv_sel = ws;
+  void* pe_sel = ws + sl.off_pe;
+  int32_t* lens = reinterpret_cast<int32_t*>(ws + sl.off_lens);
+  int32_t* table = reinterpret_cast<int32_t*>(ws + sl.off_table);
+  const size_t esz = g.bf16 ? 2 : 4;
+  const int kv_vec = (int)(g.C * esz / 16), pe_vec = (int)(g.R * esz / 16);
+  const int64_t per_block = mla::gather::kWarps;
+  int64_t bx = max_topk > 0 ? (max_topk + per_block - 1) / per_block : 1;
+  if (bx > 64) bx = 64;
+  mla::gather::select_rows_kernel<<<dim3((unsigned)bx, (unsigned)batch), mla::gather::kWarps * 32, 0, stream>>>(
+      static_cast<const uint4*>(kv_cache), static_cast<const uint4*>(pe_cache), kv_rows, indices, index_stride,
+      counts, max_topk, sl.page, kv_vec, pe_vec, static_cast<uint4*>(kv_sel), static_cast<uint4*>(pe_sel), lens,
+      table);
+  if (launch_status() != MLA_OK) return MLA_ERR_CUDA;
+  // the paged attention over one page per sequence: block table entry b = page b
+  return mla_attn_paged(dims, q_abs, q, q_row_stride, nullptr, batch, lens, batch, max_topk, kv_sel, pe_sel, batch,
+                        (int32_t)sl.page, table, 1, o_lat, ws + sl.off_attn, sl.total - sl.off_attn, num_splits,
+                        stream);
 }
 
 mla_status_t mla_expand_kv(const mla_dims_t* dims, const void* kv_c, const void* gamma, float eps,

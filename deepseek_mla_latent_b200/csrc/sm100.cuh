@@ -14,6 +14,7 @@
 #include "mla.h"
 #include "sm100_attn.cuh"
 #include "sm100_expand.cuh"
+#include "sm100_fmha.cuh"
 #include "sm100_merge_proj.cuh"
 #include "sm100_proj.cuh"
 
@@ -342,6 +343,58 @@ inline mla_status_t expand_kv(const void* kv_c, const void* gamma, float eps, co
   constexpr size_t smem = expand_smem_bytes();
   if (!set_smem(expand_kernel, smem)) return MLA_ERR_CUDA;
   return launch(false, expand_kernel, dim3((unsigned)grid), dim3(kExThreads), smem, stream, tx, tw, p);
+}
+
+// Per-head attention over expanded keys and values (the naive path of a chunked prefill):
+// out [n_q, H, 128] from q [n_q, H, 192] (row stride q_row_stride elements), K_nope and V
+// [H, kv_rows, 128] and pe [kv_rows, 64].
+inline mla_status_t attention_expanded(const void* q, int64_t q_row_stride, const void* k_nope, const void* v,
+                                       const void* pe, int64_t kv_rows, const int32_t* cu_q, const int32_t* cu_k,
+                                       int batch, int64_t n_q, int64_t max_seqlen_q, int H, float scale, void* out,
+                                       int sms, cudaStream_t stream) {
+  if (n_q >= (1LL << 31) || kv_rows >= (1LL << 31) || max_seqlen_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  const int64_t q_tiles = (max_seqlen_q + kFaTile - 1) / kFaTile;
+  const int64_t units = (int64_t)batch * H * q_tiles;
+  if (units == 0 || n_q == 0) return MLA_OK;
+  CUtensorMap tq, tk, tpe, tv;
+  // kv_rows may be 0 (every sequence empty); the maps still need one row
+  const uint64_t rows = kv_rows > 0 ? (uint64_t)kv_rows : 1;
+  const void* k_base = kv_rows > 0 ? k_nope : q;
+  const void* v_base = kv_rows > 0 ? v : q;
+  const void* pe_base = kv_rows > 0 ? pe : q;
+  {
+    // q as [n_q][H][192]: a box is 64 columns of one head for 128 query rows
+    const uint64_t d[3] = {192, (uint64_t)H, (uint64_t)n_q}, st[2] = {384, (uint64_t)q_row_stride * 2};
+    const uint32_t b[3] = {64, 1, (uint32_t)kFaTile};
+    if (!make_map(&tq, q, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
+  {
+    // K_nope and V as [H][rows][128]: a box is 64 columns of 128 keys of one head
+    const uint64_t d[3] = {128, rows, (uint64_t)H}, st[2] = {256, rows * 256};
+    const uint32_t b[3] = {64, (uint32_t)kFaTile, 1};
+    if (!make_map(&tk, k_base, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    if (!make_map(&tv, v_base, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
+  {
+    const uint64_t d[2] = {64, rows}, st[1] = {128};
+    const uint32_t b[2] = {64, (uint32_t)kFaTile};
+    if (!make_map(&tpe, pe_base, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
+  FaParams p;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.batch = batch;
+  p.heads = H;
+  p.q_tiles = (int)q_tiles;
+  p.n_units = units;
+  p.n_q = n_q;
+  p.kv_rows = kv_rows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  constexpr size_t smem = fa_smem_bytes();
+  if (!set_smem(fmha_kernel, smem)) return MLA_ERR_CUDA;
+  const int64_t grid = units < sms ? units : sms;
+  return launch(true, fmha_kernel, dim3((unsigned)grid), dim3(kFaThreads), smem, stream, tq, tk, tpe, tv, p);
 }
 
 }  // namespace sm100

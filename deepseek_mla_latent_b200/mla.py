@@ -294,6 +294,64 @@ def expand_kv(d: MlaDims, kv_c: torch.Tensor, wkv_b: torch.Tensor, batch: int, s
     return k_nope, v
 
 
+def attn_prefill_expanded(d: MlaDims, q: torch.Tensor, k_nope: torch.Tensor, v: torch.Tensor, pe: torch.Tensor,
+                          cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor, max_seqlen_q: int,
+                          out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Chunked-prefill attention on the naive path (mla_attn_prefill_expanded): out [n_q, H, Dv] from
+    q [n_q, H, Dn+R], K_nope [H, T, Dn] and V [H, T, Dv] (mla_expand_kv with batch 1 over the T
+    cache rows, viewed without the batch axis) and pe [T, R]."""
+    dt = _dtype(d)
+    H, Dn, R, Dv = d.num_heads, d.qk_nope_head_dim, d.qk_rope_head_dim, d.v_head_dim
+    rs = _q_row_stride(q, d)
+    n = q.shape[0]
+    T = pe.shape[0]
+    _need(q, "q", dt, contiguous=False)
+    _need(k_nope, "k_nope", dt, (H, T, Dn))
+    _need(v, "v", dt, (H, T, Dv))
+    _need(pe, "pe", dt, (T, R))
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    batch = cu_seqlens_q.numel() - 1
+    if cu_seqlens_k.numel() != batch + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
+    if out is None:
+        out = torch.empty((n, H, Dv), dtype=dt, device=q.device)
+    _need(out, "out", dt, (n, H, Dv))
+    _check(LIB.mla_attn_prefill_expanded(ctypes.byref(d), _ptr(q), rs, _ptr(k_nope), _ptr(v), _ptr(pe), T,
+                                         _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), batch, n, int(max_seqlen_q),
+                                         _ptr(out), _stream(stream)), "mla_attn_prefill_expanded")
+    return out
+
+
+def attn_sparse_decode(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, kv: torch.Tensor, pe: torch.Tensor,
+                       indices: torch.Tensor, counts: torch.Tensor, o_lat: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None, num_splits: int = 0, stream=None) -> torch.Tensor:
+    """Decode over a selected list of cache rows per sequence (mla_attn_sparse_decode): indices
+    [batch, max_topk] int32 (row b: the cache rows sequence b attends to), counts [batch] int32."""
+    dt = _dtype(d)
+    batch, max_topk = indices.shape
+    H, C, R = d.num_heads, d.kv_lora_rank, d.qk_rope_head_dim
+    rs = _q_row_stride(q, d)
+    _need(q_abs, "q_abs", dt, (batch, H, C))
+    _need(q, "q", dt, contiguous=False)
+    _need(kv, "kv", dt)
+    _need(pe, "pe", dt)
+    _need(indices, "indices", torch.int32, (batch, max_topk))
+    _need(counts, "counts", torch.int32, (batch,))
+    if kv.dim() != 2 or kv.shape[1] != C or pe.dim() != 2 or pe.shape[1] != R or pe.shape[0] != kv.shape[0]:
+        raise ValueError("kv must be [T, C] and pe [T, R]")
+    if o_lat is None:
+        o_lat = torch.empty((batch, H, C), dtype=dt, device=q_abs.device)
+    _need(o_lat, "o_lat", dt, (batch, H, C))
+    if ws is None:
+        nbytes = int(LIB.mla_sparse_workspace_size(ctypes.byref(d), batch, max_topk, num_splits))
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q_abs.device)
+    _check(LIB.mla_attn_sparse_decode(ctypes.byref(d), _ptr(q_abs), _ptr(q), rs, _ptr(kv), _ptr(pe), kv.shape[0],
+                                      _ptr(indices), max_topk, _ptr(counts), batch, max_topk, _ptr(o_lat), _ptr(ws),
+                                      ws.numel(), num_splits, _stream(stream)), "mla_attn_sparse_decode")
+    return o_lat
+
+
 def append_latent(d: MlaDims, kv_new: torch.Tensor, k_pe_new: torch.Tensor, positions: torch.Tensor,
                   slots: torch.Tensor, kv_cache: torch.Tensor, pe_cache: torch.Tensor,
                   gamma: Optional[torch.Tensor] = None, eps: float = 1e-6, rope_base: float = 10000.0,

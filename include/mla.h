@@ -243,6 +243,32 @@ MLA_API mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* 
                                     const void* kv_cache, const void* pe_cache, int64_t kv_rows, void* o_lat,
                                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Chunked-prefill attention on the naive path: per-head attention over keys
+ * and values expanded from the latent cache (by mla_expand_kv), with the
+ * rotary key shared by all heads.  ("Naive vs Absorb Attention
+ * Implementations in DeepSeek-V3", section "Naive Path Execution"; "Latent
+ * KV expansion with split" produces K_nope and V.)  For query i of the s_b new
+ * queries of sequence b (t_b keys; query i sees keys j <= t_b - s_b + i):
+ *   out[n,h,:] = sum_j softmax_j((q_nope[n,h] . K_nope[h,j] + q_pe[n,h] . pe[j]) * scale) V[h,j,:]
+ * which equals mla_attn_prefill_chunk followed by mla_out_proj in exact
+ * arithmetic (the pages' "mathematically identical" paths).
+ *   q          [n_q_rows, H, Dn+R] with row stride q_row_stride (nope first).
+ *   k_nope     [H, kv_rows, Dn] and v [H, kv_rows, Dv]: mla_expand_kv with
+ *              batch = 1, seq_len = kv_rows over the packed compressed cache
+ *              writes exactly this layout.
+ *   pe_cache   [kv_rows, R]; sequence b owns key rows cu_seqlens_k[b] ..
+ *              cu_seqlens_k[b+1]-1 of all three.
+ *   cu_seqlens_q, cu_seqlens_k, n_q_rows, max_seqlen_q as for mla_attn_prefill_chunk.
+ *   out        [n_q_rows, H, Dv] written (the attention output; no latent
+ *              projection follows).
+ * Needs no workspace.  Only the tensor-core kernels have this path (bf16
+ * DeepSeek-V3 shapes); other dims return MLA_ERR_UNSUPPORTED. */
+MLA_API mla_status_t mla_attn_prefill_expanded(const mla_dims_t* dims, const void* q, int64_t q_row_stride,
+                                               const void* k_nope, const void* v, const void* pe_cache,
+                                               int64_t kv_rows, const int32_t* cu_seqlens_q,
+                                               const int32_t* cu_seqlens_k, int32_t batch, int64_t n_q_rows,
+                                               int64_t max_seqlen_q, void* out, cudaStream_t stream);
+
 /* Attention over a PAGED latent cache, decode or chunked prefill.
  * ("What is DeepSeek Sparse Attention (DSA)?", section "How DSA works
  * (conceptual)": the serving runtime keeps the KV cache in pages for
@@ -278,6 +304,38 @@ MLA_API mla_status_t mla_attn_paged(const mla_dims_t* dims, const void* q_abs, c
                                     const int32_t* block_table, int64_t max_pages_per_seq, void* o_lat,
                                     void* workspace, size_t workspace_bytes, int32_t num_splits,
                                     cudaStream_t stream);
+
+/* Bytes of workspace mla_attn_sparse_decode needs (num_splits as for
+ * mla_attn_decode; 0 = automatic).  0 for dims the call does not support. */
+MLA_API size_t mla_sparse_workspace_size(const mla_dims_t* dims, int32_t batch, int32_t max_topk,
+                                         int32_t num_splits);
+
+/* Token-granular sparse decode: one query per sequence attends to a selected
+ * list of cache rows only ("What is DeepSeek Sparse Attention (DSA)? A clear,
+ * modern explainer", section "How DSA works (conceptual)": exact attention
+ * over the shortlisted tokens).  The selector itself is not part of the call.
+ *   indices      device int32 [batch, index_stride]: row b lists the cache rows
+ *                (of kv_cache / pe_cache, any rows, any order) sequence b
+ *                attends to; a row listed twice counts twice.
+ *   counts       device int32 [batch]: entries of row b that are used (clamped
+ *                to 0 .. max_topk); entries past them are never read.  A used
+ *                entry outside [0, kv_rows) reads as a key of zeros and sets
+ *                bit 1<<7 of the device error word.
+ *   max_topk     host upper bound of the counts; index_stride >= max_topk.
+ *   q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, o_lat [batch, H, C],
+ *   num_splits   as for mla_attn_decode.
+ *   workspace    at least mla_sparse_workspace_size(dims, batch, max_topk,
+ *                num_splits) bytes, 16-byte aligned.  The call copies the
+ *                selected rows there (one page per sequence) and runs the
+ *                paged attention (mla_attn_paged) over them.
+ * Needs C and R rows of a multiple of 16 bytes (C <= 512 bf16 / 256 fp32
+ * values, R <= 256 / 128); other dims return MLA_ERR_UNSUPPORTED. */
+MLA_API mla_status_t mla_attn_sparse_decode(const mla_dims_t* dims, const void* q_abs, const void* q,
+                                            int64_t q_row_stride, const void* kv_cache, const void* pe_cache,
+                                            int64_t kv_rows, const int32_t* indices, int64_t index_stride,
+                                            const int32_t* counts, int32_t batch, int32_t max_topk, void* o_lat,
+                                            void* workspace, size_t workspace_bytes, int32_t num_splits,
+                                            cudaStream_t stream);
 
 /* Output projection: out[n,h,d] = sum_c o_lat[n,h,c] * wkv_b[h*(Dn+Dv)+Dn+d, c].
  * ("Absorb Path Execution", the last einsum, with the tail rows of wkv_b.)

@@ -51,3 +51,23 @@ def test_prefill_flop_count_closed_form():
     w.dims, w.seqlens_q, w.seqlens_k = dims, sq, sk
     pairs = 4 * (1024 * 3073 + 1023 * 1024 // 2)
     assert bench.prefill_attention_flop(w) == pairs * 2 * 128 * (512 + 64 + 512)
+
+
+def test_naive_prefill_flop_count_closed_form():
+    """Workload 4 on the naive path: every one of the 4 x 4096 cache rows is expanded to all heads
+    (2 * 128 * 256 * 512 flop per row), and each (query, visible key) pair costs
+    2 * 128 * (128 + 64 + 128) flop."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from deepseek_mla_latent_b200 import workloads as wl
+    _, dims, sq, sk = wl.workload_shape(4)
+
+    class W:
+        pass
+    w = W()
+    w.dims, w.seqlens_q, w.seqlens_k = dims, sq, sk
+    w.total_k = sum(sk)
+    pairs = 4 * (1024 * 3073 + 1023 * 1024 // 2)
+    ex, at = bench.expanded_prefill_flop(w)
+    assert ex == 4 * 4096 * 2 * 128 * 256 * 512
+    assert at == pairs * 2 * 128 * (128 + 64 + 128)
