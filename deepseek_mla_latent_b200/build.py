@@ -25,28 +25,36 @@ def nvcc() -> str:
 
 
 def _newest_source_mtime() -> float:
-    paths = [os.path.join(ROOT, "include", "mla.h"), __file__]
-    for d, _, files in os.walk(os.path.join(HERE, "csrc")):
-        paths += [os.path.join(d, f) for f in files if f.endswith((".cu", ".cuh", ".h"))]
+    paths = [__file__]
+    for d in (os.path.join(ROOT, "include"), os.path.join(HERE, "csrc")):
+        for dd, _, files in os.walk(d):
+            paths += [os.path.join(dd, f) for f in files if f.endswith((".cu", ".cuh", ".h"))]
     return max(os.path.getmtime(p) for p in paths)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _newest_source_mtime():
-        return LIB
-    tmp = LIB + ".tmp"
+# Library variants: the product library, and a fault-injection build used only by the tests of
+# the bounded device waits (short wait limits and a host-set fault plan; see mla_fault_inject.h).
+VARIANTS = {"": ([], LIB),
+            "fault_inject": (["-DMLA_FAULT_INJECT"], os.path.join(HERE, "libmla_b200_fault_inject.so"))}
+
+
+def build(force: bool = False, verbose: bool = False, extra=(), variant: str = "") -> str:
+    flags, lib = VARIANTS[variant]
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= _newest_source_mtime():
+        return lib
+    tmp = lib + ".tmp"
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-cudart", "static", "--expt-relaxed-constexpr",
            "-I", os.path.join(ROOT, "include"), "-I", os.path.join(HERE, "csrc"),
-           *extra, *SOURCES, "-o", tmp]
+           *flags, *extra, *SOURCES, "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
-    print(LIB)
+    variant = "fault_inject" if "--fault-inject" in sys.argv else ""
+    print(build(force="--force" in sys.argv, verbose=True,
+                extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [], variant=variant))

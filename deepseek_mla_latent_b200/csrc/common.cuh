@@ -31,9 +31,21 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+#ifndef MLA_FAULT_INJECT
 // A wait gives up after this long (device time).  Legitimate waits in these
 // kernels last microseconds; a second means a peer will never arrive.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+__device__ __forceinline__ bool fault_plan(uint32_t) { return false; }
+#else
+// Fault-injection build (a separate library used only by the tests of the bounded waits):
+// waits give up after 2 ms, and the host sets a plan word that makes one copy go missing.
+constexpr uint64_t kWaitLimitNs = 2000000ull;
+
+// Plan bits: 1 = the score CTA of work unit 0 skips the rotary copy of its first score tile.
+__device__ uint32_t g_mla_fault_plan;
+__device__ __forceinline__ bool fault_plan(uint32_t bit) { return (*(volatile uint32_t*)&g_mla_fault_plan & bit) != 0; }
+#endif
 
 template <typename T> struct Elem;
 template <> struct Elem<float> {

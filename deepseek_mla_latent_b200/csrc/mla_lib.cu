@@ -12,6 +12,9 @@
 #include <mutex>
 
 #include "mla.h"
+#ifdef MLA_FAULT_INJECT
+#include "mla_fault_inject.h"
+#endif
 #include "common.cuh"
 #include "simt.cuh"
 #include "append.cuh"
@@ -620,6 +623,13 @@ mla_status_t mla_append_latent(const mla_dims_t* dims, const void* kv_new, const
   }
   return launch_status();
 }
+
+#ifdef MLA_FAULT_INJECT
+// Fault-injection build only (tests of the bounded waits): set the plan word the kernels read.
+mla_status_t mla_test_set_fault_plan(uint32_t plan) {
+  return cudaMemcpyToSymbol(mla::g_mla_fault_plan, &plan, sizeof(plan)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+#endif
 
 mla_status_t mla_device_status(cudaStream_t stream, uint32_t* code_out) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MLA_ERR_CUDA;

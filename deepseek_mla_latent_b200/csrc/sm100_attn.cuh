@@ -300,7 +300,9 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
         const int ps = jj % L::kPeSlots;
         bool w = ptx::mbar_wait(&pe_empty[ps], ((jj / L::kPeSlots) & 1) ^ 1, kErrTimeoutStageFree);
         if (!__all_sync(0xffffffffu, w)) break;
-        if (ptx::elect_one()) {
+        // (fault-injection builds only: a planned fault drops this copy, so the waits on it run out)
+        const bool dropped = jj == 0 && u.row == 0 && u.hg == 0 && u.sp == 0 && fault_plan(1u);
+        if (!dropped && ptx::elect_one()) {
           ptx::mbar_arrive_expect_tx(&pe_full[ps], L::kBlock);
           uint8_t* dst = smem + L::kOffPe + ps * L::kBlock;
           ptx::tma_load_2d(dst, tmap_pe, &pe_full[ps], 0, r0);

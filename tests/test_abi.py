@@ -215,3 +215,17 @@ def test_partials_entry_point_host_checks(lib):
     st = lib.LIB.mla_attn_decode_partials(ctypes.byref(d), fake, fake, 128 * 192, fake, fake, 8 * 4096, fake, 8,
                                           4096, fake, 16, 9, None)
     assert st == lib.MLA_ERR_WORKSPACE
+
+
+def test_fault_injection_hook_only_in_its_own_build(lib):
+    """mla_fault_inject.h's hook is exported by the fault-injection build and by nothing else."""
+    from deepseek_mla_latent_b200 import build
+    path = build.build(variant="fault_inject")
+    text = open(os.path.join(ROOT, "include", "mla_fault_inject.h")).read()
+    hooks = re.findall(r"MLA_API\s+[\w\s\*]*?\b(mla_\w+)\s*\(", text)
+    assert hooks == ["mla_test_set_fault_plan"]
+    variant = ctypes.CDLL(path)
+    for n in hooks + _declared_functions():
+        assert hasattr(variant, n), n
+    for n in hooks:
+        assert not hasattr(lib.LIB, n), f"the product library exports {n}"
