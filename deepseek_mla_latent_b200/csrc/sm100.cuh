@@ -241,9 +241,9 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   CUtensorMap tqa;
   {
     // q_abs viewed as [8 latent blocks][n_q * H rows][64 columns] (block stride 128 bytes): one box
-    // is a unit's 128 heads, all eight 64-column blocks (128 KB)
+    // is two 64-column blocks of a unit's 128 heads (32 KB)
     const uint64_t d[3] = {64, (uint64_t)n_q * H, 8}, st[2] = {1024, 128};
-    const uint32_t b[3] = {64, 128, 8};
+    const uint32_t b[3] = {64, 128, 2};
     if (!make_map(&tqa, q_abs, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
   AttnParams p;

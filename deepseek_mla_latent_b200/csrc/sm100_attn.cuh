@@ -240,7 +240,8 @@ struct CacheRows {
 namespace bar {
 // score CTA
 constexpr int kUFull = 0, kUEmpty = 5, kPeFull = 10, kPeEmpty = 12, kSFull = 22, kSFree = 24, kMBar = 26,
-              kPFree = 28, kQFull = 32, kQReady = 33, kEnd = 34, kScoreIdle = 35, kPSent = 36;
+              kPFree = 28, kQFull = 32, kQReady = 33, kEnd = 34, kScoreIdle = 35, kPSent = 36, kQPiece = 14,
+              kQFree = 18;
 // value CTA
 constexpr int kVFull = 0, kVEmpty = 2, kPFull = 4, kPvGo = 8, kPDone = 12, kOFinal = 16, kLFull = 17,
               kValueIdle = 18;
@@ -264,8 +265,10 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
   uint64_t* s_free = bars + bar::kSFree;       // [2] S read out (128 arrivals)
   uint64_t* m_bar = bars + bar::kMBar;         // [2] warpgroup g published the reference max of its tile (128)
   uint64_t* p_free = bars + bar::kPFree;       // [4] the value CTA finished the P V product of this P slot
-  uint64_t* q_full = bars + bar::kQFull;       // q_abs and q_pe landed
-  uint64_t* q_ready = bars + bar::kQReady;     // q_abs in TMEM, its landing zone free (256 arrivals)
+  uint64_t* q_full = bars + bar::kQFull;       // q_pe landed
+  uint64_t* q_piece = bars + bar::kQPiece;     // [4] q_abs blocks 2k, 2k+1 landed in latent slot 1 + k
+  uint64_t* q_free = bars + bar::kQFree;       // [4] those blocks moved into TMEM: slot 1 + k free (128 arrivals)
+  uint64_t* q_ready = bars + bar::kQReady;     // all of q_abs in TMEM (256 arrivals)
   uint64_t* end_bar = bars + bar::kEnd;        // warpgroup 1 published its (l, m) (128)
   uint64_t* p_sent = bars + bar::kPSent;       // [2] warpgroup g stored the P tiles of its score tile (4 warps)
   uint64_t* idle = bars + bar::kScoreIdle;
@@ -281,10 +284,15 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
       if (ptx::elect_one()) {
         ptx::prefetch_tmap(tmap_kv);
         ptx::prefetch_tmap(tmap_pe);
-        // q_abs (eight 64-column blocks of 128 heads, one copy) into latent slots 1-4, and q_pe
-        ptx::mbar_arrive_expect_tx(q_full, 128 * 1024 + 128 * 128);
-        ptx::tma_load_3d(smem + L::kOffQ, tmap_qabs, q_full, 0, (int)(u.row * p.heads + head0), 0);
+        // q_pe, and q_abs (eight 64-column blocks of 128 heads) in four 32 KB pieces into latent
+        // slots 1-4: each slot returns to the cache stream as soon as its piece is in TMEM
+        ptx::mbar_arrive_expect_tx(q_full, 128 * 128);
         ptx::tma_load_3d(smem + L::kOffQpe, tmap_qpe, q_full, 128, head0, (int)u.row);
+        for (int k = 0; k < 4; ++k) {
+          ptx::mbar_arrive_expect_tx(&q_piece[k], L::kLat);
+          ptx::tma_load_3d(smem + L::kOffQ + k * L::kLat, tmap_qabs, &q_piece[k], 0, (int)(u.row * p.heads + head0),
+                           2 * k);
+        }
       }
       __syncwarp();
       CacheRows<kPaged> cache;
@@ -315,7 +323,7 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
         for (int k = 0; k < L::kLatPerTile; ++k) {
           const int li = L::kLatPerTile * jj + k, slot = li % L::kLatSlots, use = li / L::kLatSlots;
           w = true;
-          if (use == 0 && slot >= 1) w = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax);   // held q_abs
+          if (use == 0 && slot >= 1) w = ptx::mbar_wait(&q_free[slot - 1], 0, kErrTimeoutSoftmax);   // held q_abs
           w = w && ptx::mbar_wait(&u_empty[slot], (use & 1) ^ 1, kErrTimeoutStageFree);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           if (ptx::elect_one()) {
@@ -341,13 +349,14 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
       for (int jj = (pe_issued > L::kPeSlots ? pe_issued - L::kPeSlots : 0); jj < pe_issued; ++jj)
         ptx::mbar_wait(&pe_full[jj % L::kPeSlots], (jj / L::kPeSlots) & 1, kErrTimeoutDrain);
       ptx::mbar_wait(q_full, 0, kErrTimeoutDrain);
+      for (int k = 0; k < 4; ++k) ptx::mbar_wait(&q_piece[k], 0, kErrTimeoutDrain);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ============================================================ MMA issuer
     if (ntp > 0) {
       constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, kTileQ, false, false);
-      bool ok = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax);
+      bool ok = ptx::mbar_wait(q_ready, 0, kErrTimeoutSoftmax) && ptx::mbar_wait(q_full, 0, kErrTimeoutTmaFull);
       ok = __all_sync(0xffffffffu, ok);
       // K-major operands, 128-byte rows, 8-row groups 1024 bytes apart; the start
       // address sits in the low bits, so byte offsets add directly (>> 4)
@@ -426,10 +435,12 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
     if (ntp > 0) {
       // q_abs row h, latent block b (columns 64b..) -> TMEM columns 32b.. (bf16 pairs); warpgroup g moves blocks 4g..4g+3
       const uint32_t v_base = ptx::map_peer(ptx::smem_u32(smem), 1);
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(q_full, 0, kErrTimeoutTmaFull));
-      if (ok) {
 #pragma unroll 1
-        for (int b = 4 * g; b < 4 * g + 4; ++b) {
+      for (int pc = 2 * g; ok && pc < 2 * g + 2; ++pc) {
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&q_piece[pc], 0, kErrTimeoutTmaFull));
+        if (!ok) break;
+#pragma unroll 1
+        for (int b = 2 * pc; b < 2 * pc + 2; ++b) {
           const uint8_t* src = smem + L::kOffQ + b * L::kBlock + h * 128;
           uint32_t r[32];
 #pragma unroll
@@ -439,9 +450,11 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
           }
           ptx::tmem_st32(tmem + lane_base + kColQ + 32 * b, r);
         }
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
+        // the piece's shared memory has been read into registers: its slot may be refilled
+        ptx::mbar_arrive(&q_free[pc]);
       }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
       ptx::mbar_arrive(q_ready);
 
       for (int jj = g; ok && jj < ntq; jj += 2) {
@@ -859,6 +872,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       }
       for (int s = 0; s < ValueLayout::kPSlots; ++s) ptx::mbar_init(&bars[bar::kPFree + s], 1);
       ptx::mbar_init(&bars[bar::kQFull], 1);
+      for (int k = 0; k < 4; ++k) {
+        ptx::mbar_init(&bars[bar::kQPiece + k], 1);
+        ptx::mbar_init(&bars[bar::kQFree + k], 128);
+      }
       ptx::mbar_init(&bars[bar::kQReady], 256);
       ptx::mbar_init(&bars[bar::kEnd], 128);
       ptx::mbar_init(&bars[bar::kScoreIdle], 1);
