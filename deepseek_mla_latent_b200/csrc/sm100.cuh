@@ -298,9 +298,11 @@ inline mla_status_t merge_out_proj(const void* ws, int splits, int64_t n_q, int 
                                    cudaStream_t stream) {
   if (splits < 2 || splits > kMpMaxSplits || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
   CUtensorMap tw;
-  const uint64_t wd[2] = {512, (uint64_t)H * 256}, wst[1] = {1024};
-  const uint32_t wb[2] = {64, 128};  // 64 latent columns x 128 value rows (K-major A)
-  if (!make_map(&tw, wkv_b, 2, wd, wst, wb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  // wkv_b as [8 latent blocks][H * 256 rows][64 columns]: one box is a head's 128 value rows, all
+  // eight 64-column K chunks (128 KB, K-major A chunks 16 KB apart)
+  const uint64_t wd[3] = {64, (uint64_t)H * 256, 8}, wst[2] = {1024, 128};
+  const uint32_t wb[3] = {64, 128, 8};
+  if (!make_map(&tw, wkv_b, 3, wd, wst, wb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   constexpr size_t smem = merge_proj_smem_bytes();
   if (!set_smem(merge_proj_kernel, smem)) return MLA_ERR_CUDA;
   const auto* part_o = static_cast<const __nv_bfloat16*>(ws);

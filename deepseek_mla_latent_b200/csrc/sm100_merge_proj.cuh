@@ -70,11 +70,11 @@ __global__ void __launch_bounds__(kMergeProjThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (warp == 0) {
-    if (ptx::elect_one())
-      for (int k = 0; k < L::kChunks; ++k) {
-        ptx::mbar_arrive_expect_tx(&wfull[k], L::kW);
-        ptx::tma_load_2d(smem + k * L::kW, &tmap_w, &wfull[k], 64 * k, h * 256 + 128);
-      }
+    if (ptx::elect_one()) {
+      // all eight K chunks of W_v[h] in one copy (the map's third axis steps through them)
+      ptx::mbar_arrive_expect_tx(&wfull[0], L::kChunks * L::kW);
+      ptx::tma_load_3d(smem, &tmap_w, &wfull[0], 0, h * 256 + 128, 0);
+    }
     __syncwarp();
   }
   ptx::griddep_wait();
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(kMergeProjThreads, 1)
     constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, kMpRows, false, false);
     bool ok = true;
     for (int k = 0; ok && k < L::kChunks; ++k) {
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&wfull[k], 0, kErrTimeoutTmaFull));
+      if (k == 0) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&wfull[0], 0, kErrTimeoutTmaFull));
       if (!ok) break;
       ptx::tc_fence_after();
       const uint32_t a = ptx::smem_u32(smem + k * L::kW), b = ptx::smem_u32(smem + L::kOffB + k * L::kB);
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kMergeProjThreads, 1)
   }
   // every weight copy has landed before the shared memory goes away
   if (warp == 0)
-    for (int k = 0; k < L::kChunks; ++k) ptx::mbar_wait(&wfull[k], 0, kErrTimeoutDrain);
+    ptx::mbar_wait(&wfull[0], 0, kErrTimeoutDrain);
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 0) ptx::tmem_dealloc(tmem, 32);
