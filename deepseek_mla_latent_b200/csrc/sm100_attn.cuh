@@ -676,10 +676,9 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
       __syncwarp();
       CacheRows<kPaged> cache;
       cache.init(p, u, lane);
-      // The first P tile arrives several microseconds in; loading values before then would only
-      // add to the start-up burst on HBM (these rows reach L2 through the score CTA meanwhile).
-      bool w0 = ptx::mbar_wait<true>(&p_full[0], 0, kErrTimeoutPeer);
-      for (int j = 0; w0 && j < nt; ++j) {
+      // The value tiles are the same rows the score CTA is loading: requested together they cost
+      // HBM one read, and the first P V product need not wait for a load after the first P.
+      for (int j = 0; j < nt; ++j) {
         const int st = j % L::kStages;
         const bool w = ptx::mbar_wait(&v_empty[st], ((j / L::kStages) & 1) ^ 1, kErrTimeoutStageFree);
         if (!__all_sync(0xffffffffu, w)) break;
