@@ -79,11 +79,19 @@ class DecodeBench:
                 "o_lat": torch.empty((B, H, C), dtype=dt, device=dev),
                 "out": torch.empty((B, H, Dv), dtype=dt, device=dev),
                 "ws": mla.workspace(d, B, B, max_k, 0, device=dev),
-                "ws_out": mla.decode_out_workspace(d, B, max_k, 0, device=dev)}
+                "ws_out": mla.decode_out_workspace(d, B, max_k, 0, device=dev),
+                "ws_fused": mla.decode_fused_workspace(d, B, max_k, 0, device=dev)}
         self.stream = torch.cuda.current_stream()
         inputs = self.inputs
 
         def step(k):
+            # the whole hot path through the public calls: absorb, then attention, split merge and
+            # output projection (one kernel where it fits: mla_attn_decode_fused)
+            q, kv, pe, wkv_b = inputs[k]
+            q_abs = mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
+            return mla.attn_decode_fused(d, q_abs, q, kv, pe, cu_k, max_k, wkv_b, bufs["out"], bufs["ws_fused"])
+
+        def step_two_kernels(k):
             q, kv, pe, wkv_b = inputs[k]
             q_abs = mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
             return mla.attn_decode_out(d, q_abs, q, kv, pe, cu_k, max_k, wkv_b, bufs["out"], bufs["ws_out"])
@@ -115,10 +123,11 @@ class DecodeBench:
         # The timed steps replay CUDA graphs captured from the same calls, so host-side launch
         # work does not leave the GPU idle inside the timed region.
         self.g_step = [capture(lambda k=k: step(k)) for k in range(self.copies)]
+        self.g_step2 = [capture(lambda k=k: step_two_kernels(k)) for k in range(self.copies)]
         self.g_attn = [capture(lambda k=k: attention_call(k)) for k in range(self.copies)]
         self.g_kern = [capture(lambda k=k: attention_kernel(k)) for k in range(self.copies)]
         for i in range(max(3, warmup)):
-            for g in (self.g_step, self.g_attn, self.g_kern):
+            for g in (self.g_step, self.g_step2, self.g_attn, self.g_kern):
                 g[i % self.copies].replay()
         mla.device_status()
 
@@ -925,6 +934,7 @@ def main():
         return statistics.mean(runs), len(runs)
 
     total_ms, reps = repeated(bench.g_step)
+    step2_ms, _ = repeated(bench.g_step2)
     # the attention call alone (attention kernel + split merge) and the attention kernel alone
     # (the split partials left in the workspace, mla_attn_decode_partials)
     attn_total_ms, _ = repeated(bench.g_attn)
@@ -973,6 +983,7 @@ def main():
                              "two events"},
             "repeats": reps,
             "tokens_per_s": world * B / (us_step / 1e6),
+            "step_two_kernel_us": step2_ms / args.steps * 1e3,
             "attn_kernel_us": mean_kern_ms * 1e3,
             "attn_call_us": mean_attn_ms * 1e3,
             "attn_cache_gbs": achieved_gbs,
@@ -990,9 +1001,13 @@ def main():
             "kernel_source_hash": kernel_source_hash(),
             "attn_kernel_source_hash": attn_kernel_hash(),
         }
-        # absorb_q + attention + output projection (with the split merge fused in), one launch each
+        # absorb_q, then one kernel for attention, split merge and output projection where it fits
+        # (2 x batch x splits CTAs at most the SMs), else attention + merge-projection
         splits = mla.decode_num_splits(d, B, max(w.seqlens_k), 0)
-        line["gpu_launches"] = args.steps * reps * 3
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        fused = splits >= 2 and 2 * B * (H // 128) * splits <= sms
+        line["gpu_launches"] = args.steps * reps * (2 if fused else 3)
+        line["config"]["fused_step"] = fused
         line["config"]["num_splits"] = splits
         if world == 1 and not args.no_extra_configs:
             del bench

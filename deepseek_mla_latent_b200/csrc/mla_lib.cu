@@ -82,6 +82,9 @@ int simt_auto_splits(int64_t n_q_rows, int H, int64_t max_seqlen_k) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Control words of mla_attn_decode_fused at the start of its workspace.
+constexpr size_t kFusedCtrlBytes = 256;
+
 size_t simt_workspace(const Geo& g, int64_t n_q_rows, int splits) {
   if (splits <= 1) return 0;
   return align256((size_t)splits * n_q_rows * g.H * g.C * sizeof(float)) +
@@ -399,6 +402,47 @@ mla_status_t mla_attn_decode_out(const mla_dims_t* dims, const void* q_abs, cons
                                     max_seqlen_k, o_lat, ws, ws_bytes, num_splits, stream);
   if (st != MLA_OK) return st;
   return mla_out_proj(dims, o_lat, wkv_b, out, batch, stream);
+}
+
+size_t mla_decode_fused_workspace_size(const mla_dims_t* dims, int32_t batch, int64_t max_seqlen_k,
+                                       int32_t num_splits) {
+  Geo g;
+  if (!dims || !geo_of(dims, &g) || batch < 0 || max_seqlen_k < 0 || num_splits < 0 || num_splits > 256) return 0;
+  const int splits = resolve_splits(g, batch, batch, max_seqlen_k, num_splits, true);
+  size_t rest = mla_decode_out_workspace_size(dims, batch, max_seqlen_k, num_splits);
+  if (g.family == 1) rest = std::max(rest, mla::sm100::workspace_bytes(g.H, batch, splits, /*partials=*/true));
+  return kFusedCtrlBytes + rest;
+}
+
+mla_status_t mla_attn_decode_fused(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
+                                   const void* kv_cache, const void* pe_cache, int64_t kv_rows,
+                                   const int32_t* cu_seqlens_k, int32_t batch, int64_t max_seqlen_k,
+                                   const void* wkv_b, void* out, void* workspace, size_t workspace_bytes,
+                                   int32_t num_splits, cudaStream_t stream) {
+  Geo g;
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
+  if (batch < 0 || max_seqlen_k < 0 || kv_rows < 0 || num_splits < 0 || num_splits > 256 ||
+      q_row_stride < (int64_t)g.H * (g.Dn + g.R))
+    return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  const size_t need = mla_decode_fused_workspace_size(dims, batch, max_seqlen_k, num_splits);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return MLA_ERR_WORKSPACE;
+  if (!q_abs || !q || !cu_seqlens_k || !wkv_b || !out || !aligned16(q_abs) || !aligned16(q) ||
+      !aligned16(wkv_b) || !aligned16(out))
+    return MLA_ERR_INVALID_ARG;
+  if (kv_rows > 0 && (!kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))
+    return MLA_ERR_INVALID_ARG;
+  uint32_t* ctrl = static_cast<uint32_t*>(workspace);
+  void* rest = static_cast<char*>(workspace) + kFusedCtrlBytes;
+  const size_t rest_bytes = workspace_bytes - kFusedCtrlBytes;
+  const int splits = resolve_splits(g, batch, batch, max_seqlen_k, num_splits, true);
+  if (g.family == 1 && (q_row_stride * 2) % 16 == 0 && mla::sm100::fused_fits(batch, g.H, splits, device_sm_count()))
+    return mla::sm100::decode_fused(q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_k, batch, g.H,
+                                    splits, g.scale, wkv_b, out, rest, ctrl, stream);
+  // more units than can be resident at once, or a single split: the two-kernel path
+  return mla_attn_decode_out(dims, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_k, batch,
+                             max_seqlen_k, wkv_b, out, rest, rest_bytes, num_splits, stream);
 }
 
 mla_status_t mla_attn_prefill_chunk(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,

@@ -16,6 +16,7 @@
 #include "sm100_expand.cuh"
 #include "sm100_fmha.cuh"
 #include "sm100_merge_proj.cuh"
+#include "sm100_decode_fused.cuh"
 #include "sm100_proj.cuh"
 
 namespace mla {
@@ -196,23 +197,30 @@ struct PagedKv {
   int page = 0;
 };
 
-// merge = false (split runs only): leave the partials in the workspace for merge_out_proj
-// instead of merging them into o_lat.  partials = true: write the partial form (also for one
-// split) and never merge; o_lat is not used.
-inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_stride, const void* kv, const void* pe,
-                              int64_t kv_rows, const int32_t* cu_q, const int32_t* cu_k, int batch, int64_t n_q,
-                              int H, int splits, float scale, void* o_lat, void* ws, cudaStream_t stream,
-                              bool merge = true, const PagedKv& paged = PagedKv{}, bool partials = false) {
+// The tensor maps and parameters of the latent attention kernel for one call.
+struct AttnLaunch {
+  CUtensorMap tkv_s, tpe, tqpe, tkv_v, tqa, tout;
+  AttnParams p;
+  int64_t units = 0;
+  __nv_bfloat16* part_o = nullptr;
+};
+
+inline mla_status_t prepare_attention(AttnLaunch& L, const void* q_abs, const void* q, int64_t q_row_stride,
+                                      const void* kv, const void* pe, int64_t kv_rows, const int32_t* cu_q,
+                                      const int32_t* cu_k, int batch, int64_t n_q, int H, int splits, float scale,
+                                      void* o_lat, void* ws, const PagedKv& paged, bool partials) {
+  CUtensorMap &tkv_s = L.tkv_s, &tpe = L.tpe, &tqpe = L.tqpe, &tkv_v = L.tkv_v, &tqa = L.tqa, &tout = L.tout;
+  AttnParams& p = L.p;
   if (paged.table && (paged.page <= 0 || paged.page % kTileN != 0 || !paged.seqlens || paged.stride < 0))
     return MLA_ERR_INVALID_ARG;
   // pages of 64 * odd keys: the score CTA copies 64 keys at a time
   const uint32_t score_rows = paged.table && paged.page % kTileQ != 0 ? kTileN : kTileQ;
   if (kv_rows >= (1LL << 31) || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
   const int64_t units = n_q * (H / 128) * splits;
+  L.units = units;
   if (units == 0) return MLA_OK;
   if (2 * units >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
   if ((uint64_t)n_q * H * (uint64_t)splits >= (1ULL << 31)) return MLA_ERR_INVALID_ARG;
-  CUtensorMap tkv_s, tpe, tqpe, tkv_v;
   // kv_rows may be 0 (every sequence empty); the maps still need one row.
   const uint64_t rows = kv_rows > 0 ? (uint64_t)kv_rows : 1;
   const void* kv_base = kv_rows > 0 ? kv : q_abs;   // any valid 16-byte aligned address for an unused map
@@ -238,7 +246,6 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
     const uint32_t b[3] = {64, 128, 1};
     if (!make_map(&tqpe, q, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
-  CUtensorMap tqa;
   {
     // q_abs viewed as [8 latent blocks][n_q * H rows][64 columns] (block stride 128 bytes): one box
     // is two 64-column blocks of a unit's 128 heads (32 KB)
@@ -246,7 +253,6 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
     const uint32_t b[3] = {64, 128, 2};
     if (!make_map(&tqa, q_abs, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
-  AttnParams p;
   p.q_abs = static_cast<const __nv_bfloat16*>(q_abs);
   p.cu_q = cu_q;
   p.cu_k = cu_k;
@@ -272,7 +278,6 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
     p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + partial_ml_offset(H, n_q, splits));
   }
   p.out = p.partials ? part_o : static_cast<__nv_bfloat16*>(o_lat);
-  CUtensorMap tout;
   {
     // the epilogue's output rows (o_lat, or the bf16 split partials) as [8 latent blocks][rows][64]:
     // boxes of 32 heads x 64 columns (an epilogue warp writes four of them)
@@ -280,16 +285,69 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
     const uint32_t b[3] = {64, 32, 1};
     if (!make_map(&tout, p.out, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
+  L.part_o = part_o;
+  return MLA_OK;
+}
+
+// merge = false (split runs only): leave the partials in the workspace for merge_out_proj
+// instead of merging them into o_lat.  partials = true: write the partial form (also for one
+// split) and never merge; o_lat is not used.
+inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_stride, const void* kv, const void* pe,
+                              int64_t kv_rows, const int32_t* cu_q, const int32_t* cu_k, int batch, int64_t n_q,
+                              int H, int splits, float scale, void* o_lat, void* ws, cudaStream_t stream,
+                              bool merge = true, const PagedKv& paged = PagedKv{}, bool partials = false) {
+  AttnLaunch L;
+  mla_status_t st = prepare_attention(L, q_abs, q, q_row_stride, kv, pe, kv_rows, cu_q, cu_k, batch, n_q, H, splits,
+                                      scale, o_lat, ws, paged, partials);
+  if (st != MLA_OK || L.units == 0) return st;
+  const AttnParams& p = L.p;
   auto kern = paged.table ? latent_attn_kernel<true> : latent_attn_kernel<false>;
   if (!set_smem(kern, kAttnSmem)) return MLA_ERR_CUDA;
-  mla_status_t st = launch(true, kern, dim3((unsigned)(2 * units)), dim3(kAttnThreads), kAttnSmem, stream, tkv_s,
-                           tpe, tqpe, tkv_v, tqa, tout, p);
+  st = launch(true, kern, dim3((unsigned)(2 * L.units)), dim3(kAttnThreads), kAttnSmem, stream, L.tkv_s, L.tpe,
+              L.tqpe, L.tkv_v, L.tqa, L.tout, p);
   if (st != MLA_OK || splits <= 1 || !merge || partials) return st;
   const int64_t pairs_per_block = kMergeThreads / 64;   // two warps per (row, head)
   const int64_t merge_blocks = (n_q * H + pairs_per_block - 1) / pairs_per_block;
   return launch(true, merge_splits_kernel, dim3((unsigned)merge_blocks), dim3(kMergeThreads), 0, stream,
-                (const __nv_bfloat16*)part_o, (const float*)p.part_ml, splits, n_q, H,
+                (const __nv_bfloat16*)L.part_o, (const float*)p.part_ml, splits, n_q, H,
                 static_cast<__nv_bfloat16*>(o_lat));
+}
+
+// Decode attention, split merge and output projection in one kernel (decode_fused_kernel).
+// ws: the attention's split partials, then 256 bytes of control words (zero before the call,
+// left zero after it).  Needs splits >= 2 and no more CTAs (2 per unit) than SMs.
+inline bool fused_fits(int batch, int H, int splits, int sms) {
+  return splits >= 2 && splits <= kMpMaxSplits && (int64_t)batch * (H / 128) * splits * 2 <= sms;
+}
+
+inline mla_status_t decode_fused(const void* q_abs, const void* q, int64_t q_row_stride, const void* kv,
+                                 const void* pe, int64_t kv_rows, const int32_t* cu_k, int batch, int H, int splits,
+                                 float scale, const void* wkv_b, void* out, void* ws, uint32_t* ctrl,
+                                 cudaStream_t stream) {
+  AttnLaunch L;
+  mla_status_t st = prepare_attention(L, q_abs, q, q_row_stride, kv, pe, kv_rows, nullptr, cu_k, batch, batch, H,
+                                      splits, scale, nullptr, ws, PagedKv{}, /*partials=*/true);
+  if (st != MLA_OK || L.units == 0) return st;
+  CUtensorMap tw;
+  {
+    // wkv_b as [8 latent blocks][H * 256 rows][64 columns]: one box is a head's 128 value rows
+    const uint64_t d[3] = {64, (uint64_t)H * 256, 8}, stw[2] = {1024, 128};
+    const uint32_t b[3] = {64, 128, 8};
+    if (!make_map(&tw, wkv_b, 3, d, stw, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+  }
+  FusedParams f;
+  f.ctrl = ctrl;
+  f.row_tiles = (batch + kMpRows - 1) / kMpRows;
+  f.n_items = H * f.row_tiles;
+  f.part_o = L.part_o;
+  f.part_ml = L.p.part_ml;
+  f.num_splits = splits;
+  f.n_q = batch;
+  f.heads = H;
+  f.out = static_cast<__nv_bfloat16*>(out);
+  if (!set_smem(decode_fused_kernel, kAttnSmem)) return MLA_ERR_CUDA;
+  return launch(true, decode_fused_kernel, dim3((unsigned)(2 * L.units)), dim3(kAttnThreads), kAttnSmem, stream,
+                L.tkv_s, L.tpe, L.tqpe, L.tkv_v, L.tqa, L.tout, tw, L.p, f);
 }
 
 // The output projection of a split decode with the split merge fused in: out [n_q, H, 128] from the

@@ -837,15 +837,13 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
 }
 
 // ---------------------------------------------------------------- the kernel
-// One cluster of two CTAs per work unit (query row, 128-head group, split).
-// kPaged: the cache is read through a block table (one instance per cache kind).
+// The work of one CTA of a pair on its unit (query row, 128-head group, split): set-up, then the
+// score or the value role.  Returns the TMEM base, still allocated (attn_teardown frees it).
 template <bool kPaged>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
-    latent_attn_kernel(const __grid_constant__ CUtensorMap tmap_kv_score, const __grid_constant__ CUtensorMap tmap_pe,
-                       const __grid_constant__ CUtensorMap tmap_qpe, const __grid_constant__ CUtensorMap tmap_kv_value,
-                       const __grid_constant__ CUtensorMap tmap_qabs, const __grid_constant__ CUtensorMap tmap_out,
-                       const AttnParams p) {
-  extern __shared__ __align__(1024) uint8_t smem[];
+__device__ __forceinline__ uint32_t attn_unit(uint8_t* smem, const CUtensorMap* tmap_kv_score,
+                                              const CUtensorMap* tmap_pe, const CUtensorMap* tmap_qpe,
+                                              const CUtensorMap* tmap_kv_value, const CUtensorMap* tmap_qabs,
+                                              const CUtensorMap* tmap_out, const AttnParams& p) {
   const uint32_t warp = ptx::warp_id();
   const uint32_t rank = ptx::cluster_rank();
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (rank == 0 ? ScoreLayout::kOffBars : ValueLayout::kOffBars));
@@ -913,14 +911,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     u.nt = 0;
   }
   if (rank == 0)
-    score_role<kPaged>(smem, tmem, u, p, &tmap_kv_score, &tmap_pe, &tmap_qpe, &tmap_qabs);
+    score_role<kPaged>(smem, tmem, u, p, tmap_kv_score, tmap_pe, tmap_qpe, tmap_qabs);
   else
-    value_role<kPaged>(smem, tmem, u, p, &tmap_kv_value, &tmap_out);
+    value_role<kPaged>(smem, tmem, u, p, tmap_kv_value, tmap_out);
+  return tmem;
+}
 
+__device__ __forceinline__ void attn_teardown(uint32_t tmem) {
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, 512);
+  if (ptx::warp_id() == kMmaWarp) ptx::tmem_dealloc(tmem, 512);
   ptx::cluster_sync();   // neither CTA's shared memory goes away while the partner may still write into it
+}
+
+// One cluster of two CTAs per work unit (query row, 128-head group, split).
+// kPaged: the cache is read through a block table (one instance per cache kind).
+template <bool kPaged>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
+    latent_attn_kernel(const __grid_constant__ CUtensorMap tmap_kv_score, const __grid_constant__ CUtensorMap tmap_pe,
+                       const __grid_constant__ CUtensorMap tmap_qpe, const __grid_constant__ CUtensorMap tmap_kv_value,
+                       const __grid_constant__ CUtensorMap tmap_qabs, const __grid_constant__ CUtensorMap tmap_out,
+                       const AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t tmem = attn_unit<kPaged>(smem, &tmap_kv_score, &tmap_pe, &tmap_qpe, &tmap_kv_value, &tmap_qabs,
+                                          &tmap_out, p);
+  attn_teardown(tmem);
 }
 
 // Merge split partials: o = sum_s 2^{m_s - M} O_s / sum_s 2^{m_s - M} l_s, M = max_s m_s,

@@ -189,6 +189,43 @@ def attn_decode_out(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, kv: torch.
     return out
 
 
+def decode_fused_workspace(d: MlaDims, batch: int, max_seqlen_k: int, num_splits: int = 0,
+                           device="cuda") -> torch.Tensor:
+    """Workspace of mla_attn_decode_fused, zero-filled (its control words must start at zero)."""
+    nbytes = int(LIB.mla_decode_fused_workspace_size(ctypes.byref(d), batch, max_seqlen_k, num_splits))
+    return torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def attn_decode_fused(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, kv: torch.Tensor, pe: torch.Tensor,
+                      cu_seqlens_k: torch.Tensor, max_seqlen_k: int, wkv_b: torch.Tensor,
+                      out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, num_splits: int = 0,
+                      stream=None) -> torch.Tensor:
+    """Decode attention, split merge and output projection, in one kernel where it fits
+    (mla_attn_decode_fused).  ws must come from decode_fused_workspace (or be zero-filled)."""
+    dt = _dtype(d)
+    batch = cu_seqlens_k.numel() - 1
+    H, C, R, Dn, Dv = d.num_heads, d.kv_lora_rank, d.qk_rope_head_dim, d.qk_nope_head_dim, d.v_head_dim
+    rs = _q_row_stride(q, d)
+    _need(q_abs, "q_abs", dt, (batch, H, C))
+    _need(q, "q", dt, contiguous=False)
+    _need(kv, "kv", dt)
+    _need(pe, "pe", dt)
+    _need(wkv_b, "wkv_b", dt, (H * (Dn + Dv), C))
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    if kv.dim() != 2 or kv.shape[1] != C or pe.dim() != 2 or pe.shape[1] != R or pe.shape[0] != kv.shape[0]:
+        raise ValueError("kv must be [T, C] and pe [T, R]")
+    if out is None:
+        out = torch.empty((batch, H, Dv), dtype=dt, device=q_abs.device)
+    _need(out, "out", dt, (batch, H, Dv))
+    if ws is None:
+        ws = decode_fused_workspace(d, batch, max_seqlen_k, num_splits, device=q_abs.device)
+    _need(ws, "workspace", torch.uint8)
+    _check(LIB.mla_attn_decode_fused(ctypes.byref(d), _ptr(q_abs), _ptr(q), rs, _ptr(kv), _ptr(pe), kv.shape[0],
+                                     _ptr(cu_seqlens_k), batch, int(max_seqlen_k), _ptr(wkv_b), _ptr(out), _ptr(ws),
+                                     ws.numel(), num_splits, _stream(stream)), "mla_attn_decode_fused")
+    return out
+
+
 def attn_prefill_chunk(d: MlaDims, q_abs: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
                        cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int, kv: torch.Tensor,
                        pe: torch.Tensor, o_lat: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,

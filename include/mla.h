@@ -196,6 +196,35 @@ MLA_API mla_status_t mla_attn_decode_partials(const mla_dims_t* dims, const void
                                               int64_t max_seqlen_k, void* workspace, size_t workspace_bytes,
                                               int32_t num_splits, cudaStream_t stream);
 
+/* Bytes of workspace mla_attn_decode_fused needs (num_splits as for
+ * mla_attn_decode; 0 = automatic). */
+MLA_API size_t mla_decode_fused_workspace_size(const mla_dims_t* dims, int32_t batch, int64_t max_seqlen_k,
+                                               int32_t num_splits);
+
+/* mla_attn_decode_out in one kernel where it fits: the attention, the split
+ * merge and the output projection ("Absorb Path Execution": the score and
+ * latent value einsums, then the last einsum) run as one grid, each CTA
+ * loading its head's value rows of wkv_b while the other units finish, then
+ * merging and projecting once every unit's partials are in memory (a
+ * grid-wide counter with a bounded wait).  Arguments and result as for
+ * mla_attn_decode_out (bit-identical output), except the workspace:
+ *   workspace  at least mla_decode_fused_workspace_size(dims, batch,
+ *              max_seqlen_k, num_splits) bytes, 16-byte aligned.  Its first
+ *              256 bytes are control words that MUST be zero when the
+ *              workspace is first used (zero-fill it once after allocating);
+ *              every call leaves them zero.  The rest is scratch whose
+ *              contents on entry are ignored.  Calls that share a workspace
+ *              must not overlap on the GPU.
+ * The one-kernel form needs more than one split and every CTA resident at
+ * once (2 x batch x splits x H/128 CTAs at most the number of SMs); other
+ * calls, and the CUDA-core family, run mla_attn_decode_out's kernels on the
+ * same workspace.  The wkv_b rule of mla_out_proj applies. */
+MLA_API mla_status_t mla_attn_decode_fused(const mla_dims_t* dims, const void* q_abs, const void* q,
+                                           int64_t q_row_stride, const void* kv_cache, const void* pe_cache,
+                                           int64_t kv_rows, const int32_t* cu_seqlens_k, int32_t batch,
+                                           int64_t max_seqlen_k, const void* wkv_b, void* out, void* workspace,
+                                           size_t workspace_bytes, int32_t num_splits, cudaStream_t stream);
+
 /* Size of the device scratch array behind mla_attn_decode_static_scratch. */
 #define MLA_STATIC_SCRATCH_BYTES (32u << 20)
 
