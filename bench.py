@@ -85,16 +85,17 @@ class DecodeBench:
         inputs = self.inputs
 
         def step(k):
-            # the whole hot path through the public calls: absorb, then attention, split merge and
-            # output projection (one kernel where it fits: mla_attn_decode_fused)
-            q, kv, pe, wkv_b = inputs[k]
-            q_abs = mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
-            return mla.attn_decode_fused(d, q_abs, q, kv, pe, cu_k, max_k, wkv_b, bufs["out"], bufs["ws_fused"])
-
-        def step_two_kernels(k):
+            # the whole hot path through the public calls: absorb, then attention (+ split merge
+            # fused into the output projection) in one call
             q, kv, pe, wkv_b = inputs[k]
             q_abs = mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
             return mla.attn_decode_out(d, q_abs, q, kv, pe, cu_k, max_k, wkv_b, bufs["out"], bufs["ws_out"])
+
+        def step_one_kernel(k):
+            # the same step with attention, merge and projection in one kernel (mla_attn_decode_fused)
+            q, kv, pe, wkv_b = inputs[k]
+            q_abs = mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
+            return mla.attn_decode_fused(d, q_abs, q, kv, pe, cu_k, max_k, wkv_b, bufs["out"], bufs["ws_fused"])
 
         def attention_call(k):
             q, kv, pe, _ = inputs[k]
@@ -123,7 +124,7 @@ class DecodeBench:
         # The timed steps replay CUDA graphs captured from the same calls, so host-side launch
         # work does not leave the GPU idle inside the timed region.
         self.g_step = [capture(lambda k=k: step(k)) for k in range(self.copies)]
-        self.g_step2 = [capture(lambda k=k: step_two_kernels(k)) for k in range(self.copies)]
+        self.g_step2 = [capture(lambda k=k: step_one_kernel(k)) for k in range(self.copies)]
         self.g_attn = [capture(lambda k=k: attention_call(k)) for k in range(self.copies)]
         self.g_kern = [capture(lambda k=k: attention_kernel(k)) for k in range(self.copies)]
         for i in range(max(3, warmup)):
@@ -983,7 +984,7 @@ def main():
                              "two events"},
             "repeats": reps,
             "tokens_per_s": world * B / (us_step / 1e6),
-            "step_two_kernel_us": step2_ms / args.steps * 1e3,
+            "step_fused_kernel_us": step2_ms / args.steps * 1e3,
             "attn_kernel_us": mean_kern_ms * 1e3,
             "attn_call_us": mean_attn_ms * 1e3,
             "attn_cache_gbs": achieved_gbs,
@@ -1001,13 +1002,9 @@ def main():
             "kernel_source_hash": kernel_source_hash(),
             "attn_kernel_source_hash": attn_kernel_hash(),
         }
-        # absorb_q, then one kernel for attention, split merge and output projection where it fits
-        # (2 x batch x splits CTAs at most the SMs), else attention + merge-projection
+        # absorb_q + attention + output projection (with the split merge fused in), one launch each
         splits = mla.decode_num_splits(d, B, max(w.seqlens_k), 0)
-        sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        fused = splits >= 2 and 2 * B * (H // 128) * splits <= sms
-        line["gpu_launches"] = args.steps * reps * (2 if fused else 3)
-        line["config"]["fused_step"] = fused
+        line["gpu_launches"] = args.steps * reps * 3
         line["config"]["num_splits"] = splits
         if world == 1 and not args.no_extra_configs:
             del bench

@@ -59,6 +59,20 @@ inline bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Four-dimensional map without swizzle (bf16): dims/strides innermost first, strides in bytes.
+inline bool make_map4(CUtensorMap* m, const void* base, const uint64_t* dims, const uint64_t* strides,
+                      const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[4], s3[3];
+  cuuint32_t b[4], e[4] = {1, 1, 1, 1};
+  for (int i = 0; i < 4; ++i) { d[i] = dims[i]; b[i] = box[i]; }
+  for (int i = 0; i < 3; ++i) s3[i] = strides[i];
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), d, s3, b, e,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline mla_status_t last_launch() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
 // Launch with programmatic stream serialization (pdl = true): the kernel may
@@ -317,7 +331,8 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
 // ws: the attention's split partials, then 256 bytes of control words (zero before the call,
 // left zero after it).  Needs splits >= 2 and no more CTAs (2 per unit) than SMs.
 inline bool fused_fits(int batch, int H, int splits, int sms) {
-  return splits >= 2 && splits <= kMpMaxSplits && (int64_t)batch * (H / 128) * splits * 2 <= sms;
+  return splits >= 2 && splits <= kMergeMaxSplitsFused && (int64_t)batch * (H / 128) * splits * 2 <= sms &&
+         (int64_t)(batch < kMpRows ? batch : kMpRows) * splits <= FusedTailSmem::kMaxRowSplits;
 }
 
 inline mla_status_t decode_fused(const void* q_abs, const void* q, int64_t q_row_stride, const void* kv,
@@ -336,6 +351,16 @@ inline mla_status_t decode_fused(const void* q_abs, const void* q, int64_t q_row
     if (!make_map(&tw, wkv_b, 3, d, stw, b, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   }
   FusedParams f;
+  f.part_rows = batch < kMpRows ? batch : kMpRows;
+  if ((int64_t)f.part_rows * splits > FusedTailSmem::kMaxRowSplits) return MLA_ERR_INVALID_ARG;
+  {
+    // the split partials as [splits][n_q][H][512]: a box is 256 columns of one head for R rows and
+    // every split
+    const uint64_t d[4] = {512, (uint64_t)H, (uint64_t)batch, (uint64_t)splits};
+    const uint64_t st[3] = {1024, (uint64_t)H * 1024, (uint64_t)batch * H * 1024};
+    const uint32_t b[4] = {256, 1, (uint32_t)f.part_rows, (uint32_t)splits};
+    if (!make_map4(&f.tmap_part, L.part_o, d, st, b)) return MLA_ERR_CUDA;
+  }
   f.ctrl = ctrl;
   f.row_tiles = (batch + kMpRows - 1) / kMpRows;
   f.n_items = H * f.row_tiles;

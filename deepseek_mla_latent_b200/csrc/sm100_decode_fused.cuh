@@ -10,7 +10,8 @@
 //      memory (128 KB), so the weight stream overlaps the other units' tails,
 //   3. arrives on a grid-wide counter and waits (bounded) until every CTA has arrived, i.e.
 //      every partial of every row is in memory,
-//   4. merges the split partials of its items (h, 16 query rows) into the B operand and runs the
+//   4. merges the split partials of its items (h, 16 query rows) into the B operand -- each thread
+//      loads its row's (m, l) pairs and its partials in one memory round trip -- and runs the
 //      projection's 32 tcgen05 products (M = 128 value rows, N = 16, K = 512), and stores out,
 //   5. counts itself out; the last CTA out sets both counters back to zero.
 // Items go to score CTAs first (their roles end several microseconds before the value CTAs').
@@ -23,8 +24,13 @@
 namespace mla {
 namespace sm100 {
 
+// Splits the one-kernel step merges from registers (each thread holds all of them in flight).
+constexpr int kMergeMaxSplitsFused = 12;
+
 struct FusedParams {
+  CUtensorMap tmap_part;   // the split partials as [splits][n_q][H][512] bf16, boxes [S][R][1][256]
   uint32_t* ctrl;          // [2] arrivals, departures: zero before a call, zero again after it
+  int part_rows;           // R: rows of an item's partial copy (min(16, n_q))
   int n_items;             // heads * ceil(n_q / 16)
   int row_tiles;           // ceil(n_q / 16)
   const __nv_bfloat16* part_o;
@@ -35,19 +41,23 @@ struct FusedParams {
   __nv_bfloat16* out;      // [n_q, heads, 128]
 };
 
-// Shared memory of the tail: W_v[h] (eight 16 KB K chunks), the B operand, the merge weights
-// and row factors, barriers.  It lies below both roles' barrier areas.
+// Shared memory of the tail: W_v[h] (eight 16 KB K chunks), the item's split partials (two TMA
+// copies of [splits][rows][256 columns] bf16, at most 74 rows x splits in all), the B operand, the
+// hand-off flag, barriers.  It lies below the score role's barrier area; on the value CTA it
+// covers the value role's barriers, which nothing uses once the role has ended (every copy into
+// that CTA and every arrival on its barriers completed before its epilogue).
 struct FusedTailSmem {
   static constexpr int kW = 8 * 128 * 128;
-  static constexpr int kOffB = kW;
-  static constexpr int kOffWt = kOffB + 8 * kMpRows * 128;
-  static constexpr int kOffInv = kOffWt + kMpMaxSplits * kMpRows * 4;
-  static constexpr int kOffFlag = kOffInv + kMpRows * 4;
+  static constexpr int kMaxRowSplits = 74;                  // rows x splits of an item (all CTAs resident)
+  static constexpr int kOffPart = kW;
+  static constexpr int kPartHalf = kMaxRowSplits * 256 * 2;
+  static constexpr int kOffB = kOffPart + 2 * kPartHalf;
+  static constexpr int kOffFlag = kOffB + 8 * kMpRows * 128;
   static constexpr int kOffBars = kOffFlag + 64;
   static constexpr int kEnd = kOffBars + 64;
 };
-static_assert(FusedTailSmem::kEnd <= ValueLayout::kOffBars && FusedTailSmem::kEnd <= ScoreLayout::kOffBars,
-              "the tail's shared memory overlaps a role's barriers");
+static_assert(FusedTailSmem::kEnd <= ScoreLayout::kOffBars && FusedTailSmem::kEnd <= kAttnSmem,
+              "the tail's shared memory overlaps the score role's barriers");
 
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
@@ -61,9 +71,8 @@ __device__ __forceinline__ void fused_tail(uint8_t* smem, uint32_t tmem, const C
   const uint32_t warp = ptx::warp_id(), lane = ptx::lane_id(), rank = ptx::cluster_rank();
   uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + L::kOffBars);   // W_v[h] landed
   uint64_t* done = wfull + 1;                                           // the products finished
+  uint64_t* pfull = wfull + 2;                                          // the item's partials landed
   volatile int* flag = reinterpret_cast<volatile int*>(smem + L::kOffFlag);
-  float* wt = reinterpret_cast<float*>(smem + L::kOffWt);
-  float* inv_s = reinterpret_cast<float*>(smem + L::kOffInv);
   const int total = (int)gridDim.x, pairs = total >> 1;
   const int first = rank == 0 ? (int)(blockIdx.x >> 1) : pairs + (int)(blockIdx.x >> 1);
 
@@ -82,6 +91,7 @@ __device__ __forceinline__ void fused_tail(uint8_t* smem, uint32_t tmem, const C
   if (threadIdx.x == 0) {
     ptx::mbar_init(wfull, 1);
     ptx::mbar_init(done, 1);
+    ptx::mbar_init(pfull, 1);
     ptx::fence_mbar_init();
   }
   __syncthreads();
@@ -124,54 +134,80 @@ __device__ __forceinline__ void fused_tail(uint8_t* smem, uint32_t tmem, const C
       // the previous item's products have read the weights and the B operand
       if (threadIdx.x == 0) load_w(item);
     }
-    // merge weights: warp w handles rows w, w + 10
-    for (int r = (int)warp; r < kMpRows; r += kAttnThreads / 32) {
-      const int64_t n = n0 + r;
-      if (n >= f.n_q) continue;   // warp-uniform
-      const float2* ml = reinterpret_cast<const float2*>(f.part_ml) + n * f.heads + h;
-      float M, inv;
-      const float w_lane = merge_weights(ml, split_stride, f.num_splits, (int)lane, M, inv);
-      for (int s = (int)lane; s < f.num_splits; s += 32) {
-        float w = w_lane;
-        if (s >= 32) {
-          const float2 x = __ldcg(ml + s * split_stride);
-          w = x.x == -INFINITY ? 0.f : exp2f(x.x - M);
-        }
-        wt[s * kMpRows + r] = w;
-      }
-      if (lane == 0) inv_s[r] = inv;
+    // the item's split partials into shared memory (two TMA copies: columns 0..255 and 256..511 of
+    // [splits][rows n0 .. n0 + R)[head h]), while each thread loads its row's (m, l) pairs
+    const int R = f.part_rows;
+    const int part_half = f.num_splits * R * 256 * 2;
+    if (threadIdx.x == 0) {
+      ptx::mbar_arrive_expect_tx(pfull, 2 * part_half);
+      ptx::tma_load_4d(smem + L::kOffPart, &f.tmap_part, pfull, 0, h, n0, 0);
+      ptx::tma_load_4d(smem + L::kOffPart + part_half, &f.tmap_part, pfull, 256, h, n0, 0);
     }
-    __syncthreads();
-    // merge (row r, 16-byte column group g) items into the B operand
-    const int64_t step = split_stride * 512 / 8;
-    constexpr int kInFlight = 16;
-    for (int it = (int)threadIdx.x; it < kMpRows * 64; it += kAttnThreads) {
-      const int r = it >> 6, g = it & 63;
-      uint4 o = make_uint4(0, 0, 0, 0);
-      if (n0 + r < f.n_q) {
-        const uint4* src = reinterpret_cast<const uint4*>(f.part_o + (((int64_t)n0 + r) * f.heads + h) * 512) + g;
-        float a[8];
+    // merge (row r, 16-byte column groups g and g + 32) into the B operand: thread t < 256 takes row
+    // t / 32 of a 8-row pass, with the arithmetic of merge_weights (row sum in the same order) and
+    // of the merge kernels, so the result is the two-kernel path's bit for bit
+    for (int r0 = 0; r0 < kMpRows; r0 += 8) {
+      const int r = r0 + ((int)threadIdx.x >> 5), g0 = (int)threadIdx.x & 31;
+      const bool active = threadIdx.x < 256;
+      const bool valid = active && r < R && n0 + r < f.n_q;
+      float2 ml[kMergeMaxSplitsFused];
+      if (valid) {
+        const float2* mlp = reinterpret_cast<const float2*>(f.part_ml) + ((int64_t)n0 + r) * f.heads + h;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = 0.f;
-        for (int s0 = 0; s0 < f.num_splits; s0 += kInFlight) {
-          uint4 v[kInFlight];
-#pragma unroll
-          for (int s = 0; s < kInFlight; ++s)
-            if (s0 + s < f.num_splits) v[s] = __ldcg(src + (s0 + s) * step);
-#pragma unroll
-          for (int s = 0; s < kInFlight; ++s)
-            if (s0 + s < f.num_splits) {
-              const float w = wt[(s0 + s) * kMpRows + r];
-              if (w != 0.f) merge_acc(a, w, v[s]);
-            }
-        }
-        const float inv = inv_s[r];
-        o.x = ptx::pack_bf16x2(a[0] * inv, a[1] * inv);
-        o.y = ptx::pack_bf16x2(a[2] * inv, a[3] * inv);
-        o.z = ptx::pack_bf16x2(a[4] * inv, a[5] * inv);
-        o.w = ptx::pack_bf16x2(a[6] * inv, a[7] * inv);
+        for (int sp = 0; sp < kMergeMaxSplitsFused; ++sp)
+          if (sp < f.num_splits) ml[sp] = __ldcg(mlp + sp * split_stride);
       }
-      *reinterpret_cast<uint4*>(smem + L::kOffB + (g >> 3) * (kMpRows * 128) + r * 128 + (((g & 7) ^ (r & 7)) << 4)) = o;
+      const bool landed = ptx::mbar_wait(pfull, (uint32_t)(used & 1), kErrTimeoutTmaFull);
+      if (active) {
+        uint4 o[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        if (valid && landed) {
+          float M = -INFINITY;
+#pragma unroll
+          for (int sp = 0; sp < kMergeMaxSplitsFused; ++sp)
+            if (sp < f.num_splits) M = fmaxf(M, ml[sp].x);
+          float a[2][8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[0][i] = a[1][i] = 0.f;
+          // the row sum sum_s w_s l_s added in the order of the warp butterfly merge_weights uses
+          // (xor 16, 8, 4, 2, 1 over lanes = splits; splits past the count hold 0)
+          float x[16];
+#pragma unroll
+          for (int sp = 0; sp < 16; ++sp) x[sp] = 0.f;
+#pragma unroll
+          for (int sp = 0; sp < kMergeMaxSplitsFused; ++sp)
+            if (sp < f.num_splits) {
+              const float w = ml[sp].x == -INFINITY ? 0.f : exp2f(ml[sp].x - M);
+              x[sp] = w * ml[sp].y;
+              if (w != 0.f) {
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                  // column group g = g0 + 32k: columns 8g .. 8g + 7, in copy (8g) / 256
+                  const int c = 8 * (g0 + 32 * k);
+                  const uint8_t* src = smem + L::kOffPart + (c >> 8) * part_half + ((sp * R + r) * 256 + (c & 255)) * 2;
+                  merge_acc(a[k], w, *reinterpret_cast<const uint4*>(src));
+                }
+              }
+            }
+#pragma unroll
+          for (int o2 = 8; o2 >= 1; o2 >>= 1)
+#pragma unroll
+            for (int i = 0; i < o2; ++i) x[i] = x[i] + x[i + o2];
+          const float inv = x[0] > 0.f ? 1.f / x[0] : 0.f;
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            o[k].x = ptx::pack_bf16x2(a[k][0] * inv, a[k][1] * inv);
+            o[k].y = ptx::pack_bf16x2(a[k][2] * inv, a[k][3] * inv);
+            o[k].z = ptx::pack_bf16x2(a[k][4] * inv, a[k][5] * inv);
+            o[k].w = ptx::pack_bf16x2(a[k][6] * inv, a[k][7] * inv);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int g = g0 + 32 * k;
+          *reinterpret_cast<uint4*>(smem + L::kOffB + (g >> 3) * (kMpRows * 128) + r * 128 + (((g & 7) ^ (r & 7)) << 4)) =
+              o[k];
+        }
+      }
     }
     ptx::fence_async_smem();
     __syncthreads();
@@ -234,7 +270,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_kv_score, const __grid_constant__ CUtensorMap tmap_pe,
                         const __grid_constant__ CUtensorMap tmap_qpe, const __grid_constant__ CUtensorMap tmap_kv_value,
                         const __grid_constant__ CUtensorMap tmap_qabs, const __grid_constant__ CUtensorMap tmap_out,
-                        const __grid_constant__ CUtensorMap tmap_w, const AttnParams p, const FusedParams f) {
+                        const __grid_constant__ CUtensorMap tmap_w, const AttnParams p,
+                        const __grid_constant__ FusedParams f) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t tmem = attn_unit<false>(smem, &tmap_kv_score, &tmap_pe, &tmap_qpe, &tmap_kv_value, &tmap_qabs,
                                          &tmap_out, p);
