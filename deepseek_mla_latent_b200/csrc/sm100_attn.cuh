@@ -682,25 +682,15 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
       }
       __syncwarp();
       // The value tiles are the same rows the score CTA is loading: requested together they cost
-      // HBM one read, and the first P V product need not wait for a load after the first P.  They
-      // read only the cache: with p.early_cache the stages free from the start are requested
-      // before the wait for the previous kernel (which writes q_abs), so the first score tile
-      // finds its rows in L2.
-      bool waited = false;
-      if (!p.early_cache) {
-        ptx::griddep_wait();
-        ptx::griddep_launch_dependents();
-        waited = true;
-      }
+      // HBM one read, and the first P V product need not wait for a load after the first P.  This
+      // warp reads only the cache and writes no global memory: with p.early_cache (the previous
+      // kernel does not write the cache) it never waits for the previous kernel, so the first
+      // stages are requested at once and the first score tile finds its rows in L2.
+      if (!p.early_cache) ptx::griddep_wait();
       CacheRows<kPaged> cache;
       cache.init(p, u, lane);
       for (int j = 0; j < nt; ++j) {
         const int st = j % L::kStages;
-        if (j == L::kStages && !waited) {
-          ptx::griddep_wait();
-          ptx::griddep_launch_dependents();
-          waited = true;
-        }
         const bool w = ptx::mbar_wait(&v_empty[st], ((j / L::kStages) & 1) ^ 1, kErrTimeoutStageFree);
         if (!__all_sync(0xffffffffu, w)) break;
         const int key = cache.row(u.j_begin + (int64_t)j * kTileN, u.j_end, lane);
@@ -715,13 +705,6 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
       }
       for (int j = (issued > L::kStages ? issued - L::kStages : 0); j < issued; ++j)
         ptx::mbar_wait(&v_full[j % L::kStages], (j / L::kStages) & 1, kErrTimeoutDrain);
-      if (!waited) {
-        ptx::griddep_wait();
-        ptx::griddep_launch_dependents();
-      }
-    } else {
-      ptx::griddep_wait();
-      ptx::griddep_launch_dependents();
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
