@@ -155,6 +155,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
       }
     }
   }
+  // The rows are visible device-wide before this thread exits: an attention call launched next
+  // starts its cache stream before it waits for this kernel's completion.
+  __threadfence();
 }
 
 }  // namespace append

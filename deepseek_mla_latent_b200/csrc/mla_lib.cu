@@ -497,11 +497,14 @@ mla_status_t mla_attn_prefill_expanded(const mla_dims_t* dims, const void* q, in
                                         batch, n_q_rows, max_seqlen_q, g.H, g.scale, out, device_sm_count(), stream);
 }
 
-mla_status_t mla_attn_paged(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
-                            const int32_t* cu_seqlens_q, int64_t n_q_rows, const int32_t* seqlens_k, int32_t batch,
-                            int64_t max_seqlen_k, const void* kv_cache, const void* pe_cache, int64_t num_pages,
-                            int32_t page_size, const int32_t* block_table, int64_t max_pages_per_seq, void* o_lat,
-                            void* workspace, size_t workspace_bytes, int32_t num_splits, cudaStream_t stream) {
+// mla_attn_paged; early_cache = false when the kernel just before the attention writes the cache
+// (the sparse path's row gather), so the attention must not read it before waiting for that kernel.
+static mla_status_t attn_paged_impl(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
+                                    const int32_t* cu_seqlens_q, int64_t n_q_rows, const int32_t* seqlens_k,
+                                    int32_t batch, int64_t max_seqlen_k, const void* kv_cache, const void* pe_cache,
+                                    int64_t num_pages, int32_t page_size, const int32_t* block_table,
+                                    int64_t max_pages_per_seq, void* o_lat, void* workspace, size_t workspace_bytes,
+                                    int32_t num_splits, cudaStream_t stream, bool early_cache) {
   Geo g;
   if (!dims) return MLA_ERR_INVALID_ARG;
   if (!geo_of(dims, &g)) return MLA_ERR_UNSUPPORTED;
@@ -530,13 +533,24 @@ mla_status_t mla_attn_paged(const mla_dims_t* dims, const void* q_abs, const voi
   if (g.family == 1) {
     if ((q_row_stride * 2) % 16 != 0) return MLA_ERR_INVALID_ARG;
     return mla::sm100::attention(q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, nullptr, batch,
-                                 n_q_rows, g.H, splits, g.scale, o_lat, workspace, stream, true, paged);
+                                 n_q_rows, g.H, splits, g.scale, o_lat, workspace, stream, true, paged,
+                                 /*partials=*/false, early_cache);
   }
   if (g.bf16)
     return simt_attention<mla_bf16>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, nullptr,
                                     batch, n_q_rows, splits, o_lat, workspace, stream, paged);
   return simt_attention<float>(g, q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, cu_seqlens_q, nullptr, batch,
                                n_q_rows, splits, o_lat, workspace, stream, paged);
+}
+
+mla_status_t mla_attn_paged(const mla_dims_t* dims, const void* q_abs, const void* q, int64_t q_row_stride,
+                            const int32_t* cu_seqlens_q, int64_t n_q_rows, const int32_t* seqlens_k, int32_t batch,
+                            int64_t max_seqlen_k, const void* kv_cache, const void* pe_cache, int64_t num_pages,
+                            int32_t page_size, const int32_t* block_table, int64_t max_pages_per_seq, void* o_lat,
+                            void* workspace, size_t workspace_bytes, int32_t num_splits, cudaStream_t stream) {
+  return attn_paged_impl(dims, q_abs, q, q_row_stride, cu_seqlens_q, n_q_rows, seqlens_k, batch, max_seqlen_k,
+                         kv_cache, pe_cache, num_pages, page_size, block_table, max_pages_per_seq, o_lat, workspace,
+                         workspace_bytes, num_splits, stream, /*early_cache=*/true);
 }
 
 size_t mla_sparse_workspace_size(const mla_dims_t* dims, int32_t batch, int32_t max_topk, int32_t num_splits) {
@@ -583,9 +597,9 @@ mla_status_t mla_attn_sparse_decode(const mla_dims_t* dims, const void* q_abs, c
       table);
   if (launch_status() != MLA_OK) return MLA_ERR_CUDA;
   // the paged attention over one page per sequence: block table entry b = page b
-  return mla_attn_paged(dims, q_abs, q, q_row_stride, nullptr, batch, lens, batch, max_topk, kv_sel, pe_sel, batch,
-                        (int32_t)sl.page, table, 1, o_lat, ws + sl.off_attn, sl.total - sl.off_attn, num_splits,
-                        stream);
+  return attn_paged_impl(dims, q_abs, q, q_row_stride, nullptr, batch, lens, batch, max_topk, kv_sel, pe_sel, batch,
+                         (int32_t)sl.page, table, 1, o_lat, ws + sl.off_attn, sl.total - sl.off_attn, num_splits,
+                         stream, /*early_cache=*/false);
 }
 
 mla_status_t mla_expand_kv(const mla_dims_t* dims, const void* kv_c, const void* gamma, float eps,

@@ -156,8 +156,9 @@ inline mla_status_t absorb_q(const void* q, int64_t q_row_stride, const void* wk
   uint32_t box[3] = {xb[0], xb[1], (uint32_t)(n_rows <= 16 ? 16 : n_rows <= 32 ? 32 : n_rows <= 64 ? 64 : n_rows <= 128 ? 128 : 256)};
   if (!make_map(&tw, wkv_b, 2, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   if (!make_map(&tx, q, 3, xd, xs, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-  // the first kernel of a step: an ordinary launch, so the step starts after all earlier work
-  return dispatch_proj<true, 2>(tw, tx, 4, H, n_rows, 2, 0, q_abs, (int64_t)H * 512, 512, stream, false);
+  // the first kernel of a step: its weight copies (wkv_b is never written by the kernels of a step)
+  // start before the wait for the previous kernel, so they overlap the previous layer's tail
+  return dispatch_proj<true, 2>(tw, tx, 4, H, n_rows, 2, 0, q_abs, (int64_t)H * 512, 512, stream, true);
 }
 
 inline mla_status_t out_proj(const void* o_lat, const void* wkv_b, void* out, int64_t n_rows, int H,
@@ -222,7 +223,8 @@ struct AttnLaunch {
 inline mla_status_t prepare_attention(AttnLaunch& L, const void* q_abs, const void* q, int64_t q_row_stride,
                                       const void* kv, const void* pe, int64_t kv_rows, const int32_t* cu_q,
                                       const int32_t* cu_k, int batch, int64_t n_q, int H, int splits, float scale,
-                                      void* o_lat, void* ws, const PagedKv& paged, bool partials) {
+                                      void* o_lat, void* ws, const PagedKv& paged, bool partials,
+                                      bool early_cache = true) {
   CUtensorMap &tkv_s = L.tkv_s, &tpe = L.tpe, &tqpe = L.tqpe, &tkv_v = L.tkv_v, &tqa = L.tqa, &tout = L.tout;
   AttnParams& p = L.p;
   if (paged.table && (paged.page <= 0 || paged.page % kTileN != 0 || !paged.seqlens || paged.stride < 0))
@@ -280,6 +282,7 @@ inline mla_status_t prepare_attention(AttnLaunch& L, const void* q_abs, const vo
   p.head_groups = H / 128;
   p.num_splits = splits;
   p.partials = (splits > 1 || partials) ? 1 : 0;
+  p.early_cache = early_cache ? 1 : 0;
   p.kv_rows = kv_rows;
   p.n_q = n_q;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -309,10 +312,11 @@ inline mla_status_t prepare_attention(AttnLaunch& L, const void* q_abs, const vo
 inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_stride, const void* kv, const void* pe,
                               int64_t kv_rows, const int32_t* cu_q, const int32_t* cu_k, int batch, int64_t n_q,
                               int H, int splits, float scale, void* o_lat, void* ws, cudaStream_t stream,
-                              bool merge = true, const PagedKv& paged = PagedKv{}, bool partials = false) {
+                              bool merge = true, const PagedKv& paged = PagedKv{}, bool partials = false,
+                              bool early_cache = true) {
   AttnLaunch L;
   mla_status_t st = prepare_attention(L, q_abs, q, q_row_stride, kv, pe, kv_rows, cu_q, cu_k, batch, n_q, H, splits,
-                                      scale, o_lat, ws, paged, partials);
+                                      scale, o_lat, ws, paged, partials, early_cache);
   if (st != MLA_OK || L.units == 0) return st;
   const AttnParams& p = L.p;
   auto kern = paged.table ? latent_attn_kernel<true> : latent_attn_kernel<false>;

@@ -132,6 +132,7 @@ struct AttnParams {
   int head_groups;              // heads / 128
   int num_splits;
   int partials;                 // 1: write the split partial form (O relative to m, and (m, l)) even for one split
+  int early_cache;              // 1: the value CTA starts its cache stream before waiting for the previous kernel
   int64_t kv_rows;
   int64_t n_q;
   float scale_log2;             // softmax_scale * log2(e)
@@ -279,6 +280,9 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
 
   if (warp == kProducerWarp) {
     // ============================================================ producer
+    // q comes from the previous kernel
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
     int lat_issued = 0, pe_issued = 0;
     if (ntp > 0) {
       if (ptx::elect_one()) {
@@ -422,6 +426,9 @@ __device__ __forceinline__ void score_role(uint8_t* smem, uint32_t tmem, const U
     __syncwarp();
   } else {
     // ============================================================ softmax
+    // the row sums and the partials' (m, l) are written after the previous kernel has finished
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
     const int g = (int)(warp >> 2);                 // warpgroup: score tiles jj with jj % 2 == g
     const int qd = (int)(warp & 3);                 // TMEM lane quadrant
     const int h = qd * 32 + (int)lane;              // head within the group = TMEM lane
@@ -674,10 +681,14 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
         ptx::prefetch_tmap(tmap_out);
       }
       __syncwarp();
+      // The value tiles are the same rows the score CTA is loading: requested together they cost
+      // HBM one read, and the first P V product need not wait for a load after the first P.  This
+      // warp reads only the cache and writes no global memory: with p.early_cache (the previous
+      // kernel does not write the cache) it never waits for the previous kernel, so the first
+      // stages are requested at once and the first score tile finds its rows in L2.
+      if (!p.early_cache) ptx::griddep_wait();
       CacheRows<kPaged> cache;
       cache.init(p, u, lane);
-      // The value tiles are the same rows the score CTA is loading: requested together they cost
-      // HBM one read, and the first P V product need not wait for a load after the first P.
       for (int j = 0; j < nt; ++j) {
         const int st = j % L::kStages;
         const bool w = ptx::mbar_wait(&v_empty[st], ((j / L::kStages) & 1) ^ 1, kErrTimeoutStageFree);
@@ -762,6 +773,9 @@ __device__ __forceinline__ void value_role(uint8_t* smem, uint32_t tmem, const U
     __syncwarp();
   } else {
     // ============================================================ warps 0-7
+    // the epilogue's output is written after the previous kernel has finished
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
     const int qd = (int)(warp & 3);
     const int h = qd * 32 + (int)lane;
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
@@ -902,9 +916,11 @@ __device__ __forceinline__ uint32_t attn_unit(uint8_t* smem, const CUtensorMap* 
   ptx::cluster_sync();   // the partner's barriers exist before anything remote touches them
   const uint32_t tmem = *tmem_slot;
   // set-up above touches no global memory; inputs may come from the previous kernel
-  ptx::griddep_wait();
-  ptx::griddep_launch_dependents();
-
+  // Set-up above touches no global memory.  q_abs and q_pe may come from the previous kernel in
+  // the stream, and the outputs may still be read by it: the warps that load q or write outputs
+  // wait for it first (griddepcontrol.wait) in their roles; the MMA warps touch no global memory.
+  // The unit's key range (cu_seqlens) is read before that wait, and with p.early_cache the value
+  // CTA's producer starts its cache stream before it.
   UnitRange u = unit_range(p, blockIdx.x >> 1);
   if (!aligned) {
     if (threadIdx.x == 0) raise_error(kErrBadSchedule);

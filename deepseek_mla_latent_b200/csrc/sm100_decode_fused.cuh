@@ -76,6 +76,9 @@ __device__ __forceinline__ void fused_tail(uint8_t* smem, uint32_t tmem, const C
   const int total = (int)gridDim.x, pairs = total >> 1;
   const int first = rank == 0 ? (int)(blockIdx.x >> 1) : pairs + (int)(blockIdx.x >> 1);
 
+  // 0. every thread that touches global memory below has waited for the previous kernel (the
+  // attention roles' MMA warps had no reason to)
+  ptx::griddep_wait();
   // 1. this CTA's outputs are in memory: the partial stores of the value CTA's epilogue warps
   // (each lane 0 issued its own bulk group) have completed, and every thread's generic stores
   // (the score CTA's (m, l) pairs) are ordered before the arrival below

@@ -39,6 +39,20 @@
  *    error word instead of trapping; mla_device_status reports it.
  *  - mla_attn_paged reads the same caches through a block table instead
  *    (pages of page_size tokens); its description gives the addressing.
+ *  - Early start.  The tensor-core kernels (bf16 DeepSeek-V3 shapes) are
+ *    launched with programmatic dependent launch: a kernel may start while
+ *    the kernel before it on the stream is finishing, and reads what that
+ *    kernel may write (q, q_abs, o_lat, ...) and writes its outputs only
+ *    after waiting for it.  Before that wait it reads only inputs that do
+ *    not change from one step of a model to the next or that the step has
+ *    already written: mla_absorb_q and mla_out_proj read wkv_b, and the
+ *    attention calls (decode, decode_out, decode_fused, decode_partials,
+ *    decode_static_scratch, prefill_chunk, paged) read kv_cache, pe_cache,
+ *    cu_seqlens_q, cu_seqlens_k, seqlens_k and block_table.  These must not
+ *    be written by the kernel launched just before the call on the same
+ *    stream, unless that kernel makes its writes visible device-wide before
+ *    it exits (mla_append_latent does: append -> attention is safe).  A
+ *    copy (cudaMemcpyAsync) or an event between the two is always safe.
  */
 #ifndef MLA_B200_H_
 #define MLA_B200_H_
