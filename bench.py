@@ -45,6 +45,7 @@ ROTATE_MIN_BYTES = 2 * L2_BYTES                # traffic between two uses of one
 
 
 MIN_TIMED_MS = 200.0                           # least total length of a repeated timed region
+CHAIN = 8                                      # steps per graph for the chained-step time
 
 
 def decode_algorithmic(w):
@@ -127,8 +128,12 @@ class DecodeBench:
         self.g_step2 = [capture(lambda k=k: step_one_kernel(k)) for k in range(self.copies)]
         self.g_attn = [capture(lambda k=k: attention_call(k)) for k in range(self.copies)]
         self.g_kern = [capture(lambda k=k: attention_kernel(k)) for k in range(self.copies)]
+        # CHAIN steps in one graph, as the attention of consecutive layers of a model: each step's
+        # first kernel may start (programmatic dependent launch) during the previous step's last
+        self.g_chain = [capture(lambda k=k: [step((k + i) % self.copies) for i in range(CHAIN)])
+                        for k in range(self.copies)]
         for i in range(max(3, warmup)):
-            for g in (self.g_step, self.g_step2, self.g_attn, self.g_kern):
+            for g in (self.g_step, self.g_step2, self.g_attn, self.g_kern, self.g_chain):
                 g[i % self.copies].replay()
         mla.device_status()
 
@@ -936,6 +941,8 @@ def main():
 
     total_ms, reps = repeated(bench.g_step)
     step2_ms, _ = repeated(bench.g_step2)
+    chain_ms = statistics.mean(bench.timed(bench.g_chain, max(1, args.steps // CHAIN), world) for _ in range(3))
+    chain_us = chain_ms / (max(1, args.steps // CHAIN) * CHAIN) * 1e3
     # the attention call alone (attention kernel + split merge) and the attention kernel alone
     # (the split partials left in the workspace, mla_attn_decode_partials)
     attn_total_ms, _ = repeated(bench.g_attn)
@@ -985,6 +992,9 @@ def main():
             "repeats": reps,
             "tokens_per_s": world * B / (us_step / 1e6),
             "step_fused_kernel_us": step2_ms / args.steps * 1e3,
+            "step_chained_us": chain_us,
+            "step_chained": f"{CHAIN} steps captured in one graph (consecutive layers): each absorb may start "
+                            "during the previous step's projection",
             "attn_kernel_us": mean_kern_ms * 1e3,
             "attn_call_us": mean_attn_ms * 1e3,
             "attn_cache_gbs": achieved_gbs,
