@@ -442,8 +442,8 @@ inline mla_status_t attention_expanded(const void* q, int64_t q_row_stride, cons
                                        int batch, int64_t n_q, int64_t max_seqlen_q, int H, float scale, void* out,
                                        int sms, cudaStream_t stream) {
   if (n_q >= (1LL << 31) || kv_rows >= (1LL << 31) || max_seqlen_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
-  const int64_t q_tiles = (max_seqlen_q + kFaTile - 1) / kFaTile;
-  const int64_t units = (int64_t)batch * H * q_tiles;
+  const int64_t q_pairs = (max_seqlen_q + 2 * kFaTile - 1) / (2 * kFaTile);
+  const int64_t units = (int64_t)batch * H * q_pairs;
   if (units == 0 || n_q == 0) return MLA_OK;
   CUtensorMap tq, tk, tpe, tv;
   // kv_rows may be 0 (every sequence empty); the maps still need one row
@@ -474,7 +474,7 @@ inline mla_status_t attention_expanded(const void* q, int64_t q_row_stride, cons
   p.cu_k = cu_k;
   p.batch = batch;
   p.heads = H;
-  p.q_tiles = (int)q_tiles;
+  p.q_pairs = (int)q_pairs;
   p.n_units = units;
   p.n_q = n_q;
   p.kv_rows = kv_rows;
