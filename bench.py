@@ -1012,6 +1012,11 @@ def main():
             "kernel_source_hash": kernel_source_hash(),
             "attn_kernel_source_hash": attn_kernel_hash(),
         }
+        if clocks and clocks.get("sm_mhz"):
+            # times x the median sampled SM clock: thousands of SM cycles, comparable across boxes
+            # whose clocks differ
+            line["sm_kcycles"] = {"step": us_step * clocks["sm_mhz"] / 1e3,
+                                  "attn_kernel": mean_kern_ms * 1e3 * clocks["sm_mhz"] / 1e3}
         # absorb_q + attention + output projection (with the split merge fused in), one launch each
         splits = mla.decode_num_splits(d, B, max(w.seqlens_k), 0)
         line["gpu_launches"] = args.steps * reps * 3
