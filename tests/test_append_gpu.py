@@ -76,3 +76,33 @@ def test_append_empty_is_a_no_op():
                       kvc, pec)
     mla.device_status()
     assert int(kvc.abs().sum()) == 0 and int(pec.abs().sum()) == 0
+
+
+def test_append_then_decode_without_a_kernel_between():
+    """The attention reads the cache before it waits for the kernel before it on the stream;
+    mla_append_latent makes its rows visible before it exits, so append -> decode on one stream
+    (no kernel between) attends to the appended rows: against the oracle over the appended cache."""
+    w = wl.make_workload("apd", wl.V3, [1, 1], [300, 700], seed=14)
+    d = mla.dims_from(w.dims)
+    rng = np.random.default_rng(15)
+    C, R = w.dims.kv_lora_rank, w.dims.qk_rope
+    cu = w.cu_seqlens_k
+    slots = np.array([cu[1] - 1, cu[2] - 1], dtype=np.int64)      # the last key of each sequence
+    positions = np.array([299, 699], dtype=np.int32)
+    kv_new = wl.round_to_bf16(rng.normal(size=(2, C)).astype(np.float32) * 2.0)
+    pe_new = wl.round_to_bf16(rng.normal(size=(2, R)).astype(np.float32))
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=torch.bfloat16)
+    q, wkv_b, kv, pe = T(w.q), T(w.wkv_b), T(w.kv), T(w.pe)
+    cu_k = torch.from_numpy(cu).cuda()
+    pos_d, slots_d = torch.from_numpy(positions).cuda(), torch.from_numpy(slots).cuda()
+    kv_new_d, pe_new_d = T(kv_new), T(pe_new)
+    q_abs = mla.absorb_q(d, q, wkv_b)
+    mla.append_latent(d, kv_new_d, pe_new_d, pos_d, slots_d, kv, pe, eps=1e-6)
+    o_lat = mla.attn_decode(d, q_abs, q, kv, pe, cu_k, max(w.seqlens_k))
+    out = mla.out_proj(d, o_lat, wkv_b).float().cpu().numpy().astype(np.float64)
+    mla.device_status()
+    ref_kv, ref_pe = oracle.append_latent(kv_new, pe_new, None, 1e-6, positions, slots, w.kv, w.pe)
+    dd = w.dims
+    ref = oracle.mla_naive(w.q, ref_kv, ref_pe, w.wkv_b, w.cu_seqlens_q, cu, dd.heads, dd.qk_nope, dd.qk_rope,
+                           dd.v_head, dd.scale)
+    assert_close(out, ref, "bf16", "out")
