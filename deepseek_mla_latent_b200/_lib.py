@@ -38,6 +38,8 @@ SIGNATURES = {
     "mla_decode_fused_workspace_size": (_SZ, [_DP, _I32, _I64, _I32]),
     "mla_attn_decode_fused": (_I32, [_DP, _P, _P, _I64, _P, _P, _I64, _P, _I32, _I64, _P, _P, _P, _SZ, _I32, _P]),
     "mla_attn_decode_partials": (_I32, [_DP, _P, _P, _I64, _P, _P, _I64, _P, _I32, _I64, _P, _SZ, _I32, _P]),
+    "mla_merge_partials": (_I32, [_DP, _P, _P, _I32, _I64, _P, _P]),
+    "mla_merge_partials_out": (_I32, [_DP, _P, _P, _I32, _I64, _P, _P, _P]),
     "mla_attn_decode_out": (_I32, [_DP, _P, _P, _I64, _P, _P, _I64, _P, _I32, _I64, _P, _P, _P, _SZ, _I32, _P]),
     "mla_attn_prefill_chunk": (_I32, [_DP, _P, _P, _I64, _P, _P, _I32, _I64, _I64, _I64, _P, _P, _I64, _P, _P, _SZ,
                                       _P]),

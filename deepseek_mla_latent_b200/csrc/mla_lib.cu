@@ -330,6 +330,39 @@ size_t mla_partials_workspace_size(const mla_dims_t* dims, int32_t batch, int64_
   return mla::sm100::workspace_bytes(g.H, batch, splits, /*partials=*/true);
 }
 
+// Shared checks of the two merge calls: tensor-core dims, 1 <= num_splits <= 256, pointers.
+static mla_status_t check_merge_args(const mla_dims_t* dims, const void* part_o, const void* part_ml,
+                                     int32_t num_splits, int64_t n_q_rows, Geo* g) {
+  if (!dims) return MLA_ERR_INVALID_ARG;
+  if (!geo_of(dims, g)) return MLA_ERR_UNSUPPORTED;
+  if (g->family != 1) return MLA_ERR_UNSUPPORTED;
+  if (num_splits < 1 || num_splits > 256 || n_q_rows < 0 || n_q_rows >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  if (n_q_rows > 0 && (!part_o || !part_ml || !aligned16(part_o) || !aligned16(part_ml)))
+    return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+mla_status_t mla_merge_partials(const mla_dims_t* dims, const void* part_o, const void* part_ml,
+                                int32_t num_splits, int64_t n_q_rows, void* o_lat, cudaStream_t stream) {
+  Geo g;
+  const mla_status_t st = check_merge_args(dims, part_o, part_ml, num_splits, n_q_rows, &g);
+  if (st != MLA_OK) return st;
+  if (n_q_rows == 0) return MLA_OK;
+  if (!o_lat || !aligned16(o_lat)) return MLA_ERR_INVALID_ARG;
+  return mla::sm100::merge_partials(part_o, part_ml, num_splits, n_q_rows, g.H, o_lat, stream);
+}
+
+mla_status_t mla_merge_partials_out(const mla_dims_t* dims, const void* part_o, const void* part_ml,
+                                    int32_t num_splits, int64_t n_q_rows, const void* wkv_b, void* out,
+                                    cudaStream_t stream) {
+  Geo g;
+  const mla_status_t st = check_merge_args(dims, part_o, part_ml, num_splits, n_q_rows, &g);
+  if (st != MLA_OK) return st;
+  if (n_q_rows == 0) return MLA_OK;
+  if (!wkv_b || !out || !aligned16(wkv_b) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
+  return mla::sm100::merge_partials_out(part_o, part_ml, num_splits, n_q_rows, g.H, wkv_b, out, stream);
+}
+
 mla_status_t mla_attn_decode_partials(const mla_dims_t* dims, const void* q_abs, const void* q,
                                       int64_t q_row_stride, const void* kv_cache, const void* pe_cache,
                                       int64_t kv_rows, const int32_t* cu_seqlens_k, int32_t batch,

@@ -306,6 +306,18 @@ inline mla_status_t prepare_attention(AttnLaunch& L, const void* q_abs, const vo
   return MLA_OK;
 }
 
+// The split merge alone: o_lat [n_q, H, 512] from split partials (part_o bf16 [splits, n_q, H, 512],
+// part_ml fp32 [splits, n_q, H, 2]).
+inline mla_status_t merge_partials(const void* part_o, const void* part_ml, int splits, int64_t n_q, int H,
+                                   void* o_lat, cudaStream_t stream) {
+  if (splits < 1 || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  const int64_t pairs_per_block = kMergeThreads / 64;   // two warps per (row, head)
+  const int64_t merge_blocks = (n_q * H + pairs_per_block - 1) / pairs_per_block;
+  return launch(true, merge_splits_kernel, dim3((unsigned)merge_blocks), dim3(kMergeThreads), 0, stream,
+                static_cast<const __nv_bfloat16*>(part_o), static_cast<const float*>(part_ml), splits, n_q, H,
+                static_cast<__nv_bfloat16*>(o_lat));
+}
+
 // merge = false (split runs only): leave the partials in the workspace for merge_out_proj
 // instead of merging them into o_lat.  partials = true: write the partial form (also for one
 // split) and never merge; o_lat is not used.
@@ -324,11 +336,7 @@ inline mla_status_t attention(const void* q_abs, const void* q, int64_t q_row_st
   st = launch(true, kern, dim3((unsigned)(2 * L.units)), dim3(kAttnThreads), kAttnSmem, stream, L.tkv_s, L.tpe,
               L.tqpe, L.tkv_v, L.tqa, L.tout, p);
   if (st != MLA_OK || splits <= 1 || !merge || partials) return st;
-  const int64_t pairs_per_block = kMergeThreads / 64;   // two warps per (row, head)
-  const int64_t merge_blocks = (n_q * H + pairs_per_block - 1) / pairs_per_block;
-  return launch(true, merge_splits_kernel, dim3((unsigned)merge_blocks), dim3(kMergeThreads), 0, stream,
-                (const __nv_bfloat16*)L.part_o, (const float*)p.part_ml, splits, n_q, H,
-                static_cast<__nv_bfloat16*>(o_lat));
+  return merge_partials(L.part_o, p.part_ml, splits, n_q, H, o_lat, stream);
 }
 
 // Decode attention, split merge and output projection in one kernel (decode_fused_kernel).
@@ -379,11 +387,11 @@ inline mla_status_t decode_fused(const void* q_abs, const void* q, int64_t q_row
                 L.tkv_s, L.tpe, L.tqpe, L.tkv_v, L.tqa, L.tout, tw, L.p, f);
 }
 
-// The output projection of a split decode with the split merge fused in: out [n_q, H, 128] from the
-// partials an attention(..., merge = false) call left in ws.
-inline mla_status_t merge_out_proj(const void* ws, int splits, int64_t n_q, int H, const void* wkv_b, void* out,
-                                   cudaStream_t stream) {
-  if (splits < 2 || splits > kMpMaxSplits || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+// The output projection with the split merge fused in: out [n_q, H, 128] from split partials
+// (part_o bf16 [splits, n_q, H, 512], part_ml fp32 [splits, n_q, H, 2]).
+inline mla_status_t merge_partials_out(const void* part_o, const void* part_ml, int splits, int64_t n_q, int H,
+                                       const void* wkv_b, void* out, cudaStream_t stream) {
+  if (splits < 1 || splits > kMpMaxSplits || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
   CUtensorMap tw;
   // wkv_b as [8 latent blocks][H * 256 rows][64 columns]: one box is a head's 128 value rows, all
   // eight 64-column K chunks (128 KB, K-major A chunks 16 KB apart)
@@ -392,11 +400,17 @@ inline mla_status_t merge_out_proj(const void* ws, int splits, int64_t n_q, int 
   if (!make_map(&tw, wkv_b, 3, wd, wst, wb, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
   constexpr size_t smem = merge_proj_smem_bytes();
   if (!set_smem(merge_proj_kernel, smem)) return MLA_ERR_CUDA;
-  const auto* part_o = static_cast<const __nv_bfloat16*>(ws);
-  const auto* part_ml = reinterpret_cast<const float*>(static_cast<const char*>(ws) + partial_ml_offset(H, n_q, splits));
   return launch(true, merge_proj_kernel, dim3((unsigned)H, (unsigned)((n_q + kMpRows - 1) / kMpRows)),
-                dim3(kMergeProjThreads), smem, stream, tw, part_o, part_ml, splits, (int)n_q, H,
-                static_cast<__nv_bfloat16*>(out));
+                dim3(kMergeProjThreads), smem, stream, tw, static_cast<const __nv_bfloat16*>(part_o),
+                static_cast<const float*>(part_ml), splits, (int)n_q, H, static_cast<__nv_bfloat16*>(out));
+}
+
+// The same for the partials an attention(..., merge = false) call left in ws.
+inline mla_status_t merge_out_proj(const void* ws, int splits, int64_t n_q, int H, const void* wkv_b, void* out,
+                                   cudaStream_t stream) {
+  if (splits < 2) return MLA_ERR_INVALID_ARG;
+  return merge_partials_out(ws, static_cast<const char*>(ws) + partial_ml_offset(H, n_q, splits), splits, n_q, H,
+                            wkv_b, out, stream);
 }
 
 // Latent KV expansion: K_nope and V [batch, H, seq_len, 128] from kv_c [batch * seq_len, 512].

@@ -154,6 +154,36 @@ def split_partials(d: MlaDims, ws: torch.Tensor, batch: int, splits: int):
     return o, ml
 
 
+def merge_partials(d: MlaDims, part_o: torch.Tensor, part_ml: torch.Tensor, o_lat: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """o_lat [n, H, C] from split partials O [S, n, H, C] (bf16) and (m, l) [S, n, H, 2] (fp32), e.g.
+    several attn_decode_partials results stacked along the split axis (mla_merge_partials)."""
+    S, n, H, C = part_o.shape
+    _need(part_o, "part_o", torch.bfloat16, (S, n, d.num_heads, d.kv_lora_rank))
+    _need(part_ml, "part_ml", torch.float32, (S, n, d.num_heads, 2))
+    if o_lat is None:
+        o_lat = torch.empty((n, H, C), dtype=torch.bfloat16, device=part_o.device)
+    _need(o_lat, "o_lat", torch.bfloat16, (n, H, C))
+    _check(LIB.mla_merge_partials(ctypes.byref(d), _ptr(part_o), _ptr(part_ml), S, n, _ptr(o_lat), _stream(stream)),
+           "mla_merge_partials")
+    return o_lat
+
+
+def merge_partials_out(d: MlaDims, part_o: torch.Tensor, part_ml: torch.Tensor, wkv_b: torch.Tensor,
+                       out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out [n, H, Dv]: the merge of merge_partials fused into the output projection (mla_merge_partials_out)."""
+    S, n, H, C = part_o.shape
+    _need(part_o, "part_o", torch.bfloat16, (S, n, d.num_heads, d.kv_lora_rank))
+    _need(part_ml, "part_ml", torch.float32, (S, n, d.num_heads, 2))
+    _need(wkv_b, "wkv_b", torch.bfloat16, (H * (d.qk_nope_head_dim + d.v_head_dim), C))
+    if out is None:
+        out = torch.empty((n, H, d.v_head_dim), dtype=torch.bfloat16, device=part_o.device)
+    _need(out, "out", torch.bfloat16, (n, H, d.v_head_dim))
+    _check(LIB.mla_merge_partials_out(ctypes.byref(d), _ptr(part_o), _ptr(part_ml), S, n, _ptr(wkv_b), _ptr(out),
+                                      _stream(stream)), "mla_merge_partials_out")
+    return out
+
+
 def decode_out_workspace(d: MlaDims, batch: int, max_seqlen_k: int, num_splits: int = 0,
                          device="cuda") -> torch.Tensor:
     nbytes = int(LIB.mla_decode_out_workspace_size(ctypes.byref(d), batch, max_seqlen_k, num_splits))

@@ -210,6 +210,32 @@ MLA_API mla_status_t mla_attn_decode_partials(const mla_dims_t* dims, const void
                                               int64_t max_seqlen_k, void* workspace, size_t workspace_bytes,
                                               int32_t num_splits, cudaStream_t stream);
 
+/* Merge of split partials into o_lat: o_lat[n, h] = sum_s 2^(m_s - M) O_s /
+ * sum_s 2^(m_s - M) l_s, M = max_s m_s (the log-sum-exp combination of
+ * softmaxes over disjoint key ranges; "Absorb Path Execution", the latent
+ * value einsum summed over the ranges).  The partials are in the form
+ * mla_attn_decode_partials leaves them, and may come from several such calls
+ * over disjoint key ranges of the same query rows, stacked along the split
+ * axis (e.g. the parts of one long sequence held by several GPUs, gathered):
+ *   part_o   [num_splits, n_q_rows, H, C] bf16 (O relative to each split's m)
+ *   part_ml  [num_splits, n_q_rows, H, 2] fp32 (m, l); a split with m = -inf
+ *            (no key) contributes nothing and its O rows are not read.
+ *   o_lat    [n_q_rows, H, C] bf16, written.  A row whose splits all have
+ *            l = 0 gets zeros.
+ * 1 <= num_splits <= 256.  Tensor-core dims (bf16 DeepSeek-V3 shapes) only;
+ * other dims return MLA_ERR_UNSUPPORTED. */
+MLA_API mla_status_t mla_merge_partials(const mla_dims_t* dims, const void* part_o, const void* part_ml,
+                                        int32_t num_splits, int64_t n_q_rows, void* o_lat, cudaStream_t stream);
+
+/* The same merge fused into the output projection (as mla_attn_decode_out
+ * does): out[n, h, :] = o_lat[n, h, :] . W_v[h]^T with o_lat never written.
+ *   wkv_b  [H*(Dn+Dv), C] row-major; out [n_q_rows, H, Dv] bf16, written.
+ * The kernel reads wkv_b before waiting for the previous kernel on the stream
+ * (see "Early start" above). */
+MLA_API mla_status_t mla_merge_partials_out(const mla_dims_t* dims, const void* part_o, const void* part_ml,
+                                            int32_t num_splits, int64_t n_q_rows, const void* wkv_b, void* out,
+                                            cudaStream_t stream);
+
 /* Bytes of workspace mla_attn_decode_fused needs (num_splits as for
  * mla_attn_decode; 0 = automatic). */
 MLA_API size_t mla_decode_fused_workspace_size(const mla_dims_t* dims, int32_t batch, int64_t max_seqlen_k,
