@@ -187,7 +187,12 @@ inline int auto_decode_splits(int batch, int H, int64_t max_seqlen_k, int sms) {
   const int64_t max_tiles = (max_seqlen_k + kTileQ - 1) / kTileQ;
   if (s > max_tiles) s = max_tiles;
   if (s > 256) s = 256;
-  return s < 1 ? 1 : (int)s;
+  if (s < 1) return 1;
+  // splits are whole score tiles: with `per` keys per split the longest sequence fills only
+  // ceil(t / per) of them, and a unit with no key would only hold a CTA pair
+  const int64_t per = ((max_seqlen_k + s - 1) / s + kTileQ - 1) / kTileQ * kTileQ;
+  const int64_t used = (max_seqlen_k + per - 1) / per;
+  return (int)(used < s ? used : s);
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
