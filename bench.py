@@ -192,17 +192,21 @@ def parse_args():
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", type=int, default=1, help="workload index (1 = DeepSeek-V3 decode b8 t4096)")
+    p.add_argument("--workload", type=int, default=None,
+                   help="workload index (default 1 = DeepSeek-V3 decode b8 t4096; 4 for --op prefill, 3 for --op seqpar)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extra-configs", action="store_true",
                    help="skip the ragged, long-context and chunked-prefill workloads in the decode line")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
-    p.add_argument("--op", choices=["decode", "append", "paged", "expand", "prefill", "sparse"], default="decode",
+    p.add_argument("--op", choices=["decode", "append", "paged", "expand", "prefill", "sparse", "seqpar"],
+                   default="decode",
                    help="decode: the decode step (the benchmark); append: the latent-cache append alone; "
                         "paged: the decode attention call over a paged cache beside the packed one; "
                         "expand: the latent KV expansion; prefill: the chunked-prefill step "
                         "(workload 4 unless --workload names another prefill workload); sparse: decode "
-                        "over --topk selected rows per sequence beside the dense call")
+                        "over --topk selected rows per sequence beside the dense call; seqpar: decode with "
+                        "every sequence's cache split over the ranks (NCCL all-gather of the split partials), "
+                        "workload 3 unless --workload names another decode workload")
     p.add_argument("--batch", type=int, default=4, help="sequences per expansion call (--op expand)")
     p.add_argument("--seq-len", type=int, default=1024, help="tokens per sequence (--op expand)")
     p.add_argument("--tokens", type=int, default=65536, help="new tokens per append call (--op append)")
@@ -881,8 +885,87 @@ def run_expand(args, rank, world):
         "gpu_launches": args.steps}), flush=True)
 
 
+def run_seqpar(args, rank, world, local):
+    """Decode with every sequence's cache split along its tokens over the ranks (seqpar): each rank
+    attends to its range in the partial form, the ranks all-gather the partials (NCCL) and merge
+    them fused into the output projection.  Strong scaling: the same sequences at any N.  One JSON
+    line from rank 0 with the time per step (max over ranks) beside the single-GPU decode step."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from deepseek_mla_latent_b200 import mla, seqpar
+    from deepseek_mla_latent_b200 import workloads as wl
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    else:
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        store = dist.TCPStore("127.0.0.1", port, 1, True, timeout=datetime.timedelta(seconds=60))
+        dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = wl.workload(args.workload)
+        if any(s != 1 for s in w.seqlens_q):
+            raise SystemExit("--op seqpar times decode workloads")
+        d = mla.dims_from(w.dims)
+        T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device=dev, dtype=torch.bfloat16)
+        q, kv, pe, wkv_b = T(w.q), T(w.kv), T(w.pe), T(w.wkv_b)
+        B, H = w.batch, w.dims.heads
+        q_abs = mla.absorb_q(d, q, wkv_b)
+        kv_r, pe_r, cu_r, max_r = seqpar.local_cache(kv, pe, w.cu_seqlens_k, world, rank)
+        # splits per rank: enough units to fill this GPU with the rank's range
+        splits = mla.decode_num_splits(d, B, max_r, 0)
+        step = lambda: seqpar.decode_sequence_parallel(d, q_abs, q, kv_r, pe_r, cu_r, max_r, splits, wkv_b=wkv_b)
+        for _ in range(max(3, args.warmup)):
+            out = step()
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            out = step()
+        e1.record()
+        torch.cuda.synchronize()
+        dist.barrier()
+        us, = reduce_max([e0.elapsed_time(e1) / args.steps * 1e3], dev)
+        mla.device_status()
+        # the single-GPU decode step on the whole cache, for the result and the time beside it
+        cu_k = torch.from_numpy(w.cu_seqlens_k).to(dev)
+        dense = mla.attn_decode_out(d, q_abs, q, kv, pe, cu_k, max(w.seqlens_k), wkv_b)
+        for _ in range(3):
+            mla.attn_decode_out(d, q_abs, q, kv, pe, cu_k, max(w.seqlens_k), wkv_b, dense)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            mla.attn_decode_out(d, q_abs, q, kv, pe, cu_k, max(w.seqlens_k), wkv_b, dense)
+        e1.record()
+        torch.cuda.synchronize()
+        dense_us = e0.elapsed_time(e1) / args.steps * 1e3
+        mla.device_status()
+        rel = float((out.float() - dense.float()).abs().max() / dense.float().abs().max())
+        exchange = splits * B * H * (w.dims.kv_lora_rank * 2 + 8)
+        if rank == 0:
+            print(json.dumps({
+                "metric": "MLA sequence-parallel decode us/step (cache split over the GPUs, NCCL exchange)",
+                "value": us, "unit": "us/step", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "higher_is_better": False, "scaling": "strong", "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": w.name, "batch": B, "seq_len_k": int(max(w.seqlens_k)),
+                           "parallelism": f"sequence split over {world} GPU(s)", "splits_per_rank": splits},
+                "single_gpu_decode_us": dense_us, "exchange_bytes_per_rank": exchange,
+                "max_rel_diff_vs_single_gpu": rel,
+                "timing": "eager calls between CUDA events, inputs resident (the cache is read once per step)",
+                "gpu_launches": args.steps * 2}), flush=True)
+    finally:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
+    if args.workload is None:
+        args.workload = {"seqpar": 3, "prefill": 4}.get(args.op, 1)
     rank, world, local = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
@@ -901,6 +984,9 @@ def main():
         return
     if args.op == "sparse":
         run_sparse(args, rank, world)
+        return
+    if args.op == "seqpar":
+        run_seqpar(args, rank, world, local)
         return
 
     import torch
