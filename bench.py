@@ -106,6 +106,19 @@ class DecodeBench:
             q, kv, pe, _ = inputs[k]
             mla.attn_decode_partials(d, bufs["q_abs"], q, kv, pe, cu_k, max_k, bufs["ws"])
 
+        # the absorb kernel alone, and the merge fused into the output projection alone (over the
+        # partials attention_kernel leaves in the workspace)
+        self.splits = mla.decode_num_splits(d, B, max_k, 0)
+        tensor_cores = mla.kernel_family(d) == 1   # the partial form and its merge exist there only
+        part_o, part_ml = mla.split_partials(d, bufs["ws"], B, self.splits) if tensor_cores else (None, None)
+
+        def absorb_kernel(k):
+            q, _, _, wkv_b = inputs[k]
+            mla.absorb_q(d, q, wkv_b, bufs["q_abs"])
+
+        def merge_proj_kernel(k):
+            mla.merge_partials_out(d, part_o, part_ml, inputs[k][3], bufs["out"])
+
         self.step = step
         for i in range(max(3, warmup)):
             step(i % self.copies)
@@ -128,12 +141,15 @@ class DecodeBench:
         self.g_step2 = [capture(lambda k=k: step_one_kernel(k)) for k in range(self.copies)]
         self.g_attn = [capture(lambda k=k: attention_call(k)) for k in range(self.copies)]
         self.g_kern = [capture(lambda k=k: attention_kernel(k)) for k in range(self.copies)]
+        self.g_absorb = [capture(lambda k=k: absorb_kernel(k)) for k in range(self.copies)]
+        self.g_mproj = [capture(lambda k=k: merge_proj_kernel(k)) for k in range(self.copies)] if tensor_cores else None
         # CHAIN steps in one graph, as the attention of consecutive layers of a model: each step's
         # first kernel may start (programmatic dependent launch) during the previous step's last
         self.g_chain = [capture(lambda k=k: [step((k + i) % self.copies) for i in range(CHAIN)])
                         for k in range(self.copies)]
         for i in range(max(3, warmup)):
-            for g in (self.g_step, self.g_step2, self.g_attn, self.g_kern, self.g_chain):
+            for g in (self.g_step, self.g_step2, self.g_attn, self.g_kern, self.g_chain, self.g_absorb,
+                      self.g_mproj or self.g_absorb):
                 g[i % self.copies].replay()
         mla.device_status()
 
@@ -1028,6 +1044,8 @@ def main():
     total_ms, reps = repeated(bench.g_step)
     step2_ms, _ = repeated(bench.g_step2)
     chain_ms = statistics.mean(bench.timed(bench.g_chain, max(1, args.steps // CHAIN), world) for _ in range(3))
+    absorb_ms, _ = repeated(bench.g_absorb)
+    mproj_ms = repeated(bench.g_mproj)[0] if bench.g_mproj else float("nan")
     chain_us = chain_ms / (max(1, args.steps // CHAIN) * CHAIN) * 1e3
     # the attention call alone (attention kernel + split merge) and the attention kernel alone
     # (the split partials left in the workspace, mla_attn_decode_partials)
@@ -1066,6 +1084,9 @@ def main():
         alg_bytes, alg_flop = decode_algorithmic(w)
         attn_s, kern_s = mean_attn_ms / 1e3, mean_kern_ms / 1e3
         achieved_gbs = alg_bytes / kern_s / 1e9
+        Dn, Cl = w.dims.qk_nope, w.dims.kv_lora_rank
+        absorb_bytes = H * Dn * Cl * 2 + B * H * Dn * 2 + B * H * Cl * 2
+        mproj_bytes = H * Dv * Cl * 2 + bench.splits * B * H * (Cl * 2 + 8) + B * H * Dv * 2
         traffic = profiled_traffic(w.name)
         line = {
             "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -1086,6 +1107,13 @@ def main():
             "attn_cache_gbs": achieved_gbs,
             "attn_call_gbs": alg_bytes / attn_s / 1e9,
             "attn_tflops": alg_flop / kern_s / 1e12,
+            # the other two kernels of the step, each alone: the absorb (W_k 16.8 MB + q in, q_abs
+            # out) and the merge fused into the output projection (W_v 16.8 MB + the split partials
+            # in, out out; the partials are L2-resident, as after the attention in the step)
+            "absorb_kernel_us": absorb_ms / args.steps * 1e3,
+            "absorb_gbs": absorb_bytes / (absorb_ms / args.steps * 1e-3) / 1e9,
+            "merge_proj_kernel_us": mproj_ms / args.steps * 1e3,
+            "merge_proj_gbs": mproj_bytes / (mproj_ms / args.steps * 1e-3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": achieved_gbs / hbm, "traffic": traffic, "peak_kind": peak_kind,
                          "kernel": "latent attention kernel alone (CUDA events around its launches)",
