@@ -1112,8 +1112,8 @@ def main():
             # in, out out; the partials are L2-resident, as after the attention in the step)
             "absorb_kernel_us": absorb_ms / args.steps * 1e3,
             "absorb_gbs": absorb_bytes / (absorb_ms / args.steps * 1e-3) / 1e9,
-            "merge_proj_kernel_us": mproj_ms / args.steps * 1e3,
-            "merge_proj_gbs": mproj_bytes / (mproj_ms / args.steps * 1e-3) / 1e9,
+            "merge_proj_kernel_us": mproj_ms / args.steps * 1e3 if bench.g_mproj else None,
+            "merge_proj_gbs": mproj_bytes / (mproj_ms / args.steps * 1e-3) / 1e9 if bench.g_mproj else None,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": achieved_gbs / hbm, "traffic": traffic, "peak_kind": peak_kind,
                          "kernel": "latent attention kernel alone (CUDA events around its launches)",
