@@ -176,8 +176,9 @@ def test_expand_host_checks(lib):
 @pytest.mark.parametrize("max_k", [1, 128, 129, 4096, 131072])
 def test_decode_split_plan(lib, batch, max_k):
     """The automatic split plan of the tensor-core decode: at least one split, never more
-    splits than 128-key score tiles, and with more than one split no more (row, split) units
-    than CTA pairs of a 148-SM GPU (the host has no device here, so the planner uses 148).
+    splits than 128-key score tiles, no split left empty by the tile rounding, and with more
+    than one split no more (row, split) units than CTA pairs of a 148-SM GPU (the host has no
+    device here, so the planner uses 148).
     An explicit split count is used as given, and the workspace grows with the splits."""
     L = lib.LIB
     v3 = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
@@ -186,6 +187,9 @@ def test_decode_split_plan(lib, batch, max_k):
     assert 1 <= s <= max(1, tiles)
     if s > 1:
         assert batch * s <= 74
+    # splits are whole 128-key tiles; the plan leaves none of them empty for the longest sequence
+    per = -(-(-(-max_k // s)) // 128) * 128
+    assert -(-max_k // per) == s
     assert L.mla_decode_num_splits(ctypes.byref(v3), batch, max_k, 5) == 5
     w1 = L.mla_workspace_size(ctypes.byref(v3), batch, batch, max_k, 1)
     w2 = L.mla_workspace_size(ctypes.byref(v3), batch, batch, max_k, 2)
