@@ -318,6 +318,7 @@ inline mla_status_t merge_partials(const void* part_o, const void* part_ml, int 
   if (splits < 1 || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
   const int64_t pairs_per_block = kMergeThreads / 64;   // two warps per (row, head)
   const int64_t merge_blocks = (n_q * H + pairs_per_block - 1) / pairs_per_block;
+  if (merge_blocks >= (1LL << 31)) return MLA_ERR_INVALID_ARG;   // one grid dimension
   return launch(true, merge_splits_kernel, dim3((unsigned)merge_blocks), dim3(kMergeThreads), 0, stream,
                 static_cast<const __nv_bfloat16*>(part_o), static_cast<const float*>(part_ml), splits, n_q, H,
                 static_cast<__nv_bfloat16*>(o_lat));
@@ -397,6 +398,7 @@ inline mla_status_t decode_fused(const void* q_abs, const void* q, int64_t q_row
 inline mla_status_t merge_partials_out(const void* part_o, const void* part_ml, int splits, int64_t n_q, int H,
                                        const void* wkv_b, void* out, cudaStream_t stream) {
   if (splits < 1 || splits > kMpMaxSplits || n_q >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  if ((n_q + kMpRows - 1) / kMpRows > 65535) return MLA_ERR_INVALID_ARG;   // row tiles on the grid's y axis
   CUtensorMap tw;
   // wkv_b as [8 latent blocks][H * 256 rows][64 columns]: one box is a head's 128 value rows, all
   // eight 64-column K chunks (128 KB, K-major A chunks 16 KB apart)

@@ -201,6 +201,29 @@ def test_decode_split_plan(lib, batch, max_k):
     assert out >= w9 + batch * 128 * 512 * 2
 
 
+def test_merge_entry_points_host_checks(lib):
+    """mla_merge_partials(_out): tensor-core dims only, 1..256 splits, aligned non-null pointers,
+    grids that fit; every refusal comes back before any launch (no device here)."""
+    d = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
+    if lib.LIB.mla_kernel_family(ctypes.byref(d)) != 1:
+        pytest.skip("tensor-core family not selected")
+    L, D = lib.LIB, ctypes.byref(d)
+    bad = lib.MLA_ERR_INVALID_ARG
+    for f in (lambda *a: L.mla_merge_partials(D, *a[:4], A, None),
+              lambda *a: L.mla_merge_partials_out(D, *a[:4], A, A, None)):
+        assert f(A, A, 2, 0) == lib.MLA_OK                     # no rows: nothing to do
+        assert f(A, A, 0, 8) == bad and f(A, A, 257, 8) == bad  # split count
+        assert f(None, A, 2, 8) == bad and f(A, None, 2, 8) == bad
+        assert f(A + 8, A, 2, 8) == bad                          # misaligned partials
+        assert f(A, A, 2, -1) == bad and f(A, A, 2, 1 << 31) == bad
+    assert L.mla_merge_partials(D, A, A, 2, 8, None, None) == bad
+    assert L.mla_merge_partials(D, A, A, 2, 1 << 30, A, None) == bad          # grid of (row, head) pairs
+    assert L.mla_merge_partials_out(D, A, A, 2, 8, None, A, None) == bad
+    assert L.mla_merge_partials_out(D, A, A, 2, 1 << 21, A, A, None) == bad   # row tiles on the grid's y axis
+    f32 = lib.make_dims(8, 64, 32, 16, 32, "f32", 0.1)
+    assert L.mla_merge_partials(ctypes.byref(f32), A, A, 2, 8, A, None) == lib.MLA_ERR_UNSUPPORTED
+
+
 def test_partials_entry_point_host_checks(lib):
     """mla_attn_decode_partials exists only on the tensor-core kernels and needs its workspace."""
     d = lib.make_dims(**V3, dtype="bf16", softmax_scale=0.07)
