@@ -608,7 +608,7 @@ mla_status_t mla_attn_sparse_decode(const mla_dims_t* dims, const void* q_abs, c
   SparseLayout sl;
   if (!sparse_layout(g, batch, max_topk, num_splits, &sl)) return MLA_ERR_UNSUPPORTED;
   if (batch == 0) return MLA_OK;
-  if ((int64_t)batch * sl.page >= (1LL << 31)) return MLA_ERR_INVALID_ARG;
+  if ((int64_t)batch * sl.page >= (1LL << 31) || batch > 65535) return MLA_ERR_INVALID_ARG;
   if (!q_abs || !q || !counts || !o_lat || !aligned16(q_abs) || !aligned16(q) || !aligned16(o_lat))
     return MLA_ERR_INVALID_ARG;
   if (max_topk > 0 && (!indices || !kv_cache || !pe_cache || !aligned16(kv_cache) || !aligned16(pe_cache)))

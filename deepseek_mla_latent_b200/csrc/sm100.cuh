@@ -134,6 +134,7 @@ inline mla_status_t dispatch_proj(const CUtensorMap& tw, const CUtensorMap& tx, 
   auto go = [&](auto tile) {
     constexpr int NT = decltype(tile)::value;
     constexpr int STAGES = NT <= 64 ? MAX_STAGES : (MAX_STAGES < 4 ? MAX_STAGES : 4);
+    if ((n_rows + NT - 1) / NT > 65535 || H > 65535) return MLA_ERR_INVALID_ARG;   // grid's y and z axes
     dim3 grid(m_tiles, H, (unsigned)((n_rows + NT - 1) / NT));
     return launch_proj<A_MN, NT, STAGES>(tw, tx, grid, k_chunks, w_row_base, (int)n_rows, out, out_row_stride,
                                          out_head_stride, stream, pdl);

@@ -114,7 +114,8 @@ typedef struct mla_dims {
  *            head h of a row at + h*(Dn+R); only dims 0..Dn-1 are read.
  *   wkv_b    [H*(Dn+Dv), C] row-major.
  *   q_abs    [n_rows, H, C] contiguous, written.
- *   n_rows   >= 0 (0 is a no-op).  q_row_stride >= H*(Dn+R).  */
+ *   n_rows   >= 0 (0 is a no-op).  q_row_stride >= H*(Dn+R).  The tensor-core
+ *            kernels take at most 65535 * 256 rows per call (MLA_ERR_INVALID_ARG above). */
 MLA_API mla_status_t mla_absorb_q(const mla_dims_t* dims, const void* q, int64_t q_row_stride,
                           const void* wkv_b, void* q_abs, int64_t n_rows, cudaStream_t stream);
 
@@ -391,6 +392,7 @@ MLA_API size_t mla_sparse_workspace_size(const mla_dims_t* dims, int32_t batch, 
  *                entry outside [0, kv_rows) reads as a key of zeros and sets
  *                bit 1<<7 of the device error word.
  *   max_topk     host upper bound of the counts; index_stride >= max_topk.
+ *   batch        at most 65535.
  *   q_abs, q, q_row_stride, kv_cache, pe_cache, kv_rows, o_lat [batch, H, C],
  *   num_splits   as for mla_attn_decode.
  *   workspace    at least mla_sparse_workspace_size(dims, batch, max_topk,
@@ -409,6 +411,7 @@ MLA_API mla_status_t mla_attn_sparse_decode(const mla_dims_t* dims, const void* 
 /* Output projection: out[n,h,d] = sum_c o_lat[n,h,c] * wkv_b[h*(Dn+Dv)+Dn+d, c].
  * ("Absorb Path Execution", the last einsum, with the tail rows of wkv_b.)
  *   o_lat [n_rows, H, C] contiguous; out [n_rows, H, Dv] contiguous, written.
+ *   The tensor-core kernel takes at most 65535 * 256 rows per call.
  * The tensor-core kernel may start while the previous kernel on the stream is
  * still finishing (programmatic dependent launch, when that kernel allows it,
  * as this library's attention calls do) and reads wkv_b before waiting for it:
