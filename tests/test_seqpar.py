@@ -104,3 +104,20 @@ def test_gathered_partials_merge_to_attention_over_the_whole_cache():
         p = np.exp(s - s.max(axis=1, keepdims=True))
         ref = (p / p.sum(axis=1, keepdims=True)) @ rows
         np.testing.assert_allclose(got[b], ref, rtol=1e-5, atol=1e-6)
+
+
+def test_local_cache_takes_each_sequences_range_in_order():
+    """local_cache packs rank r's rows of every sequence, in sequence order, with its cu_seqlens
+    and longest range (CPU tensors: the index arithmetic is the same on any device)."""
+    lens = [7, 0, 12, 3]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    kv = torch.arange(cu[-1] * 4, dtype=torch.float32).view(-1, 4)
+    pe = torch.arange(cu[-1] * 2, dtype=torch.float32).view(-1, 2) + 1000
+    world = 3
+    for r in range(world):
+        kv_r, pe_r, cu_r, max_r = seqpar.local_cache(kv, pe, cu, world, r)
+        lo, hi = seqpar.shard_bounds(cu, world, r)
+        rows = np.concatenate([np.arange(a, b) for a, b in zip(lo, hi)])
+        assert torch.equal(kv_r, kv[rows]) and torch.equal(pe_r, pe[rows])
+        assert cu_r.tolist() == [0] + np.cumsum(hi - lo).tolist()
+        assert max_r == int((hi - lo).max())
