@@ -82,6 +82,9 @@ class DecodeBench:
                 "ws": mla.workspace(d, B, B, max_k, 0, device=dev),
                 "ws_out": mla.decode_out_workspace(d, B, max_k, 0, device=dev),
                 "ws_fused": mla.decode_fused_workspace(d, B, max_k, 0, device=dev)}
+        tensor_cores = mla.kernel_family(d) == 1   # the partial form and its merge exist there only
+        # the split partials of the attention kernel alone (also for one split)
+        bufs["ws_part"] = mla.partials_workspace(d, B, max_k, 0, device=dev) if tensor_cores else None
         self.stream = torch.cuda.current_stream()
         inputs = self.inputs
 
@@ -104,13 +107,12 @@ class DecodeBench:
 
         def attention_kernel(k):
             q, kv, pe, _ = inputs[k]
-            mla.attn_decode_partials(d, bufs["q_abs"], q, kv, pe, cu_k, max_k, bufs["ws"])
+            mla.attn_decode_partials(d, bufs["q_abs"], q, kv, pe, cu_k, max_k, bufs["ws_part"])
 
         # the absorb kernel alone, and the merge fused into the output projection alone (over the
         # partials attention_kernel leaves in the workspace)
         self.splits = mla.decode_num_splits(d, B, max_k, 0)
-        tensor_cores = mla.kernel_family(d) == 1   # the partial form and its merge exist there only
-        part_o, part_ml = mla.split_partials(d, bufs["ws"], B, self.splits) if tensor_cores else (None, None)
+        part_o, part_ml = mla.split_partials(d, bufs["ws_part"], B, self.splits) if tensor_cores else (None, None)
 
         def absorb_kernel(k):
             q, _, _, wkv_b = inputs[k]
