@@ -71,3 +71,16 @@ def test_naive_prefill_flop_count_closed_form():
     ex, at = bench.expanded_prefill_flop(w)
     assert ex == 4 * 4096 * 2 * 128 * 256 * 512
     assert at == pairs * 2 * 128 * (128 + 64 + 128)
+
+
+def test_committed_attention_profile_matches_the_sources():
+    """profiles/attn_decode_v3_decode_b8_t4096.md was captured on the current attention-kernel
+    sources (its hash is bench.py's), so the bench line's roofline.traffic is not null; a kernel
+    change without a new capture fails here."""
+    sys.path.insert(0, ROOT)
+    import bench
+    traffic = bench.profiled_traffic("v3_decode_b8_t4096")
+    assert traffic is not None, "attention profile is stale: recapture it on the current sources"
+    # DRAM bytes per launch close to the algorithmic bytes (32768 x 1152 cache + q_abs, q_pe, o_lat)
+    alg = 32768 * 1152 + 8 * 128 * (512 + 64 + 512) * 2
+    assert 0.9 * alg <= traffic <= 1.1 * alg
